@@ -1,0 +1,201 @@
+"""CPU oracle for the block-causal, frame-wise linear-attention scan.
+
+TEST INFRASTRUCTURE ONLY.  This package is a plain, slow, obviously correct
+float64 restatement of what the scan computes.  Only the test suite, the
+smoke check in ``__graft_entry__`` and the CPU-baseline leg of ``bench.py``
+may import it; the CUDA library and its Python binding never do, and share
+no code with it.  The two meet only through the seeded generator in
+``synth``.
+
+Equations (frozen before any kernel was written).  Per batch b and head h,
+frame f = 1..F holds Q_f, K_f, V_f of shape [S, D].  The state is stored
+key-major, M in R^{D_k x D_v}, so that the output is always O_f = Q~_f M_f.
+
+ReLU mode -- SANA-Video talk (ICLR 2026 oral), block KV cache segment: the
+D x D state is updated additively block by block and each block reads the
+cached state of all earlier blocks plus its own contribution; SANA-Video
+guide (lpnh.cn), section "核心机制": each block attends to itself and to
+every earlier block.  phi = max(x, 0):
+    M_f = M_{f-1} + phi(K_f)^T V_f
+    z_f = z_{f-1} + sum_t phi(K_f[t, :])
+    O_f[t, :] = phi(Q_f[t, :]) M_f / (phi(Q_f[t, :]) . z_f + eps)
+
+GDN mode -- SANA-WM digest, method details ("Periodic softmax" and "Spatial
+Explosion" paragraphs) and SANA-WM paper summary (paperlayer), section 3,
+"Hybrid GDN/Softmax Attention": a D x D state is scanned latent frame by
+latent frame, all spatial tokens of a frame enter one update, a decay gate
+and an update gate control forgetting, and keys are scaled by 1/sqrt(D*S):
+    Kh_f = k_scale * K_f
+    M_f  = alpha_f (I - beta_f Kh_f^T Kh_f) M_{f-1} + beta_f Kh_f^T V_f
+    O_f  = Q_f M_f
+Readings where the pages are silent: inclusive causality (frame f reads
+M_f); alpha scales the decayed-and-erased old state but not the write;
+beta scales both erase and write; gates are per (b, h, f); no feature map
+or normaliser in GDN mode; eps = 1e-6 by default in ReLU mode.
+
+Composite form (SANA-WM paper summary, appendix C.1, context-parallel
+training): each frame is affine, M_f = A_f M_{f-1} + B_f with
+A_f = alpha_f (I - beta_f G_f), G_f = Kh_f^T Kh_f, B_f = beta_f Kh_f^T V_f,
+so a frame interval has a transition composite and an input composite, and
+an exclusive prefix over intervals recovers each interval's exact initial
+state.
+
+Array layout: q, k, v, o are [B, H, F, S, D]; alpha, beta are [B, H, F];
+state is [B, H, D, D] (key-major); z is [B, H, D].  Every input is widened
+to float64 first (bf16 and fp32 widen exactly).
+"""
+from __future__ import annotations
+
+from typing import List, Optional, Sequence, Tuple
+
+import numpy as np
+
+__all__ = [
+    "relu_scan", "gdn_scan", "relu_state_step", "gdn_state_step",
+    "gdn_interval_composite", "compose_exclusive_prefix",
+]
+
+
+def _f64(x):
+    return None if x is None else np.asarray(x, dtype=np.float64)
+
+
+def _phi(x: np.ndarray) -> np.ndarray:
+    """ReLU feature map of the SANA-Video linear attention."""
+    return np.maximum(x, 0.0)
+
+
+def _shape(k: np.ndarray) -> Tuple[int, int, int, int, int]:
+    if k.ndim != 5:
+        raise ValueError("expected [B, H, F, S, D]")
+    return k.shape  # type: ignore[return-value]
+
+
+# ----------------------------------------------------------------------------
+# ReLU linear attention with normaliser
+# ----------------------------------------------------------------------------
+def relu_scan(q, k, v, eps: float = 1e-6, state_in=None, z_in=None,
+              want_output: bool = True):
+    """Block-causal ReLU linear attention over latent frames.
+
+    SANA-Video talk, block KV cache segment (state S of fixed shape D x D,
+    added to block by block, cached between blocks) and SANA-Video guide,
+    "核心机制" (each block sees itself and all earlier blocks).
+
+    Returns (o, M_F, z_F); o is None when want_output is False.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, F, S, D = _shape(k)
+    o = np.zeros((B, H, F, S, D)) if want_output else None
+    m_out = np.zeros((B, H, D, D))
+    z_out = np.zeros((B, H, D))
+    m0 = _f64(state_in)
+    z0 = _f64(z_in)
+    for b in range(B):
+        for h in range(H):
+            M = np.zeros((D, D)) if m0 is None else m0[b, h].copy()
+            z = np.zeros(D) if z0 is None else z0[b, h].copy()
+            for f in range(F):
+                pk = _phi(k[b, h, f])                 # [S, D_k]
+                M = M + pk.T @ v[b, h, f]             # additive state update
+                z = z + pk.sum(axis=0)                # normaliser update
+                if want_output:
+                    pq = _phi(q[b, h, f])             # [S, D_k]
+                    num = pq @ M                      # [S, D_v]
+                    den = pq @ z                      # [S]
+                    o[b, h, f] = num / (den + eps)[:, None]
+            m_out[b, h] = M
+            z_out[b, h] = z
+    return o, m_out, z_out
+
+
+def relu_state_step(k, v, state_in=None, z_in=None):
+    """Advance the ReLU cache over finished frames without producing outputs."""
+    _, m, z = relu_scan(k, k, v, 0.0, state_in, z_in, want_output=False)
+    return m, z
+
+
+# ----------------------------------------------------------------------------
+# Frame-wise Gated DeltaNet
+# ----------------------------------------------------------------------------
+def gdn_scan(q, k, v, alpha, beta, k_scale: float, state_in=None,
+             want_output: bool = True):
+    """Frame-wise Gated DeltaNet with key scaling.
+
+    SANA-WM digest, method details, and SANA-WM paper summary, section 3
+    ("Hybrid GDN/Softmax Attention"): one D x D state per head, one update
+    per latent frame that takes in all of the frame's spatial tokens; decay
+    and update gates; keys scaled by 1/sqrt(D*S) (passed as k_scale).
+
+    Each frame is computed in the direct order
+        P = Kh M;  M <- alpha (M - beta Kh^T P) + beta Kh^T V;  O = Q M.
+    Returns (o, M_F); o is None when want_output is False.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    alpha, beta = _f64(alpha), _f64(beta)
+    B, H, F, S, D = _shape(k)
+    o = np.zeros((B, H, F, S, D)) if want_output else None
+    m_out = np.zeros((B, H, D, D))
+    m0 = _f64(state_in)
+    kappa = float(k_scale)
+    for b in range(B):
+        for h in range(H):
+            M = np.zeros((D, D)) if m0 is None else m0[b, h].copy()
+            for f in range(F):
+                a = alpha[b, h, f]
+                bt = beta[b, h, f]
+                kh = kappa * k[b, h, f]               # [S, D_k]
+                P = kh @ M                            # [S, D_v]  read old state
+                M = a * (M - bt * (kh.T @ P)) + bt * (kh.T @ v[b, h, f])
+                if want_output:
+                    o[b, h, f] = q[b, h, f] @ M       # reads the updated state
+            m_out[b, h] = M
+    return o, m_out
+
+
+def gdn_state_step(k, v, alpha, beta, k_scale: float, state_in=None):
+    """Advance the GDN state over finished frames without producing outputs."""
+    _, m = gdn_scan(k, k, v, alpha, beta, k_scale, state_in, want_output=False)
+    return m
+
+
+def gdn_interval_composite(k, v, alpha, beta, k_scale: float):
+    """Transition and input composites of one frame interval for one head.
+
+    SANA-WM paper summary, appendix C.1: a rank owning a frame interval
+    summarises it by a compact transition composite and input composite.
+    For frames j = 1..n of the interval, with A_j = alpha_j (I - beta_j G_j)
+    and B_j = beta_j Kh_j^T V_j:
+        T = A_n ... A_1,    U = sum_j A_n ... A_{j+1} B_j,
+    so that M_end = T M_start + U.
+    k, v: [n, S, D]; alpha, beta: [n].  Returns (T, U), each [D, D].
+    """
+    k, v = _f64(k), _f64(v)
+    alpha, beta = _f64(alpha), _f64(beta)
+    n, S, D = k.shape
+    T = np.eye(D)
+    U = np.zeros((D, D))
+    for j in range(n):
+        kh = float(k_scale) * k[j]
+        A = alpha[j] * (np.eye(D) - beta[j] * (kh.T @ kh))
+        Bj = beta[j] * (kh.T @ v[j])
+        T = A @ T
+        U = A @ U + Bj
+    return T, U
+
+
+def compose_exclusive_prefix(composites: Sequence[Tuple[np.ndarray, np.ndarray]],
+                             m0: Optional[np.ndarray] = None) -> List[np.ndarray]:
+    """Initial state of each interval from the interval composites.
+
+    SANA-WM paper summary, appendix C.1: the gathered composite summaries are
+    combined by an exclusive prefix, giving every interval its exact initial
+    state.  Returns [M_start of interval 0, M_start of interval 1, ...].
+    """
+    D = composites[0][0].shape[0]
+    M = np.zeros((D, D)) if m0 is None else _f64(m0).copy()
+    starts = []
+    for T, U in composites:
+        starts.append(M.copy())
+        M = T @ M + U
+    return starts
