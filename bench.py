@@ -1,0 +1,473 @@
+#!/usr/bin/env python
+"""Throughput of the block-causal, frame-wise linear-attention scan on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference]
+
+One step is one pass of the whole scan (load Q/K/V, per-frame contractions,
+state recurrence, outputs and final state) over one batch of seeded
+synthetic input already resident in HBM.  The default workload is the
+720p, 60 s frame-wise GDN scan (B=1, H=20, D=128, F=181 latent frames of
+22x40 tokens).  Prints one JSON line.
+
+Metric: latent frames per second (B*F per step, all heads), with TFLOP/s
+(algorithmic count) and the fraction of the HBM roofline.  Inputs (>3 GB a
+step) are far larger than the 126 MB L2, so no L2 flush is needed between
+steps.
+
+--impl reference times the CPU oracle on the host cores instead (a bounded
+sample of the same workload each step).  N > 1 (torchrun) runs the
+workload once per rank on its own data, no collective on the data path
+(weak scaling); the reported time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import glob
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+WORKLOADS = {
+    # name: (config index, mode)
+    "gdn_720p_60s": (2, "gdn"),
+    "relu_480p": (1, "relu"),
+    "stream_gdn": (3, "gdn"),
+    "stress_gdn": (4, "gdn"),
+    "stress_relu": (4, "relu"),
+    "tiny_gdn": (0, "gdn"),
+    "tiny_relu": (0, "relu"),
+}
+DEFAULT_WORKLOAD = "gdn_720p_60s"
+METRIC = "latent frames/s and TFLOP/s of block-causal GDN/ReLU scan; % of B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------
+# Algorithmic counts (fixed formulas, whatever the kernels do)
+# ----------------------------------------------------------------------------
+def frame_flops(mode: str, S: int, D: int) -> int:
+    """ReLU: phi(K)^T V and phi(Q) M (2SD^2 each), z and phi(Q) z (2SD each).
+    GDN: Kh^T Kh, Kh^T V, Q M (2SD^2 each) and G M (2D^3)."""
+    if mode == "relu":
+        return 4 * S * D * D + 4 * S * D
+    return 6 * S * D * D + 2 * D ** 3
+
+
+def call_bytes(mode: str, B: int, H: int, F: int, S: int, D: int, elem: int,
+               state_in: bool) -> int:
+    """q, k, v read once and o written once; alpha, beta read once (GDN);
+    the state (and z) written once per (b, h) and read once if given."""
+    per_frame = 4 * S * D * elem + (8 if mode == "gdn" else 0)
+    per_bh = D * D * 4 * (2 if state_in else 1)
+    if mode == "relu":
+        per_bh += D * 4 * (2 if state_in else 1)
+    return B * H * (F * per_frame + per_bh)
+
+
+def step_plan(spec, mode):
+    """List of calls one step makes: (frame offset, frames, state_in?)."""
+    if spec.chunk_frames:
+        C = spec.chunk_frames
+        return [(c * C, C, c > 0) for c in range(spec.F // C)]
+    return [(0, spec.F, False)]
+
+
+def step_counts(spec, mode):
+    elem = spec.elem_bytes
+    byts = sum(call_bytes(mode, spec.B, spec.H, n, spec.S, spec.D, elem, si)
+               for _, n, si in step_plan(spec, mode))
+    flops = spec.B * spec.H * spec.F * frame_flops(mode, spec.S, spec.D)
+    return byts, flops
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "linear_attention_video_frame_b200", "csrc", "*"))):
+        h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(workload: str):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu
+    summary, if it was taken on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p)).get(workload)
+    except Exception:
+        return None
+    if not d or d.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------
+# Clock sampling during the timed region (NVML; read-only)
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report nothing rather than guess
+            self.nv = None
+            self.err = str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.nv:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+
+    def stop(self):
+        if self._thr:
+            self._stop.set()
+            self._thr.join()
+
+    def summary(self):
+        if not self.nv:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml_unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": names, "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------
+# The CPU oracle arm (reported baseline, never the product path)
+# ----------------------------------------------------------------------------
+def oracle_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max(int(i.get("num_threads", 1)) for i in info) if info else 1
+    except Exception:
+        return 1
+
+
+def time_oracle_sample(spec, mode, budget_s: float, max_heads=None):
+    """Run the oracle on whole (b, h) slices of the workload until about
+    budget_s of CPU time has passed; return (equivalent frames/s, sample text)."""
+    import oracle
+    a_all, b_all = synth.gates(spec)
+    pairs = [(b, h) for b in range(spec.B) for h in range(spec.H)]
+    done, t_total = 0, 0.0
+    for b, h in pairs:
+        q, k, v = (synth.slice_values(spec, n, b, h).astype(np.float64)[None, None] for n in "qkv")
+        a = a_all[b:b + 1, h:h + 1]
+        bt = b_all[b:b + 1, h:h + 1]
+        t0 = time.perf_counter()
+        if mode == "relu":
+            oracle.relu_scan(q, k, v, spec.eps)
+        else:
+            oracle.gdn_scan(q, k, v, a, bt, spec.k_scale)
+        t_total += time.perf_counter() - t0
+        done += 1
+        if t_total >= budget_s or (max_heads and done >= max_heads):
+            break
+    frames = spec.B * spec.F * done / (spec.B * spec.H)   # equivalent whole-batch frames
+    sample = (f"oracle on {done} of {spec.B * spec.H} (b,h) slices x all {spec.F} frames of "
+              f"{spec.name} ({mode}); frames/s scaled by slices/(B*H)")
+    return frames / t_total, t_total, sample
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    idx, mode = WORKLOADS[args.workload]
+    spec = synth.config(idx)
+    byts, flops = step_counts(spec, mode)
+    for _ in range(args.warmup):
+        time_oracle_sample(spec, mode, 0.0, max_heads=1)
+    vals, ts = [], 0.0
+    for _ in range(args.steps):
+        v, t, sample = time_oracle_sample(spec, mode, 0.0, max_heads=1)
+        vals.append(v)
+        ts += t
+    value = args.steps / sum(1.0 / v for v in vals)      # frames / total time
+    cores = oracle_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "latent frames/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * ts / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy PCG64)",
+        "config": {"workload": spec.name, "mode": mode, "B": spec.B, "H": spec.H, "F": spec.F,
+                   "S": spec.S, "D": spec.D},
+        "cpu_baseline": {"value": value, "unit": "latent frames/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "latent frames/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------
+# Our arm: the CUDA library through its C ABI
+# ----------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import linear_attention_video_frame_b200 as la
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+
+    idx, mode = WORKLOADS[args.workload]
+    base = synth.config(idx)
+    spec = base.with_(seed=base.seed + 1000 * rank) if rank else base   # own data per rank
+    B, H, F, S, D = spec.B, spec.H, spec.F, spec.S, spec.D
+    tdt = torch.bfloat16 if spec.dtype == "bf16" else torch.float32
+    dtc = la.LA_BF16 if spec.dtype == "bf16" else la.LA_F32
+
+    # ---- inputs resident in HBM (pinned host copies kept for the e2e leg) ----
+    host = {}
+    dev_in = {}
+    for name in ("q", "k", "v"):
+        h = torch.empty((B, H, F, S, D), dtype=tdt, pin_memory=True)
+        hv = h.view(torch.int16) if spec.dtype == "bf16" else h
+
+        def put(b, hh, arr, hv=hv):
+            hv[b, hh].copy_(torch.from_numpy(arr.view(np.int16) if arr.dtype == np.uint16
+                                             else arr))
+
+        synth.for_each_slice(spec, name, put)
+        host[name] = h
+        dev_in[name] = h.to(dev)
+    a, bt = synth.gates(spec)
+    host["alpha"] = torch.from_numpy(a).pin_memory()
+    host["beta"] = torch.from_numpy(bt).pin_memory()
+    dev_in["alpha"] = host["alpha"].to(dev)
+    dev_in["beta"] = host["beta"].to(dev)
+    o = torch.empty_like(dev_in["q"])
+    state = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    z = torch.empty((B, H, D), dtype=torch.float32, device=dev)
+    plan = step_plan(spec, mode)
+    ws = la.workspace_for(la.LA_MODE_GDN if mode == "gdn" else la.LA_MODE_RELU,
+                          B, H, max(n for _, n, _ in plan), S, D, dev)
+    views = []
+    for f0, n, si in plan:
+        if len(plan) == 1:
+            views.append((dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"],
+                          dev_in["beta"], o, si))
+        else:   # chunked streaming: contiguous per-chunk copies, made once
+            sl = slice(f0, f0 + n)
+            views.append(tuple(dev_in[x][:, :, sl].contiguous()
+                               for x in ("q", "k", "v", "alpha", "beta")) +
+                         (torch.empty((B, H, n, S, D), dtype=tdt, device=dev), si))
+    stream = torch.cuda.current_stream()
+
+    def one_step():
+        for (q, k, v, al, be, oo, si) in views:
+            if mode == "gdn":
+                la.la_scan_gdn(q, k, v, al, be, spec.k_scale, o=oo,
+                               state_in=state if si else None, state_out=state,
+                               workspace=ws, stream=stream)
+            else:
+                la.la_scan_relu(q, k, v, o=oo, state_in=state if si else None,
+                                z_in=z if si else None, state_out=state, z_out=z,
+                                eps=spec.eps, workspace=ws, stream=stream)
+
+    path, kernels_per_call = la.la_plan(la.LA_MODE_GDN if mode == "gdn" else la.LA_MODE_RELU,
+                                        dtc, B, H, plan[0][1], S, D)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- warm-up ----
+    for _ in range(max(args.warmup, 0)):
+        one_step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: exactly K steps ----
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0.record(stream)
+    for i in range(K):
+        evs[i][0].record(stream)
+        one_step()
+        evs[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks.stop()
+    barrier()
+    t_local = t0.elapsed_time(t1) / 1e3
+    call_ms = [s.elapsed_time(e) / len(plan) for s, e in evs]
+    t_max = t_local
+    if world > 1:
+        tt = torch.tensor([t_local], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_max = float(tt.item())
+
+    byts, flops = step_counts(spec, mode)
+    frames_all = B * F * K * world
+    value = frames_all / t_max
+    ms_per_step = 1e3 * t_max / K
+    tflops = flops * K * world / t_max / 1e12
+
+    # ---- e2e: host buffers, H2D of inputs and D2H of the output inside the timed region ----
+    Ke = max(3, min(K, 10))
+    o_host = torch.empty_like(host["q"], pin_memory=True)
+    h2d = sum(host[x].numel() * host[x].element_size() for x in ("q", "k", "v", "alpha", "beta"))
+    d2h = o_host.numel() * o_host.element_size()
+
+    def e2e_step():
+        for x in ("q", "k", "v", "alpha", "beta"):
+            dev_in[x].copy_(host[x], non_blocking=True)
+        if len(views) > 1:   # chunked: re-slice from the freshly copied tensors
+            for j, (f0, n, si) in enumerate(plan):
+                sl = slice(f0, f0 + n)
+                for i, x in enumerate(("q", "k", "v", "alpha", "beta")):
+                    views[j][i].copy_(dev_in[x][:, :, sl])
+        one_step()
+        if len(views) > 1:
+            o.copy_(torch.cat([vw[5] for vw in views], dim=2))
+        o_host.copy_(o, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(Ke):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    te = e0.elapsed_time(e1) / 1e3
+    if world > 1:
+        tt = torch.tensor([te], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        te = float(tt.item())
+    e2e_value = B * F * Ke * world / te
+    status = la.la_query_device_status(ws)
+
+    # ---- roofline of the dominant kernel ----
+    peaks, peak_src = load_peaks()
+    kern_s = statistics.mean(call_ms) / 1e3
+    per_call_bytes = byts / len(plan)
+    achieved = per_call_bytes / kern_s / 1e9
+    traffic = traffic_record(args.workload)
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                "peak_source": f"{peak_src} (hbm_gbs, STREAM-style copy)",
+                "kernel": path, "kernel_ms": kern_s * 1e3,
+                "alg_bytes_per_launch": per_call_bytes,
+                "tensor_tflops_achieved": flops / len(plan) / kern_s / 1e12,
+                "tensor_frac_of_bf16_peak": flops / len(plan) / kern_s / 1e12 /
+                peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, t, sample = time_oracle_sample(base, mode, args.cpu_budget)
+        cpu = {"value": v, "unit": "latent frames/s", "cores": oracle_threads(),
+               "kind": "oracle", "sample": sample, "seconds": t}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "latent frames/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if spec.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded numpy PCG64, bf16 round-to-nearest-even)",
+        "config": {"workload": base.name, "mode": mode, "B": B, "H": H, "F": F, "S": S, "D": D,
+                   "calls_per_step": len(plan), "global_batch": B * world,
+                   "l2": "inputs larger than L2 (no flush)",
+                   "parallelism": f"replicas x{world} (no data-path collective)"},
+        "tflops": tflops,
+        "gpu_launches": kernels_per_call * len(plan) * K,
+        "kernel_path": path,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "latent frames/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": Ke},
+        "clocks": clocks.summary(),
+        "device_status": la.la_status_string(status),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-budget", type=float, default=10.0,
+                    help="seconds of oracle work for the cpu_baseline field")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,163 @@
+/*
+ * la_scan.h -- C ABI of the block-causal, frame-wise linear-attention scan
+ * (SANA-Video ReLU linear attention and SANA-WM frame-wise Gated DeltaNet)
+ * for NVIDIA B200 (sm_100a).
+ *
+ * Equations (per batch item b and head h; frame f = 1..F holds the [S, D]
+ * token matrices Q_f, K_f, V_f; the state is stored key-major, M[dk][dv]):
+ *
+ *   ReLU mode  (SANA-Video talk, ICLR 2026 oral, block KV cache segment;
+ *               SANA-Video guide, lpnh.cn, section "核心机制"):
+ *     M_f = M_{f-1} + phi(K_f)^T V_f,     z_f = z_{f-1} + sum_t phi(K_f[t,:])
+ *     O_f[t,:] = phi(Q_f[t,:]) M_f / (phi(Q_f[t,:]) . z_f + eps),  phi = max(x,0)
+ *
+ *   GDN mode   (SANA-WM paper summary, paperlayer, section 3 "Hybrid
+ *               GDN/Softmax Attention"; SANA-WM digest, method details,
+ *               "Spatial Explosion" paragraph for the key scale):
+ *     Kh_f = k_scale * K_f
+ *     M_f  = alpha_f (I - beta_f Kh_f^T Kh_f) M_{f-1} + beta_f Kh_f^T V_f
+ *     O_f  = Q_f M_f
+ *
+ * Causality is inclusive: frame f reads the state after its own update.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout.      q, k, v, o: [B, H, F, S, D] contiguous, D fastest.
+ *              alpha, beta: [B, H, F] float32.
+ *              state_in / state_out: [B, H, D, D] float32, key-major
+ *              (element [b][h][dk][dv]).  z_in / z_out: [B, H, D] float32.
+ * Dtype.       q, k, v, o share one dtype, LA_F32 or LA_BF16 (bf16 outputs
+ *              are rounded to nearest even).  The state, the normaliser and
+ *              all accumulation are float32.
+ * Memory.      Every pointer is a device pointer of the current device (or
+ *              managed memory), 16-byte aligned.  The caller owns all
+ *              buffers, including the workspace; the library never
+ *              allocates, frees or synchronises (except
+ *              la_query_device_status, which synchronises on purpose).
+ * Asynchrony.  Work is enqueued on `stream`; argument errors are returned
+ *              before anything is enqueued; a failed launch returns
+ *              LA_ERR_CUDA.  Device-side waits are bounded: a wait that
+ *              gives up records LA_ERR_TIMEOUT in the workspace, which
+ *              la_query_device_status reports.
+ * Aliasing.    state_in == state_out (and z_in == z_out) is allowed (in
+ *              place).  o must not overlap q, k or v.
+ * NULL state.  state_in == NULL (z_in == NULL) means a zero initial state;
+ *              state_out == NULL (z_out == NULL) means "do not write".
+ * Shapes.      B >= 1, H >= 1, F >= 0, S >= 1; D a multiple of 16 in
+ *              [16, 256], else LA_ERR_UNSUPPORTED.  F == 0 writes state_in
+ *              (or zeros) to state_out and touches nothing else.
+ * Workspace.   At least la_workspace_size(mode, B, H, F, S, D) bytes of
+ *              device memory, 256-byte aligned, private to the call while
+ *              it runs (two calls in flight need two workspaces).
+ * Threads.     Thread-safe when concurrent calls use distinct workspaces.
+ */
+#ifndef LA_SCAN_H
+#define LA_SCAN_H
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define LA_API __attribute__((visibility("default")))
+#else
+#define LA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum la_status {
+    LA_OK = 0,
+    LA_ERR_INVALID_ARG = 1,   /* NULL/misaligned/overlapping pointer, bad size, small workspace */
+    LA_ERR_UNSUPPORTED = 2,   /* D not a multiple of 16 in [16, 256], or no sm_100 device      */
+    LA_ERR_CUDA = 3,          /* a CUDA runtime call or kernel launch failed                   */
+    LA_ERR_TIMEOUT = 4        /* a bounded device-side wait gave up (see la_query_device_status) */
+} la_status;
+
+typedef enum la_dtype { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
+typedef enum la_mode { LA_MODE_RELU = 0, LA_MODE_GDN = 1 } la_mode;
+
+/*
+ * Block-causal ReLU linear attention with normaliser over latent frames.
+ * Source: SANA-Video talk (ICLR 2026 oral), block KV cache segment -- the
+ * D x D state is updated additively, block by block, and each block reads
+ * the cached state of the earlier blocks plus its own contribution;
+ * SANA-Video guide (lpnh.cn), section "核心机制".
+ *
+ * q, k, v     in : [B,H,F,S,D] of dtype dt.
+ * o           out: [B,H,F,S,D] of dtype dt.
+ * state_in    in : [B,H,D,D] f32 or NULL (zeros).   z_in  in : [B,H,D] f32 or NULL.
+ * state_out   out: [B,H,D,D] f32 or NULL.           z_out out: [B,H,D] f32 or NULL.
+ * eps         finite, >= 0; added to the denominator (1e-6 is the usual value).
+ */
+LA_API la_status la_scan_relu(const void* q, const void* k, const void* v, void* o, la_dtype dt,
+                       const float* state_in, const float* z_in,
+                       float* state_out, float* z_out,
+                       int B, int H, int F, int S, int D, float eps,
+                       void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Frame-wise Gated DeltaNet with key scaling.
+ * Source: SANA-WM paper summary (paperlayer), section 3 "Hybrid GDN/Softmax
+ * Attention" -- a D x D recurrent state is kept while each latent frame's
+ * spatial tokens are processed together; a decay gate and an update gate
+ * control forgetting; SANA-WM digest, method details, "Spatial Explosion"
+ * paragraph -- keys are scaled by 1/sqrt(D*S) so that the transition's
+ * spectral norm stays at most 1.
+ *
+ * alpha, beta in : [B,H,F] f32 (decay and update gate of each frame).
+ * k_scale        : the key scale, usually 1/sqrt(D*S); applied inside the
+ *                  scan in f32 (it is not folded into bf16 keys).
+ * state_in/out   : [B,H,D,D] f32, key-major; NULL as described above.
+ */
+LA_API la_status la_scan_gdn(const void* q, const void* k, const void* v, void* o, la_dtype dt,
+                      const float* alpha, const float* beta, float k_scale,
+                      const float* state_in, float* state_out,
+                      int B, int H, int F, int S, int D,
+                      void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Advance the cached state over finished frames without producing outputs:
+ * the scan above minus Q and O.  Source: SANA-Video talk, block KV cache
+ * segment -- after a block is final its contribution is added to the cache
+ * that the next block reads; SANA-WM paper summary, section 3,
+ * "Chunk-causal deployment" -- autoregressive rollout carries the recurrent
+ * state from chunk to chunk.
+ *
+ * mode LA_MODE_RELU uses (state, z) and ignores alpha, beta, k_scale;
+ * mode LA_MODE_GDN uses (state) and ignores z_in / z_out.
+ */
+LA_API la_status la_state_step(la_mode mode, const void* k, const void* v, la_dtype dt,
+                        const float* alpha, const float* beta, float k_scale,
+                        const float* state_in, const float* z_in,
+                        float* state_out, float* z_out,
+                        int B, int H, int F, int S, int D,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Workspace bytes a call of this mode and shape needs (either dtype).
+ * Returns 0 for an unsupported shape.  The library has no counterpart in
+ * the pages; it exists because the library never allocates. */
+LA_API size_t la_workspace_size(la_mode mode, int B, int H, int F, int S, int D);
+
+/* Synchronise `stream`, then report the device-side status that the most
+ * recent call using `workspace` recorded: LA_OK, or LA_ERR_TIMEOUT when a
+ * bounded inter-block wait gave up (its outputs are then not valid).
+ * Returns LA_ERR_CUDA if the synchronisation itself fails. */
+LA_API la_status la_query_device_status(void* workspace, cudaStream_t stream);
+
+/* How a call of this mode, dtype and shape runs: stores the number of
+ * kernels one call launches in *kernels (if not NULL) and returns the name
+ * of the kernel path ("tcgen05" or "simt_f32"); NULL for an unsupported
+ * shape.  No counterpart in the pages: it lets a caller check which
+ * kernels its calls use. */
+LA_API const char* la_plan(la_mode mode, la_dtype dt, int B, int H, int F, int S, int D,
+                           int* kernels);
+
+/* Static, human-readable name of a status code. */
+LA_API const char* la_status_string(la_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LA_SCAN_H */

@@ -1,0 +1,189 @@
+"""Python binding of the ``la_scan`` C ABI (include/la_scan.h).
+
+Argument marshalling only: every step of the scan runs in the CUDA kernels of
+``liblavf.so``.  PyTorch supplies device memory and streams.  There is no CPU
+fallback: importing this package fails if the library is missing, and every
+call raises ``LaScanError`` on a non-zero status.
+
+The functions keep the C names.  Tensors follow the C layouts:
+q, k, v, o ``[B, H, F, S, D]`` (bfloat16 or float32, contiguous); alpha, beta
+``[B, H, F]`` float32; state ``[B, H, D, D]`` float32 key-major; z
+``[B, H, D]`` float32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "LA_OK", "LA_ERR_INVALID_ARG", "LA_ERR_UNSUPPORTED", "LA_ERR_CUDA", "LA_ERR_TIMEOUT",
+    "LA_F32", "LA_BF16", "LA_MODE_RELU", "LA_MODE_GDN", "LaScanError", "lib", "LIB_PATH",
+    "la_scan_relu", "la_scan_gdn", "la_state_step", "la_workspace_size",
+    "la_query_device_status", "la_status_string", "la_plan", "workspace_for",
+]
+
+LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CUDA, LA_ERR_TIMEOUT = 0, 1, 2, 3, 4
+LA_F32, LA_BF16 = 0, 1
+LA_MODE_RELU, LA_MODE_GDN = 0, 1
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblavf.so")
+
+
+class LaScanError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {la_status_string(status)} ({status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing; build it with "
+            "`python linear_attention_video_frame_b200/build.py` (there is no fallback)")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    L.la_scan_relu.argtypes = [P, P, P, P, I, P, P, P, P, I, I, I, I, I, F, P, Z, P]
+    L.la_scan_relu.restype = I
+    L.la_scan_gdn.argtypes = [P, P, P, P, I, P, P, F, P, P, I, I, I, I, I, P, Z, P]
+    L.la_scan_gdn.restype = I
+    L.la_state_step.argtypes = [I, P, P, I, P, P, F, P, P, P, P, I, I, I, I, I, P, Z, P]
+    L.la_state_step.restype = I
+    L.la_workspace_size.argtypes = [I, I, I, I, I, I]
+    L.la_workspace_size.restype = Z
+    L.la_query_device_status.argtypes = [P, P]
+    L.la_query_device_status.restype = I
+    L.la_plan.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(ctypes.c_int)]
+    L.la_plan.restype = ctypes.c_char_p
+    L.la_status_string.argtypes = [I]
+    L.la_status_string.restype = ctypes.c_char_p
+    return L
+
+
+lib = _load()
+
+
+def la_status_string(s: int) -> str:
+    return lib.la_status_string(int(s)).decode()
+
+
+def la_plan(mode: int, dt: int, B: int, H: int, F: int, S: int, D: int):
+    """(path name, kernels per call) of a call of this shape; (None, 0) if unsupported."""
+    n = ctypes.c_int(0)
+    name = lib.la_plan(mode, dt, B, H, F, S, D, ctypes.byref(n))
+    return (name.decode() if name else None), int(n.value)
+
+
+def la_workspace_size(mode: int, B: int, H: int, F: int, S: int, D: int) -> int:
+    return int(lib.la_workspace_size(mode, B, H, F, S, D))
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return LA_BF16
+    if t.dtype == torch.float32:
+        return LA_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _check(t: Optional[torch.Tensor], name: str, shape=None, dtype=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+
+
+def workspace_for(mode: int, B: int, H: int, F: int, S: int, D: int, device=None) -> torch.Tensor:
+    """A caller-owned workspace tensor of the size the library asks for."""
+    n = la_workspace_size(mode, B, H, F, S, D)
+    if n == 0:
+        raise LaScanError(LA_ERR_UNSUPPORTED, "la_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def _raise(st: int, where: str):
+    if st != LA_OK:
+        raise LaScanError(st, where)
+
+
+def la_scan_relu(q, k, v, o=None, state_in=None, z_in=None, state_out=None, z_out=None,
+                 eps: float = 1e-6, workspace=None, stream=None):
+    B, H, F, S, D = k.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _check(t, n, (B, H, F, S, D), k.dtype)
+    for t, n in ((state_in, "state_in"), (state_out, "state_out")):
+        _check(t, n, (B, H, D, D), torch.float32)
+    for t, n in ((z_in, "z_in"), (z_out, "z_out")):
+        _check(t, n, (B, H, D), torch.float32)
+    if o is None:
+        o = torch.empty_like(q)
+    if workspace is None:
+        workspace = workspace_for(LA_MODE_RELU, B, H, F, S, D, q.device)
+    st = lib.la_scan_relu(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _dtype_code(k), _ptr(state_in),
+                          _ptr(z_in), _ptr(state_out), _ptr(z_out), B, H, F, S, D, float(eps),
+                          _ptr(workspace), workspace.numel(), _stream(stream))
+    _raise(st, "la_scan_relu")
+    return o
+
+
+def la_scan_gdn(q, k, v, alpha, beta, k_scale: float, o=None, state_in=None, state_out=None,
+                workspace=None, stream=None):
+    B, H, F, S, D = k.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _check(t, n, (B, H, F, S, D), k.dtype)
+    for t, n in ((alpha, "alpha"), (beta, "beta")):
+        _check(t, n, (B, H, F), torch.float32)
+    for t, n in ((state_in, "state_in"), (state_out, "state_out")):
+        _check(t, n, (B, H, D, D), torch.float32)
+    if o is None:
+        o = torch.empty_like(q)
+    if workspace is None:
+        workspace = workspace_for(LA_MODE_GDN, B, H, F, S, D, q.device)
+    st = lib.la_scan_gdn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _dtype_code(k), _ptr(alpha),
+                         _ptr(beta), float(k_scale), _ptr(state_in), _ptr(state_out),
+                         B, H, F, S, D, _ptr(workspace), workspace.numel(), _stream(stream))
+    _raise(st, "la_scan_gdn")
+    return o
+
+
+def la_state_step(mode: int, k, v, alpha=None, beta=None, k_scale: float = 1.0,
+                  state_in=None, z_in=None, state_out=None, z_out=None, workspace=None,
+                  stream=None):
+    B, H, F, S, D = k.shape
+    _check(k, "k", (B, H, F, S, D))
+    _check(v, "v", (B, H, F, S, D), k.dtype)
+    for t, n in ((alpha, "alpha"), (beta, "beta")):
+        _check(t, n, (B, H, F), torch.float32)
+    for t, n in ((state_in, "state_in"), (state_out, "state_out")):
+        _check(t, n, (B, H, D, D), torch.float32)
+    for t, n in ((z_in, "z_in"), (z_out, "z_out")):
+        _check(t, n, (B, H, D), torch.float32)
+    if workspace is None:
+        workspace = workspace_for(mode, B, H, F, S, D, k.device)
+    st = lib.la_state_step(int(mode), _ptr(k), _ptr(v), _dtype_code(k), _ptr(alpha), _ptr(beta),
+                           float(k_scale), _ptr(state_in), _ptr(z_in), _ptr(state_out),
+                           _ptr(z_out), B, H, F, S, D, _ptr(workspace), workspace.numel(),
+                           _stream(stream))
+    _raise(st, "la_state_step")
+
+
+def la_query_device_status(workspace, stream=None) -> int:
+    return int(lib.la_query_device_status(_ptr(workspace), _stream(stream)))

@@ -1,0 +1,62 @@
+// Shared definitions of the scan library (host and device).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "la_scan.h"
+
+namespace la {
+
+// Workspace header: the first 256 bytes of every workspace.
+struct WsHeader {
+    unsigned int status;        // 0 = ok, LA_ERR_TIMEOUT when a bounded wait gave up
+    unsigned int where;         // which wait gave up (diagnostic)
+    unsigned int ticket;        // dynamic work counter of persistent kernels
+    unsigned int done;          // blocks finished (persistent kernels)
+    unsigned int pad[60];
+};
+static_assert(sizeof(WsHeader) == 256, "header is 256 bytes");
+
+constexpr size_t kWsHeaderBytes = 256;
+
+__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Arguments shared by every scan launcher.
+struct ScanArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    void* o;                 // NULL for a state step
+    const float* alpha;      // GDN only
+    const float* beta;       // GDN only
+    const float* state_in;   // may be NULL
+    const float* z_in;       // ReLU only, may be NULL
+    float* state_out;        // may be NULL
+    float* z_out;            // ReLU only, may be NULL
+    float k_scale;
+    float eps;
+    int B, H, F, S, D;
+    int mode;                // LA_MODE_RELU / LA_MODE_GDN
+    int bf16;                // 1 if q,k,v,o are bf16
+    void* ws;
+    size_t ws_bytes;
+};
+
+// Element access for the two storage types.
+__device__ __forceinline__ float load_elem(const void* p, size_t i, int bf16) {
+    if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
+    return reinterpret_cast<const float*>(p)[i];
+}
+__device__ __forceinline__ void store_elem(void* p, size_t i, float x, int bf16) {
+    if (bf16) reinterpret_cast<__nv_bfloat16*>(p)[i] = __float2bfloat16_rn(x);
+    else reinterpret_cast<float*>(p)[i] = x;
+}
+
+// Launchers (host side), each returns cudaGetLastError() of its launches.
+cudaError_t launch_simt(const ScanArgs& a, cudaStream_t st);
+size_t simt_workspace_bytes(const ScanArgs& a);
+
+}  // namespace la

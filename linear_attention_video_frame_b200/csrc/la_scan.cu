@@ -1,0 +1,204 @@
+// Host side of the C ABI: argument validation, workspace sizing, dispatch.
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+
+#include "common.cuh"
+
+namespace la {
+namespace {
+
+bool shape_supported(int D) { return D >= 16 && D <= 256 && D % 16 == 0; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// A pointer the kernels may dereference: device or managed memory of the
+// current device.  NULL is accepted here (callers decide whether NULL is legal).
+la_status check_ptr(const void* p, int dev) {
+    if (!p) return LA_OK;
+    if (!aligned16(p)) return LA_ERR_INVALID_ARG;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();
+        return LA_ERR_INVALID_ARG;
+    }
+    if (at.type == cudaMemoryTypeManaged) return LA_OK;
+    if (at.type != cudaMemoryTypeDevice || at.device != dev) return LA_ERR_INVALID_ARG;
+    return LA_OK;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+    if (!a || !b) return false;
+    uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+// sm_100 (B200 family) is required: kernels are built for sm_100a only.
+la_status check_device(int* dev_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return LA_ERR_CUDA; }
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return LA_ERR_CUDA;
+    }
+    if (major != 10 || minor != 0) return LA_ERR_UNSUPPORTED;
+    *dev_out = dev;
+    return LA_OK;
+}
+
+size_t workspace_needed(const ScanArgs& a) {
+    return simt_workspace_bytes(a);
+}
+
+// Validation common to every entry point.  `need_q` is false for a state step.
+la_status validate(const ScanArgs& a, bool need_q) {
+    if (a.B < 1 || a.H < 1 || a.F < 0 || a.S < 1) return LA_ERR_INVALID_ARG;
+    if (a.B > 65535 || a.H > 65535) return LA_ERR_INVALID_ARG;
+    if (!shape_supported(a.D)) return LA_ERR_UNSUPPORTED;
+    const double elems = (double)a.B * a.H * a.F * a.S * a.D;
+    if (elems > 9.0e15) return LA_ERR_INVALID_ARG;
+    if (a.mode == LA_MODE_RELU && !(std::isfinite(a.eps) && a.eps >= 0.f)) return LA_ERR_INVALID_ARG;
+    if (a.mode == LA_MODE_GDN && !std::isfinite(a.k_scale)) return LA_ERR_INVALID_ARG;
+    if (!a.ws) return LA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(a.ws) & 255u) != 0) return LA_ERR_INVALID_ARG;
+    if (a.ws_bytes < workspace_needed(a)) return LA_ERR_INVALID_ARG;
+    if (a.F > 0) {
+        if (!a.k || !a.v) return LA_ERR_INVALID_ARG;
+        if (need_q && (!a.q || !a.o)) return LA_ERR_INVALID_ARG;
+        if (a.mode == LA_MODE_GDN && (!a.alpha || !a.beta)) return LA_ERR_INVALID_ARG;
+    }
+    int dev = 0;
+    la_status s = check_device(&dev);
+    if (s != LA_OK) return s;
+    const void* ptrs[] = {a.q, a.k, a.v, a.o, a.alpha, a.beta, a.state_in, a.z_in,
+                          a.state_out, a.z_out, a.ws};
+    for (const void* p : ptrs)
+        if ((s = check_ptr(p, dev)) != LA_OK) return s;
+    if (a.o) {
+        const size_t n = (size_t)a.B * a.H * a.F * a.S * a.D * (a.bf16 ? 2 : 4);
+        if (overlaps(a.o, n, a.q, n) || overlaps(a.o, n, a.k, n) || overlaps(a.o, n, a.v, n))
+            return LA_ERR_INVALID_ARG;
+    }
+    return LA_OK;
+}
+
+la_status run(const ScanArgs& a, cudaStream_t st) {
+    // Reset the device status word recorded in the workspace header.
+    if (cudaMemsetAsync(a.ws, 0, kWsHeaderBytes, st) != cudaSuccess) {
+        cudaGetLastError();
+        return LA_ERR_CUDA;
+    }
+    cudaError_t e = launch_simt(a, st);
+    if (e != cudaSuccess) { cudaGetLastError(); return LA_ERR_CUDA; }
+    return LA_OK;
+}
+
+ScanArgs base_args(const void* k, const void* v, la_dtype dt, int B, int H, int F, int S, int D,
+                   void* ws, size_t wsb) {
+    ScanArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.k = k; a.v = v;
+    a.bf16 = (dt == LA_BF16);
+    a.B = B; a.H = H; a.F = F; a.S = S; a.D = D;
+    a.ws = ws; a.ws_bytes = wsb;
+    a.k_scale = 1.f;
+    return a;
+}
+
+}  // namespace
+}  // namespace la
+
+using namespace la;
+
+extern "C" la_status la_scan_relu(const void* q, const void* k, const void* v, void* o, la_dtype dt,
+                                  const float* state_in, const float* z_in,
+                                  float* state_out, float* z_out,
+                                  int B, int H, int F, int S, int D, float eps,
+                                  void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (dt != LA_F32 && dt != LA_BF16) return LA_ERR_INVALID_ARG;
+    ScanArgs a = base_args(k, v, dt, B, H, F, S, D, workspace, workspace_bytes);
+    a.q = q; a.o = o; a.mode = LA_MODE_RELU; a.eps = eps;
+    a.state_in = state_in; a.z_in = z_in; a.state_out = state_out; a.z_out = z_out;
+    la_status s = validate(a, true);
+    if (s != LA_OK) return s;
+    return run(a, stream);
+}
+
+extern "C" la_status la_scan_gdn(const void* q, const void* k, const void* v, void* o, la_dtype dt,
+                                 const float* alpha, const float* beta, float k_scale,
+                                 const float* state_in, float* state_out,
+                                 int B, int H, int F, int S, int D,
+                                 void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (dt != LA_F32 && dt != LA_BF16) return LA_ERR_INVALID_ARG;
+    ScanArgs a = base_args(k, v, dt, B, H, F, S, D, workspace, workspace_bytes);
+    a.q = q; a.o = o; a.mode = LA_MODE_GDN; a.k_scale = k_scale;
+    a.alpha = alpha; a.beta = beta; a.state_in = state_in; a.state_out = state_out;
+    la_status s = validate(a, true);
+    if (s != LA_OK) return s;
+    return run(a, stream);
+}
+
+extern "C" la_status la_state_step(la_mode mode, const void* k, const void* v, la_dtype dt,
+                                   const float* alpha, const float* beta, float k_scale,
+                                   const float* state_in, const float* z_in,
+                                   float* state_out, float* z_out,
+                                   int B, int H, int F, int S, int D,
+                                   void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (dt != LA_F32 && dt != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (mode != LA_MODE_RELU && mode != LA_MODE_GDN) return LA_ERR_INVALID_ARG;
+    ScanArgs a = base_args(k, v, dt, B, H, F, S, D, workspace, workspace_bytes);
+    a.mode = mode;
+    a.state_in = state_in; a.state_out = state_out;
+    if (mode == LA_MODE_GDN) {
+        a.alpha = alpha; a.beta = beta; a.k_scale = k_scale;
+    } else {
+        a.z_in = z_in; a.z_out = z_out;
+    }
+    la_status s = validate(a, false);
+    if (s != LA_OK) return s;
+    return run(a, stream);
+}
+
+extern "C" size_t la_workspace_size(la_mode mode, int B, int H, int F, int S, int D) {
+    if (B < 1 || H < 1 || F < 0 || S < 1 || !shape_supported(D)) return 0;
+    if (mode != LA_MODE_RELU && mode != LA_MODE_GDN) return 0;
+    ScanArgs a = base_args(nullptr, nullptr, LA_BF16, B, H, F, S, D, nullptr, 0);
+    a.mode = mode;
+    size_t n = workspace_needed(a);
+    a.bf16 = 0;
+    size_t n32 = workspace_needed(a);
+    return n > n32 ? n : n32;
+}
+
+extern "C" la_status la_query_device_status(void* workspace, cudaStream_t stream) {
+    if (!workspace) return LA_ERR_INVALID_ARG;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) { cudaGetLastError(); return LA_ERR_CUDA; }
+    unsigned int status = 0;
+    if (cudaMemcpy(&status, workspace, sizeof(status), cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        return LA_ERR_CUDA;
+    }
+    return status == 0 ? LA_OK : (la_status)status;
+}
+
+extern "C" const char* la_plan(la_mode mode, la_dtype dt, int B, int H, int F, int S, int D,
+                               int* kernels) {
+    if (B < 1 || H < 1 || F < 0 || S < 1 || !shape_supported(D)) return nullptr;
+    if ((mode != LA_MODE_RELU && mode != LA_MODE_GDN) || (dt != LA_F32 && dt != LA_BF16))
+        return nullptr;
+    if (kernels) *kernels = 1;
+    return "simt_f32";
+}
+
+extern "C" const char* la_status_string(la_status s) {
+    switch (s) {
+        case LA_OK: return "LA_OK";
+        case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG";
+        case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED";
+        case LA_ERR_CUDA: return "LA_ERR_CUDA";
+        case LA_ERR_TIMEOUT: return "LA_ERR_TIMEOUT";
+    }
+    return "LA_ERR_UNKNOWN";
+}

@@ -156,13 +156,37 @@ def slice_values(spec: Spec, tensor: str, b: int, h: int) -> np.ndarray:
     return s
 
 
-def full_storage(spec: Spec, tensor: str) -> np.ndarray:
+def for_each_slice(spec: Spec, tensor: str, sink, threads: Optional[int] = None) -> None:
+    """Generate every (b, h) slice of `tensor` on a thread pool and hand each
+    to sink(b, h, storage_array).  Slices are independent streams, so the
+    result does not depend on the thread count or order."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    jobs = [(b, h) for b in range(spec.B) for h in range(spec.H)]
+    n = threads or min(len(jobs), max(1, len(os.sched_getaffinity(0))))
+
+    def one(bh):
+        b, h = bh
+        return b, h, slice_storage(spec, tensor, b, h)
+
+    if n <= 1:
+        for bh in jobs:
+            sink(*one(bh))
+        return
+    with ThreadPoolExecutor(n) as ex:
+        for b, h, arr in ex.map(one, jobs):
+            sink(b, h, arr)
+
+
+def full_storage(spec: Spec, tensor: str, threads: Optional[int] = None) -> np.ndarray:
     """Storage array [B, H, F, S, D] (float32 or uint16 bf16 bits)."""
     dt = np.float32 if spec.dtype == "f32" else np.uint16
     out = np.empty((spec.B, spec.H, spec.F, spec.S, spec.D), dtype=dt)
-    for b in range(spec.B):
-        for h in range(spec.H):
-            out[b, h] = slice_storage(spec, tensor, b, h)
+
+    def put(b, h, arr):
+        out[b, h] = arr
+
+    for_each_slice(spec, tensor, put, threads)
     return out
 
 

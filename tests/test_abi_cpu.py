@@ -1,0 +1,106 @@
+"""The C-ABI library on a machine without a GPU: it loads, exports every
+declared symbol, and rejects bad arguments before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_attention_video_frame_b200 as la
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                      "include", "la_scan.h")
+
+
+def declared_symbols():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"LA_API\s+[\w\s\*]+?\b(la_\w+)\s*\(", txt)))
+
+
+def test_header_declares_the_abi():
+    assert declared_symbols() == sorted([
+        "la_scan_relu", "la_scan_gdn", "la_state_step", "la_workspace_size",
+        "la_query_device_status", "la_status_string", "la_plan"])
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(la.LIB_PATH)
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_plan_reports_a_path_and_kernel_count():
+    name, n = la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 20, 181, 880, 128)
+    assert name in ("tcgen05", "simt_f32") and n >= 1
+    name, n = la.la_plan(la.LA_MODE_RELU, la.LA_F32, 1, 2, 8, 64, 32)
+    assert name == "simt_f32" and n == 1
+    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 1, 1, 1, 24) == (None, 0)
+
+
+def test_status_strings():
+    assert la.la_status_string(la.LA_OK) == "LA_OK"
+    assert la.la_status_string(la.LA_ERR_TIMEOUT) == "LA_ERR_TIMEOUT"
+    assert la.la_status_string(99) == "LA_ERR_UNKNOWN"
+
+
+@pytest.mark.parametrize("D", [0, 8, 24, 100, 272])
+def test_workspace_size_rejects_unsupported_head_dims(D):
+    assert la.la_workspace_size(la.LA_MODE_GDN, 1, 1, 4, 64, D) == 0
+
+
+@pytest.mark.parametrize("mode", [la.LA_MODE_RELU, la.LA_MODE_GDN])
+@pytest.mark.parametrize("cfg", [(1, 2, 8, 64, 32), (1, 20, 21, 1560, 112),
+                                 (1, 20, 181, 880, 128), (1, 16, 512, 1024, 256)])
+def test_workspace_size_positive_and_aligned(mode, cfg):
+    n = la.la_workspace_size(mode, *cfg)
+    assert n >= 256 and n % 256 == 0
+
+
+def _fake(addr=0x10000):
+    return ctypes.c_void_p(addr)
+
+
+def test_argument_errors_return_before_any_cuda_call():
+    L = la.lib
+    P = _fake
+    ws = la.la_workspace_size(la.LA_MODE_GDN, 1, 1, 2, 8, 32)
+    # unsupported head dim
+    assert L.la_scan_gdn(P(), P(), P(), P(), la.LA_BF16, P(), P(), 0.1, None, None,
+                         1, 1, 2, 8, 24, P(), ws, None) == la.LA_ERR_UNSUPPORTED
+    # bad sizes
+    assert L.la_scan_gdn(P(), P(), P(), P(), la.LA_BF16, P(), P(), 0.1, None, None,
+                         0, 1, 2, 8, 32, P(), ws, None) == la.LA_ERR_INVALID_ARG
+    assert L.la_scan_relu(P(), P(), P(), P(), la.LA_BF16, None, None, None, None,
+                          1, 1, 2, 0, 32, 1e-6, P(), ws, None) == la.LA_ERR_INVALID_ARG
+    # negative / non-finite eps, non-finite key scale
+    assert L.la_scan_relu(P(), P(), P(), P(), la.LA_BF16, None, None, None, None,
+                          1, 1, 2, 8, 32, -1.0, P(), ws, None) == la.LA_ERR_INVALID_ARG
+    assert L.la_scan_gdn(P(), P(), P(), P(), la.LA_BF16, P(), P(), float("nan"), None, None,
+                         1, 1, 2, 8, 32, P(), ws, None) == la.LA_ERR_INVALID_ARG
+    # missing / misaligned / undersized workspace
+    assert L.la_scan_gdn(P(), P(), P(), P(), la.LA_BF16, P(), P(), 0.1, None, None,
+                         1, 1, 2, 8, 32, None, ws, None) == la.LA_ERR_INVALID_ARG
+    assert L.la_scan_gdn(P(), P(), P(), P(), la.LA_BF16, P(), P(), 0.1, None, None,
+                         1, 1, 2, 8, 32, P(0x10010), ws, None) == la.LA_ERR_INVALID_ARG
+    assert L.la_scan_gdn(P(), P(), P(), P(), la.LA_BF16, P(), P(), 0.1, None, None,
+                         1, 1, 2, 8, 32, P(), 16, None) == la.LA_ERR_INVALID_ARG
+    # missing gates / inputs / output
+    assert L.la_scan_gdn(P(), P(), P(), P(), la.LA_BF16, None, P(), 0.1, None, None,
+                         1, 1, 2, 8, 32, P(), ws, None) == la.LA_ERR_INVALID_ARG
+    assert L.la_scan_gdn(P(), None, P(), P(), la.LA_BF16, P(), P(), 0.1, None, None,
+                         1, 1, 2, 8, 32, P(), ws, None) == la.LA_ERR_INVALID_ARG
+    assert L.la_scan_relu(P(), P(), P(), None, la.LA_BF16, None, None, None, None,
+                          1, 1, 2, 8, 32, 1e-6, P(), ws, None) == la.LA_ERR_INVALID_ARG
+    # bad dtype / mode
+    assert L.la_scan_relu(P(), P(), P(), P(), 7, None, None, None, None,
+                          1, 1, 2, 8, 32, 1e-6, P(), ws, None) == la.LA_ERR_INVALID_ARG
+    assert L.la_state_step(5, P(), P(), la.LA_BF16, None, None, 1.0, None, None, None, None,
+                           1, 1, 2, 8, 32, P(), ws, None) == la.LA_ERR_INVALID_ARG
+
+
+def test_python_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 1, 1, 16, 16, dtype=torch.bfloat16)
+    a = torch.ones(1, 1, 1)
+    with pytest.raises(ValueError):
+        la.la_scan_gdn(x, x, x, a, a, 0.1, workspace=torch.zeros(1024, dtype=torch.uint8))

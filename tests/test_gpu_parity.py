@@ -1,0 +1,250 @@
+"""GPU parity: the CUDA scan (through the C ABI) against the CPU oracle.
+
+Bars (max|gpu - ref| / max|ref| over the compared tensor): 1e-4 for float32
+inputs, 2e-2 for bfloat16 inputs with a float32 state.  Small cases are
+compared element by element in full; the full-size workloads in the launch
+configuration the benchmark times are compared on every head where the
+oracle is quick (480p ReLU, 720p GDN) and on sampled heads otherwise.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import linear_attention_video_frame_b200 as la
+import oracle
+import synth
+from helpers import (TOL_BF16, TOL_F32, device_inputs, oracle_slice, rel_err, to_device,
+                     to_np, tol_for)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    torch.cuda.init()
+
+
+def _run(spec, mode, inp, state_in=None, z_in=None, want_state=True):
+    B, H, D = spec.B, spec.H, spec.D
+    so = torch.full((B, H, D, D), float("nan"), device="cuda") if want_state else None
+    if mode == "relu":
+        zo = torch.full((B, H, D), float("nan"), device="cuda") if want_state else None
+        o = la.la_scan_relu(inp["q"], inp["k"], inp["v"], state_in=state_in, z_in=z_in,
+                            state_out=so, z_out=zo, eps=spec.eps)
+        return o, so, zo
+    o = la.la_scan_gdn(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], spec.k_scale,
+                       state_in=state_in, state_out=so)
+    return o, so, None
+
+
+def _oracle(spec, mode, b, h, m0=None, z0=None):
+    q, k, v, a, bt = oracle_slice(spec, b, h)
+    if mode == "relu":
+        o, m, z = oracle.relu_scan(q, k, v, spec.eps, m0, z0)
+        return o[0, 0], m[0, 0], z[0, 0]
+    o, m = oracle.gdn_scan(q, k, v, a, bt, spec.k_scale, m0)
+    return o[0, 0], m[0, 0], None
+
+
+def _compare(spec, mode, heads=None, with_state=False):
+    inp = device_inputs(spec)
+    m0 = z0 = None
+    if with_state:
+        m0n, z0n = synth.random_state(spec, scale=0.05)
+        m0, z0 = torch.from_numpy(m0n).cuda(), torch.from_numpy(z0n).cuda()
+    o, so, zo = _run(spec, mode, inp, m0, z0 if mode == "relu" else None)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o.float()).all()
+    tol = tol_for(spec)
+    pairs = heads if heads is not None else [(b, h) for b in range(spec.B) for h in range(spec.H)]
+    worst = 0.0
+    ref_o, got_o, ref_m, got_m = [], [], [], []
+    for b, h in pairs:
+        rm0 = None if m0 is None else m0n[b:b + 1, h:h + 1]
+        rz0 = None if z0 is None else z0n[b:b + 1, h:h + 1]
+        ro, rm, rz = _oracle(spec, mode, b, h, rm0, rz0)
+        ref_o.append(ro); got_o.append(to_np(o[b, h]))
+        ref_m.append(rm); got_m.append(to_np(so[b, h]))
+        if rz is not None:
+            assert rel_err(to_np(zo[b, h]), rz) < 1e-5
+    e_o = rel_err(np.stack(got_o), np.stack(ref_o))
+    e_m = rel_err(np.stack(got_m), np.stack(ref_m))
+    assert e_o <= tol, f"output error {e_o:.3e} > {tol}"
+    assert e_m <= tol, f"state error {e_m:.3e} > {tol}"
+    return e_o, e_m
+
+
+# ----------------------------------------------------------------------------
+# The five workloads
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("mode", ["relu", "gdn"])
+def test_tiny_fp32_config(mode):
+    _compare(synth.config(0), mode)
+
+
+@pytest.mark.parametrize("mode", ["relu", "gdn"])
+def test_tiny_fp32_config_with_state_in(mode):
+    _compare(synth.config(0), mode, with_state=True)
+
+
+def test_relu_480p_all_heads():
+    _compare(synth.config(1), "relu")
+
+
+def test_gdn_720p_60s_all_heads():
+    _compare(synth.config(2), "gdn")
+
+
+@pytest.mark.parametrize("mode", ["relu", "gdn"])
+def test_stress_d256_sampled_heads(mode):
+    _compare(synth.config(4), mode, heads=[(0, 0), (0, 11)])
+
+
+def test_streaming_chunks_equal_single_scan():
+    spec = synth.config(3)
+    inp = device_inputs(spec)
+    B, H, F, D, C = spec.B, spec.H, spec.F, spec.D, spec.chunk_frames
+    whole, m_whole, _ = _run(spec, "gdn", inp)
+    state = torch.empty((B, H, D, D), device="cuda")
+    outs = []
+    for c in range(F // C):
+        sl = slice(c * C, (c + 1) * C)
+        part = {n: inp[n][:, :, sl].contiguous() for n in ("q", "k", "v", "alpha", "beta")}
+        o = la.la_scan_gdn(part["q"], part["k"], part["v"], part["alpha"], part["beta"],
+                           spec.k_scale, state_in=state if c else None, state_out=state)
+        outs.append(o)
+    chunked = torch.cat(outs, dim=2)
+    torch.cuda.synchronize()
+    # chunked == single scan up to float32 summation order
+    assert rel_err(to_np(chunked), to_np(whole)) < 1e-2
+    assert rel_err(to_np(state), to_np(m_whole)) < 1e-3
+    # and both match the oracle's single 64-frame scan on sampled batch items
+    for b, h in [(0, 0), (3, 19)]:
+        ro, rm, _ = _oracle(spec, "gdn", b, h)
+        assert rel_err(to_np(chunked[b, h]), ro) <= TOL_BF16
+        assert rel_err(to_np(state[b, h]), rm) <= TOL_BF16
+
+
+# ----------------------------------------------------------------------------
+# Edge cases: ragged token tails, odd head dims, one token, in-place state
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("mode", ["relu", "gdn"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("D,S,F", [(16, 1, 3), (48, 17, 2), (64, 130, 3), (112, 200, 2),
+                                   (128, 129, 3), (256, 70, 2)])
+def test_small_shapes(mode, dtype, D, S, F):
+    spec = synth.small(B=2, H=2, F=F, S=S, D=D, dtype=dtype, seed=D + S)
+    _compare(spec, mode, with_state=True)
+
+
+@pytest.mark.parametrize("mode", ["relu", "gdn"])
+def test_zero_frames_copies_state(mode):
+    spec = synth.small(B=1, H=3, F=0, S=8, D=32, dtype="bf16")
+    m0n, z0n = synth.random_state(spec)
+    m0, z0 = torch.from_numpy(m0n).cuda(), torch.from_numpy(z0n).cuda()
+    inp = device_inputs(spec)
+    o, so, zo = _run(spec, mode, inp, m0, z0 if mode == "relu" else None)
+    torch.cuda.synchronize()
+    assert torch.equal(so, m0)
+    if mode == "relu":
+        assert torch.equal(zo, z0)
+    # NULL state_in: zeros
+    o, so, zo = _run(spec, mode, inp)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(so) == 0
+
+
+@pytest.mark.parametrize("mode", ["relu", "gdn"])
+def test_in_place_state(mode):
+    spec = synth.small(B=1, H=2, F=3, S=40, D=64, dtype="bf16", seed=9)
+    inp = device_inputs(spec)
+    m0n, z0n = synth.random_state(spec, 0.1)
+    m, z = torch.from_numpy(m0n).cuda(), torch.from_numpy(z0n).cuda()
+    if mode == "relu":
+        la.la_scan_relu(inp["q"], inp["k"], inp["v"], state_in=m, z_in=z, state_out=m, z_out=z)
+    else:
+        la.la_scan_gdn(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], spec.k_scale,
+                       state_in=m, state_out=m)
+    torch.cuda.synchronize()
+    for h in range(2):
+        _, rm, rz = _oracle(spec, mode, 0, h, m0n[:, h:h + 1], z0n[:, h:h + 1])
+        assert rel_err(to_np(m[0, h]), rm) <= TOL_BF16
+        if mode == "relu":
+            assert rel_err(to_np(z[0, h]), rz) <= 1e-5
+
+
+@pytest.mark.parametrize("mode", ["relu", "gdn"])
+def test_state_step_matches_oracle(mode):
+    spec = synth.small(B=2, H=2, F=4, S=100, D=128, dtype="bf16", seed=21, keys_l2=True)
+    inp = device_inputs(spec)
+    m0n, z0n = synth.random_state(spec, 0.05)
+    m0, z0 = torch.from_numpy(m0n).cuda(), torch.from_numpy(z0n).cuda()
+    so = torch.empty_like(m0)
+    zo = torch.empty_like(z0)
+    mode_c = la.LA_MODE_RELU if mode == "relu" else la.LA_MODE_GDN
+    la.la_state_step(mode_c, inp["k"], inp["v"], inp["alpha"], inp["beta"], spec.k_scale,
+                     state_in=m0, z_in=z0, state_out=so, z_out=zo)
+    torch.cuda.synchronize()
+    for b in range(2):
+        for h in range(2):
+            _, k, v, a, bt = oracle_slice(spec, b, h)
+            if mode == "relu":
+                rm, rz = oracle.relu_state_step(k, v, m0n[b:b + 1, h:h + 1], z0n[b:b + 1, h:h + 1])
+                assert rel_err(to_np(zo[b, h]), rz[0, 0]) < 1e-5
+            else:
+                rm = oracle.gdn_state_step(k, v, a, bt, spec.k_scale, m0n[b:b + 1, h:h + 1])
+            assert rel_err(to_np(so[b, h]), rm[0, 0]) <= TOL_BF16
+
+
+def test_outputs_do_not_write_outside_their_buffers():
+    spec = synth.small(B=1, H=2, F=2, S=77, D=48, dtype="bf16", seed=5)
+    inp = device_inputs(spec)
+    n = spec.B * spec.H * spec.F * spec.S * spec.D
+    guard = 4096
+    buf = torch.full((n + 2 * guard,), 7.0, dtype=torch.bfloat16, device="cuda")
+    o = buf[guard:guard + n].view(spec.B, spec.H, spec.F, spec.S, spec.D)
+    sbuf = torch.full((spec.H * spec.D * spec.D + 2 * guard,), 3.0, device="cuda")
+    so = sbuf[guard:guard + spec.H * spec.D * spec.D].view(1, spec.H, spec.D, spec.D)
+    la.la_scan_gdn(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], spec.k_scale,
+                   o=o, state_out=so)
+    la.la_scan_relu(inp["q"], inp["k"], inp["v"], o=o, state_out=so)
+    torch.cuda.synchronize()
+    assert torch.all(buf[:guard] == 7.0) and torch.all(buf[guard + n:] == 7.0)
+    assert torch.all(sbuf[:guard] == 3.0) and torch.all(sbuf[-guard:] == 3.0)
+
+
+# ----------------------------------------------------------------------------
+# Argument errors that need a device to detect
+# ----------------------------------------------------------------------------
+def test_rejects_host_and_overlapping_pointers():
+    spec = synth.small(B=1, H=1, F=2, S=16, D=32, dtype="bf16")
+    inp = device_inputs(spec)
+    ws = la.workspace_for(la.LA_MODE_GDN, 1, 1, 2, 16, 32)
+    host = torch.zeros(1, 1, 2, 16, 32, dtype=torch.bfloat16).pin_memory()
+    P = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    L = la.lib
+    s = torch.cuda.current_stream().cuda_stream
+    # unregistered host memory
+    h = np.zeros(2 * 16 * 32, dtype=np.uint16)
+    st = L.la_scan_gdn(P(inp["q"]), P(inp["k"]), P(inp["v"]), h.ctypes.data, la.LA_BF16,
+                       P(inp["alpha"]), P(inp["beta"]), 0.1, None, None, 1, 1, 2, 16, 32,
+                       P(ws), ws.numel(), s)
+    assert st == la.LA_ERR_INVALID_ARG
+    # output overlapping an input
+    st = L.la_scan_gdn(P(inp["q"]), P(inp["k"]), P(inp["v"]), P(inp["q"]), la.LA_BF16,
+                       P(inp["alpha"]), P(inp["beta"]), 0.1, None, None, 1, 1, 2, 16, 32,
+                       P(ws), ws.numel(), s)
+    assert st == la.LA_ERR_INVALID_ARG
+    # misaligned pointer
+    o = torch.empty(2 * 16 * 32 + 8, dtype=torch.bfloat16, device="cuda")
+    st = L.la_scan_gdn(P(inp["q"]), P(inp["k"]), P(inp["v"]), o.data_ptr() + 2, la.LA_BF16,
+                       P(inp["alpha"]), P(inp["beta"]), 0.1, None, None, 1, 1, 2, 16, 32,
+                       P(ws), ws.numel(), s)
+    assert st == la.LA_ERR_INVALID_ARG
+    # a rejected call enqueues nothing; a valid call afterwards records LA_OK
+    la.la_scan_gdn(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], 0.1, workspace=ws)
+    assert la.la_query_device_status(ws) == la.LA_OK
+    del host
