@@ -59,4 +59,10 @@ __device__ __forceinline__ void store_elem(void* p, size_t i, float x, int bf16)
 cudaError_t launch_simt(const ScanArgs& a, cudaStream_t st);
 size_t simt_workspace_bytes(const ScanArgs& a);
 
+// Tensor-core path: bf16 inputs, 64 <= D <= 128, F > 0.
+bool tc_eligible(const ScanArgs& a);
+size_t tc_workspace_bytes(const ScanArgs& a);
+int tc_kernel_count(const ScanArgs& a);
+cudaError_t launch_tc(const ScanArgs& a, cudaStream_t st);
+
 }  // namespace la

@@ -48,8 +48,17 @@ la_status check_device(int* dev_out) {
     return LA_OK;
 }
 
+// LA_SCAN_FORCE_SIMT=1 in the environment routes every call to the float32
+// SIMT kernel (used by tests to compare the two kernel paths).
+bool force_simt() {
+    const char* e = std::getenv("LA_SCAN_FORCE_SIMT");
+    return e && e[0] == '1';
+}
+
+bool use_tc(const ScanArgs& a) { return !force_simt() && tc_eligible(a); }
+
 size_t workspace_needed(const ScanArgs& a) {
-    return simt_workspace_bytes(a);
+    return use_tc(a) ? tc_workspace_bytes(a) : simt_workspace_bytes(a);
 }
 
 // Validation common to every entry point.  `need_q` is false for a state step.
@@ -90,7 +99,7 @@ la_status run(const ScanArgs& a, cudaStream_t st) {
         cudaGetLastError();
         return LA_ERR_CUDA;
     }
-    cudaError_t e = launch_simt(a, st);
+    cudaError_t e = use_tc(a) ? launch_tc(a, st) : launch_simt(a, st);
     if (e != cudaSuccess) { cudaGetLastError(); return LA_ERR_CUDA; }
     return LA_OK;
 }
@@ -188,6 +197,13 @@ extern "C" const char* la_plan(la_mode mode, la_dtype dt, int B, int H, int F, i
     if (B < 1 || H < 1 || F < 0 || S < 1 || !shape_supported(D)) return nullptr;
     if ((mode != LA_MODE_RELU && mode != LA_MODE_GDN) || (dt != LA_F32 && dt != LA_BF16))
         return nullptr;
+    ScanArgs a = base_args(nullptr, nullptr, dt, B, H, F, S, D, nullptr, 0);
+    a.mode = mode;
+    a.o = reinterpret_cast<void*>(uintptr_t(1));    // a scan (with outputs)
+    if (use_tc(a)) {
+        if (kernels) *kernels = tc_kernel_count(a);
+        return "tcgen05";
+    }
     if (kernels) *kernels = 1;
     return "simt_f32";
 }

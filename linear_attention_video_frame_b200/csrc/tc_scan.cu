@@ -1,0 +1,787 @@
+// Tensor-core (tcgen05) scan for bf16 inputs and 64 <= D <= 128.
+//
+// The scan is split along what depends on what:
+//
+//   gram   (frame-parallel)  per (b, h, f): stream K_f, V_f through TMA and
+//          contract over the frame's tokens on the tensor core.
+//            GDN : G'_f = beta kappa^2 K^T K  (bf16 operand image)
+//                  B_f  = beta kappa   K^T V  (fp32)
+//            ReLU: dM_f = phi(K)^T V (fp32), dz_f = phi(K)^T 1 (fp32)
+//   chain  (sequential per (b, h)): the fp32 state lives in tensor memory.
+//            GDN : M_f = alpha_f (M_{f-1} - G'_f bf16(M_{f-1})) + B_f
+//                  (one D x D x D MMA per frame, negated A accumulated onto M)
+//            ReLU: M_f = M_{f-1} + dM_f,  z_f = z_{f-1} + dz_f
+//          and publishes bf16(M_f) as an MMA operand image for the outputs.
+//   output (frame-parallel)  per (b, h, f): O_f = Q~_f bf16(M_f), with the
+//          ReLU feature map and the normaliser phi(Q) z_f + eps fused.
+//
+// This is the frame-wise Gated DeltaNet of the SANA-WM paper summary
+// (section 3, "Hybrid GDN/Softmax Attention"), written in its affine form
+// M_f = A_f M_{f-1} + B_f with A_f = alpha_f (I - beta_f Kh^T Kh) -- the same
+// per-frame affine map whose composites the paper's context-parallel training
+// exchanges (appendix C.1) -- and the block-causal ReLU linear attention of
+// the SANA-Video talk (block KV cache segment).
+//
+// Layouts.  q, k, v, o are viewed by TMA as [B*H*F][S][D] bf16 with a 64-wide
+// (128-byte) swizzled box; out-of-range tokens and columns read as zero.
+// Operand images in the workspace are byte-exact shared-memory images
+// (128 B rows, 128-byte swizzle, two 64-column blocks of 16 KB):
+//   G' image: K-major, row i = key dim, columns = key dim (symmetric).
+//   M  image: MN-major, row i = key dim, columns = value dim.
+// The fp32 per-frame matrices B_f / dM_f are stored "quad-interleaved":
+// element (i, j) at ((j / 4) * 128 + i) * 4 + j % 4, so that the 32 lanes of
+// a warp, which own 32 consecutive rows, touch 512 contiguous bytes.
+#include "tc_common.cuh"
+#include "tmap.cuh"
+
+namespace la {
+namespace {
+
+using namespace tc;
+
+constexpr int kTokG = 64;                   // tokens per gram tile
+constexpr int kTokO = 128;                  // tokens per output tile
+constexpr int kGStages = 4;                 // gram TMA ring depth
+constexpr int kCStages = 2;                 // chain operand ring depth
+constexpr int kOStages = 2;                 // output Q ring depth
+constexpr int kOAcc = 4;                    // output accumulator slots (128 cols each)
+constexpr uint32_t kBoxG = 64 * kTokG * 2;  // 8 KB: one 64-column box of a gram tile
+constexpr uint32_t kBoxO = 64 * kTokO * 2;  // 16 KB: one 64-column box of an output tile
+constexpr uint32_t kImg = 2 * 16384;        // 32 KB: 128 rows x 128 columns bf16 image
+constexpr uint32_t kQuadMat = 128 * 128 * 4;// 64 KB: fp32 128 x 128 quad-interleaved
+constexpr int kEpiThreads = 128;            // 4 epilogue warps
+
+struct TcParams {
+    const float* alpha;
+    const float* beta;
+    const float* state_in;
+    const float* z_in;
+    float* state_out;
+    float* z_out;
+    unsigned int* status;   // workspace header (status, where)
+    uint8_t* gimg;          // [BHF] x kImg          (GDN)
+    float* bmat;            // [BHF] x 128 x 128 fp32 quad-interleaved
+    uint8_t* mimg;          // [BHF] x kImg
+    float* dz;              // [BHF] x 128           (ReLU)
+    float* zf;              // [BHF] x 128           (ReLU)
+    float k_scale;
+    float eps;
+    int BH, F, S, D;
+    int want_output;
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// ReLU of 8 packed bf16 values: clear every element whose sign bit is set.
+__device__ __forceinline__ uint32_t relu_bf16x2(uint32_t w) {
+    const uint32_t m = ((w >> 15) & 0x00010001u) * 0xFFFFu;
+    return w & ~m;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Write 16 consecutive columns [c0, c0+16) of row `row` of a 2-block image.
+__device__ __forceinline__ void store_row16_bf16(uint8_t* img, int row, int c0, const float (&v)[16]) {
+    const int blk = c0 >> 6, ch = (c0 & 63) >> 3;
+    uint4 a = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                         pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+    uint4 b = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
+                         pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+    *reinterpret_cast<uint4*>(img + blk * 16384 + sw128_off(row, ch)) = a;
+    *reinterpret_cast<uint4*>(img + blk * 16384 + sw128_off(row, ch + 1)) = b;
+}
+
+// ============================================================================
+// gram: per-frame contractions over tokens
+// ============================================================================
+// warp 0: TMA producer; warp 1: TMEM owner + MMA issuer; warps 2-5: epilogue;
+// warps 6-9 (ReLU): apply phi to each K tile in shared memory before the MMA.
+template <bool RELU>
+__global__ void __launch_bounds__(RELU ? 320 : 192, 1)
+tc_gram_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapK,
+               const __grid_constant__ CUtensorMap mapV) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* ring = smem;                              // kGStages x (K 16 KB | V 16 KB)
+    uint8_t* stage_img = ring + kGStages * 32768;      // G' image staging (GDN)
+    uint8_t* ones = stage_img + kImg;                  // 2 KB of bf16 1.0 (ReLU)
+    uint64_t* full = reinterpret_cast<uint64_t*>(ones + 2048);
+    uint64_t* empty = full + kGStages;
+    uint64_t* xform = empty + kGStages;
+    uint64_t* accfull = xform + kGStages;
+    uint64_t* accempty = accfull + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + 2);
+    uint32_t* abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kGStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&xform[s], 4);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&accfull[a], 1);
+            mbar_init(&accempty[a], 4);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (RELU)
+        for (int i = threadIdx.x; i < 2048 / 4; i += blockDim.x)
+            reinterpret_cast<uint32_t*>(ones)[i] = 0x3F803F80u;
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    const Abort ab{abort_flag, p.status};
+    const int nitems = p.BH * p.F;
+    const int nt = (p.S + kTokG - 1) / kTokG;
+    const int D = p.D;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&mapK);
+            tma_prefetch_desc(&mapV);
+            const uint64_t pol = policy_evict_first();
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x) {
+                for (int t = 0; t < nt; ++t) {
+                    if (!(ok = mbar_wait(&empty[s], ph ^ 1, ab, 0x101))) break;
+                    uint8_t* st = ring + s * 32768;
+                    mbar_expect_tx(&full[s], 4 * kBoxG);
+                    tma_load_3d(st, &mapK, &full[s], 0, t * kTokG, item, pol);
+                    tma_load_3d(st + kBoxG, &mapK, &full[s], 64, t * kTokG, item, pol);
+                    tma_load_3d(st + 16384, &mapV, &full[s], 0, t * kTokG, item, pol);
+                    tma_load_3d(st + 16384 + kBoxG, &mapV, &full[s], 64, t * kTokG, item, pol);
+                    if (++s == kGStages) { s = 0; ph ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idKK = idesc_bf16(128, D, true, true);
+            const uint32_t idZ = idesc_bf16(128, 16, true, false);
+            const uint64_t ones_d = sdesc_sw128(smem_u32(ones), 16, 1024);
+            int s = 0, li = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
+                const int slot = li & 1;
+                if (!(ok = mbar_wait(&accempty[slot], ((li >> 1) & 1) ^ 1, ab, 0x102))) break;
+                tc_fence_after();
+                const uint32_t dG = tbase + slot * 256, dW = dG + 128;
+                for (int t = 0; t < nt; ++t) {
+                    if (!(ok = mbar_wait(RELU ? &xform[s] : &full[s], ph, ab, 0x103))) break;
+                    tc_fence_after();
+                    const uint32_t sk = smem_u32(ring + s * 32768), sv = sk + 16384;
+#pragma unroll
+                    for (int k = 0; k < kTokG / 16; ++k) {
+                        const uint64_t ad = sdesc_sw128(sk + k * 2048, kBoxG, 1024);
+                        const uint64_t bv = sdesc_sw128(sv + k * 2048, kBoxG, 1024);
+                        const uint32_t acc = (t | k) ? 1u : 0u;
+                        if (RELU) {
+                            mma_bf16(dW, ad, bv, idKK, acc);
+                            mma_bf16(dG, ad, ones_d, idZ, acc);
+                        } else {
+                            mma_bf16(dG, ad, ad, idKK, acc);
+                            mma_bf16(dW, ad, bv, idKK, acc);
+                        }
+                    }
+                    mma_commit(&empty[s]);
+                    if (++s == kGStages) { s = 0; ph ^= 1; }
+                }
+                if (ok) mma_commit(&accfull[slot]);
+            }
+        }
+    } else if (warp < 6) {
+        // ---------------- epilogue: TMEM -> workspace ----------------
+        const int q = warp & 3, row = q * 32 + lane;
+        const bool issuer = (threadIdx.x == 64);
+        int li = 0;
+        bool ok = true;     // every epilogue warp runs every named barrier, even after an abort
+        for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++li) {
+            const int slot = li & 1;
+            ok = ok && mbar_wait(&accfull[slot], (li >> 1) & 1, ab, 0x104);
+            tc_fence_after();
+            const uint32_t tl = tbase + (uint32_t(q * 32) << 16) + slot * 256;
+            float* bq = p.bmat + (size_t)item * (kQuadMat / 4);
+            if (!RELU) {
+                const float bt = p.beta[item];
+                const float sg = bt * p.k_scale * p.k_scale, sw = bt * p.k_scale;
+                if (issuer) bulk_wait_read<0>();       // staging free again
+                named_bar_sync(1, kEpiThreads);
+                for (int c0 = 0; c0 < D && ok; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tl + c0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] *= sg;
+                    store_row16_bf16(stage_img, row, c0, v);
+                }
+                for (int c0 = 0; c0 < D && ok; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tl + 128 + c0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        *reinterpret_cast<float4*>(bq + ((c0 / 4 + u) * 128 + row) * 4) =
+                            make_float4(v[4 * u] * sw, v[4 * u + 1] * sw, v[4 * u + 2] * sw,
+                                        v[4 * u + 3] * sw);
+                }
+            } else if (ok) {
+                for (int c0 = 0; c0 < D; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tl + 128 + c0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        *reinterpret_cast<float4*>(bq + ((c0 / 4 + u) * 128 + row) * 4) =
+                            make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                }
+                float v[16];
+                tmem_ld16(tl, v);
+                tmem_wait_ld();
+                p.dz[(size_t)item * 128 + row] = v[0];
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&accempty[slot]);
+            if (!RELU) {
+                fence_proxy_async_smem();
+                named_bar_sync(1, kEpiThreads);
+                if (issuer && ok) {
+                    bulk_store(p.gimg + (size_t)item * kImg, stage_img, kImg);
+                    bulk_commit();
+                }
+            }
+        }
+        if (issuer) bulk_wait_all<0>();
+    } else {
+        // ---------------- ReLU transform: phi(K) in place ----------------
+        const int tl = threadIdx.x - 192;          // 0..127
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x) {
+            for (int t = 0; t < nt; ++t) {
+                if (!(ok = mbar_wait(&full[s], ph, ab, 0x105))) break;
+                uint4* kt = reinterpret_cast<uint4*>(ring + s * 32768);
+                for (int i = tl; i < 2 * (int)kBoxG / 16; i += 128) {
+                    uint4 x = kt[i];
+                    x.x = relu_bf16x2(x.x); x.y = relu_bf16x2(x.y);
+                    x.z = relu_bf16x2(x.z); x.w = relu_bf16x2(x.w);
+                    kt[i] = x;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xform[s]);
+                if (++s == kGStages) { s = 0; ph ^= 1; }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tbase, 512);
+}
+
+// ============================================================================
+// chain: the per-(b, h) recurrence, state resident in tensor memory
+// ============================================================================
+// warp 0: bulk loader of the per-frame operands; warp 1: TMEM owner + MMA
+// issuer (GDN); warps 2-5: epilogue (thread <-> state row).
+template <bool RELU>
+__global__ void __launch_bounds__(192, 1)
+tc_chain_kernel(const TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    // stage s: [G' image 32 KB (GDN)] [B / dM 64 KB] [dz 512 B (ReLU)]
+    constexpr uint32_t kStage = (RELU ? 0 : kImg) + kQuadMat + (RELU ? 512 : 0);
+    uint8_t* ring = smem;
+    uint8_t* mimg = ring + kCStages * kStage;          // bf16(M) operand image
+    mimg = align1024(mimg);
+    uint64_t* full = reinterpret_cast<uint64_t*>(mimg + kImg);
+    uint64_t* empty = full + kCStages;
+    uint64_t* mdone = empty + kCStages;    // MMA of the frame finished
+    uint64_t* mready = mdone + 1;          // image of the current state written
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mready + 1);
+    uint32_t* abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.x;
+    const int F = p.F, D = p.D;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kCStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], RELU ? 4 : 5);     // epilogue warps (+ the MMA for GDN)
+        }
+        mbar_init(mdone, 1);
+        mbar_init(mready, 4);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tM = *tmem_slot;
+    const Abort ab{abort_flag, p.status};
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            for (int f = 0; f < F; ++f) {
+                if (!mbar_wait(&empty[s], ph ^ 1, ab, 0x201)) break;
+                const size_t frame = (size_t)bh * F + f;
+                uint8_t* st = ring + s * kStage;
+                mbar_expect_tx(&full[s], kStage);
+                if (!RELU) {
+                    bulk_load(st, p.gimg + frame * kImg, kImg, &full[s]);
+                    bulk_load(st + kImg, p.bmat + frame * (kQuadMat / 4), kQuadMat, &full[s]);
+                } else {
+                    bulk_load(st, p.bmat + frame * (kQuadMat / 4), kQuadMat, &full[s]);
+                    bulk_load(st + kQuadMat, p.dz + frame * 128, 512, &full[s]);
+                }
+                if (++s == kCStages) { s = 0; ph ^= 1; }
+            }
+        }
+    } else if (warp == 1) {
+        if (!RELU && lane == 0) {
+            const uint32_t idC = idesc_bf16(128, D, false, true, /*negate_a=*/true);
+            int s = 0;
+            uint32_t ph = 0;
+            for (int f = 0; f < F; ++f) {
+                if (!mbar_wait(&full[s], ph, ab, 0x202)) break;
+                if (!mbar_wait(mready, f & 1, ab, 0x203)) break;
+                tc_fence_after();
+                const uint32_t ga = smem_u32(ring + s * kStage), mb = smem_u32(mimg);
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t ad = sdesc_sw128(ga + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(mb + kk * 2048, 16384, 1024);
+                    mma_bf16(tM, ad, bd, idC, 1u);
+                }
+                mma_commit(mdone);
+                mma_commit(&empty[s]);
+                if (++s == kCStages) { s = 0; ph ^= 1; }
+            }
+        }
+    } else {
+        // ---------------- epilogue: thread <-> state row ----------------
+        const int q = warp & 3, row = q * 32 + lane;
+        const bool issuer = (threadIdx.x == 64);
+        const uint32_t tl = tM + (uint32_t(q * 32) << 16);
+        const bool live = row < D;
+        // initial state: TMEM (fp32) and operand image (bf16)
+        for (int c0 = 0; c0 < D; c0 += 16) {
+            float v[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                v[e] = (p.state_in && live) ? p.state_in[((size_t)bh * D + row) * D + c0 + e] : 0.f;
+            tmem_st16(tl + c0, v);
+            store_row16_bf16(mimg, row, c0, v);
+        }
+        float z = 0.f;
+        if (RELU && p.z_in && live) z = p.z_in[(size_t)bh * D + row];
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(mready);
+
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true;     // every epilogue warp runs every named barrier, even after an abort
+        for (int f = 0; f < F; ++f) {
+            const size_t frame = (size_t)bh * F + f;
+            ok = ok && mbar_wait(&full[s], ph, ab, 0x204);
+            if (!RELU) ok = ok && mbar_wait(mdone, f & 1, ab, 0x205);
+            tc_fence_after();
+            const float al = RELU ? 1.f : p.alpha[frame];
+            const uint8_t* st = ring + s * kStage;
+            const float* bq = reinterpret_cast<const float*>(st + (RELU ? 0 : kImg));
+            if (issuer && p.want_output) bulk_wait_read<0>();   // image free for rewriting
+            named_bar_sync(1, kEpiThreads);
+            const bool last = (f == F - 1);
+            for (int c0 = 0; c0 < D && ok; c0 += 16) {
+                float v[16];
+                tmem_ld16(tl + c0, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 b = *reinterpret_cast<const float4*>(bq + ((c0 / 4 + u) * 128 + row) * 4);
+                    v[4 * u] = fmaf(al, v[4 * u], b.x);
+                    v[4 * u + 1] = fmaf(al, v[4 * u + 1], b.y);
+                    v[4 * u + 2] = fmaf(al, v[4 * u + 2], b.z);
+                    v[4 * u + 3] = fmaf(al, v[4 * u + 3], b.w);
+                }
+                tmem_st16(tl + c0, v);
+                store_row16_bf16(mimg, row, c0, v);
+                if (last && p.state_out && live)
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        *reinterpret_cast<float4*>(p.state_out + ((size_t)bh * D + row) * D + c0 + 4 * u) =
+                            make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+            }
+            if (RELU && ok) {
+                z += reinterpret_cast<const float*>(st + kQuadMat)[row];
+                if (p.want_output) p.zf[frame * 128 + row] = z;
+                if (last && p.z_out && live) p.z_out[(size_t)bh * D + row] = z;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);     // this warp is done with stage s
+            tmem_wait_st();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(1, kEpiThreads);
+            if (issuer && p.want_output && ok) {
+                bulk_store(p.mimg + frame * kImg, mimg, kImg);
+                bulk_commit();
+            }
+            if (lane == 0) mbar_arrive(mready);
+            if (++s == kCStages) { s = 0; ph ^= 1; }
+        }
+        if (issuer) bulk_wait_all<0>();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tM, 128);
+}
+
+// ============================================================================
+// output: O_f = Q~_f bf16(M_f)   (ReLU: / (phi(Q_f) z_f + eps))
+// ============================================================================
+// warp 0: producer (M image + z by bulk copy, Q tiles by TMA); warp 1: TMEM
+// owner + MMA issuer; warps 2-5: epilogue (TMEM -> bf16 -> TMA store);
+// warps 6-9 (ReLU): phi(Q) in place and the per-token denominators.
+template <bool RELU>
+__global__ void __launch_bounds__(RELU ? 320 : 192, 1)
+tc_output_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapQ,
+                 const __grid_constant__ CUtensorMap mapO) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* qring = smem;                             // kOStages x 32 KB
+    uint8_t* mbuf = qring + kOStages * 32768;          // 2 x 32 KB M images
+    uint8_t* ostage = mbuf + 2 * kImg;                 // 2 x 32 KB output staging
+    float* zbuf = reinterpret_cast<float*>(ostage + 2 * 32768);   // 2 x 128
+    float* denbuf = zbuf + 2 * 128;                                // kOAcc x 128
+    uint64_t* qfull = reinterpret_cast<uint64_t*>(denbuf + kOAcc * 128);
+    uint64_t* qempty = qfull + kOStages;
+    uint64_t* xform = qempty + kOStages;
+    uint64_t* mfull = xform + kOStages;
+    uint64_t* mempty = mfull + 2;
+    uint64_t* accfull = mempty + 2;
+    uint64_t* accempty = accfull + kOAcc;
+    uint64_t* denready = accempty + kOAcc;     // ReLU denominators of a slot written
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(denready + kOAcc);
+    uint32_t* abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kOStages; ++s) {
+            mbar_init(&qfull[s], 1);
+            mbar_init(&qempty[s], 1);
+            mbar_init(&xform[s], 4);
+        }
+        for (int m = 0; m < 2; ++m) {
+            mbar_init(&mfull[m], 1);
+            mbar_init(&mempty[m], RELU ? 5 : 1);
+        }
+        for (int a = 0; a < kOAcc; ++a) {
+            mbar_init(&accfull[a], 1);
+            mbar_init(&accempty[a], 4);
+            mbar_init(&denready[a], 4);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    const Abort ab{abort_flag, p.status};
+    const int nitems = p.BH * p.F;
+    const int nt = (p.S + kTokO - 1) / kTokO;
+    const int D = p.D;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&mapQ);
+            tma_prefetch_desc(&mapO);
+            const uint64_t pol = policy_evict_first();
+            int s = 0, li = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
+                const int mb = li & 1;
+                if (!(ok = mbar_wait(&mempty[mb], ((li >> 1) & 1) ^ 1, ab, 0x301))) break;
+                mbar_expect_tx(&mfull[mb], kImg + (RELU ? 512 : 0));
+                bulk_load(mbuf + mb * kImg, p.mimg + (size_t)item * kImg, kImg, &mfull[mb]);
+                if (RELU) bulk_load(zbuf + mb * 128, p.zf + (size_t)item * 128, 512, &mfull[mb]);
+                for (int t = 0; t < nt; ++t) {
+                    if (!(ok = mbar_wait(&qempty[s], ph ^ 1, ab, 0x302))) break;
+                    uint8_t* st = qring + s * 32768;
+                    mbar_expect_tx(&qfull[s], 2 * kBoxO);
+                    tma_load_3d(st, &mapQ, &qfull[s], 0, t * kTokO, item, pol);
+                    tma_load_3d(st + kBoxO, &mapQ, &qfull[s], 64, t * kTokO, item, pol);
+                    if (++s == kOStages) { s = 0; ph ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idO = idesc_bf16(128, D, false, true);
+            int s = 0, li = 0, gt = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
+                const int mb = li & 1;
+                if (!(ok = mbar_wait(&mfull[mb], (li >> 1) & 1, ab, 0x303))) break;
+                const uint32_t mimg_a = smem_u32(mbuf + mb * kImg);
+                for (int t = 0; t < nt; ++t, ++gt) {
+                    const int a = gt % kOAcc;
+                    if (!(ok = mbar_wait(&accempty[a], ((gt / kOAcc) & 1) ^ 1, ab, 0x304))) break;
+                    if (!(ok = mbar_wait(RELU ? &xform[s] : &qfull[s], ph, ab, 0x305))) break;
+                    tc_fence_after();
+                    const uint32_t qa = smem_u32(qring + s * 32768);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t ad = sdesc_sw128(qa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                        const uint64_t bd = sdesc_sw128(mimg_a + kk * 2048, 16384, 1024);
+                        mma_bf16(tbase + a * 128, ad, bd, idO, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&qempty[s]);
+                    mma_commit(&accfull[a]);
+                    if (++s == kOStages) { s = 0; ph ^= 1; }
+                }
+                if (ok) mma_commit(&mempty[mb]);
+            }
+        }
+    } else if (warp < 6) {
+        // ---------------- epilogue: TMEM -> bf16 -> TMA store ----------------
+        const int q = warp & 3, row = q * 32 + lane;
+        const bool issuer = (threadIdx.x == 64);
+        int gt = 0;
+        bool ok = true;     // every epilogue warp runs every named barrier, even after an abort
+        for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+            for (int t = 0; t < nt; ++t, ++gt) {
+                const int a = gt % kOAcc, ob = gt & 1;
+                ok = ok && mbar_wait(&accfull[a], (gt / kOAcc) & 1, ab, 0x306);
+                if (RELU) ok = ok && mbar_wait(&denready[a], (gt / kOAcc) & 1, ab, 0x30a);
+                tc_fence_after();
+                if (issuer) bulk_wait_read<1>();     // staging ob no longer read by its store
+                named_bar_sync(1, kEpiThreads);
+                uint8_t* os = ostage + ob * 32768;
+                const float inv = (RELU && ok) ? 1.f / denbuf[a * 128 + row] : 1.f;
+                const uint32_t tl = tbase + (uint32_t(q * 32) << 16) + a * 128;
+                for (int c0 = 0; c0 < D && ok; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tl + c0, v);
+                    tmem_wait_ld();
+                    if (RELU) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] *= inv;
+                    }
+                    store_row16_bf16(os, row, c0, v);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&accempty[a]);
+                fence_proxy_async_smem();
+                named_bar_sync(1, kEpiThreads);
+                if (issuer && ok) {
+                    tma_store_3d(&mapO, os, 0, t * kTokO, item);
+                    if (D > 64) tma_store_3d(&mapO, os + kBoxO, 64, t * kTokO, item);
+                    bulk_commit();
+                }
+            }
+        }
+        if (issuer) bulk_wait_all<0>();
+    } else {
+        // ---------------- ReLU: phi(Q) in place, denominators ----------------
+        const int row = threadIdx.x - 192;                // token row in the tile
+        int s = 0, li = 0, gt = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
+            const int mb = li & 1;
+            if (!(ok = mbar_wait(&mfull[mb], (li >> 1) & 1, ab, 0x307))) break;
+            const float* z = zbuf + mb * 128;
+            for (int t = 0; t < nt; ++t, ++gt) {
+                const int a = gt % kOAcc;
+                if (!(ok = mbar_wait(&qfull[s], ph, ab, 0x308))) break;
+                if (!(ok = mbar_wait(&accempty[a], ((gt / kOAcc) & 1) ^ 1, ab, 0x309))) break;
+                uint8_t* st = qring + s * 32768;
+                float den = 0.f;
+                for (int blk = 0; blk < 2; ++blk) {
+                    if (blk * 64 >= D) break;
+                    for (int c = 0; c < 8; ++c) {
+                        uint4* pch = reinterpret_cast<uint4*>(st + blk * 16384 + sw128_off(row, c));
+                        uint4 x = *pch;
+                        x.x = relu_bf16x2(x.x); x.y = relu_bf16x2(x.y);
+                        x.z = relu_bf16x2(x.z); x.w = relu_bf16x2(x.w);
+                        *pch = x;
+                        const float* zz = z + blk * 64 + c * 8;
+                        den = fmaf(bf16_lo(x.x), zz[0], den);
+                        den = fmaf(bf16_hi(x.x), zz[1], den);
+                        den = fmaf(bf16_lo(x.y), zz[2], den);
+                        den = fmaf(bf16_hi(x.y), zz[3], den);
+                        den = fmaf(bf16_lo(x.z), zz[4], den);
+                        den = fmaf(bf16_hi(x.z), zz[5], den);
+                        den = fmaf(bf16_lo(x.w), zz[6], den);
+                        den = fmaf(bf16_hi(x.w), zz[7], den);
+                    }
+                }
+                denbuf[a * 128 + row] = den + p.eps;
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&xform[s]);
+                    mbar_arrive(&denready[a]);
+                }
+                if (++s == kOStages) { s = 0; ph ^= 1; }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&mempty[mb]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tbase, 512);
+}
+
+// ----------------------------------------------------------------------------
+// Host side
+// ----------------------------------------------------------------------------
+struct WsLayout {
+    size_t gimg, bmat, mimg, dz, zf, total;
+};
+
+WsLayout ws_layout(const ScanArgs& a) {
+    const size_t bhf = (size_t)a.B * a.H * a.F;
+    WsLayout L;
+    size_t off = kWsHeaderBytes;
+    L.gimg = off;
+    if (a.mode == LA_MODE_GDN) off += bhf * kImg;
+    L.bmat = off;
+    off += bhf * kQuadMat;
+    L.mimg = off;
+    off += bhf * kImg;
+    L.dz = off;
+    L.zf = off;
+    if (a.mode == LA_MODE_RELU) {
+        off += bhf * 512;
+        L.zf = off;
+        off += bhf * 512;
+    }
+    L.total = align_up(off, 256);
+    return L;
+}
+
+constexpr size_t smem_gram = 1024 + kGStages * 32768 + kImg + 2048 + 256;
+constexpr size_t smem_chain_gdn = 1024 + kCStages * (kImg + kQuadMat) + 1024 + kImg + 256;
+constexpr size_t smem_chain_relu = 1024 + kCStages * (kQuadMat + 512) + 1024 + kImg + 256;
+constexpr size_t smem_out = 1024 + kOStages * 32768 + 2 * kImg + 2 * 32768 +
+                            (2 + kOAcc) * 512 + 256;
+static_assert(smem_chain_gdn <= 232448, "chain smem");
+static_assert(smem_out <= 232448, "output smem");
+
+int sm_count() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+template <bool RELU>
+cudaError_t launch_tc_mode(const ScanArgs& a, cudaStream_t st) {
+    const WsLayout L = ws_layout(a);
+    uint8_t* ws = reinterpret_cast<uint8_t*>(a.ws);
+    TcParams p;
+    p.alpha = a.alpha;
+    p.beta = a.beta;
+    p.state_in = a.state_in;
+    p.z_in = a.z_in;
+    p.state_out = a.state_out;
+    p.z_out = a.z_out;
+    p.status = reinterpret_cast<unsigned int*>(ws);
+    p.gimg = ws + L.gimg;
+    p.bmat = reinterpret_cast<float*>(ws + L.bmat);
+    p.mimg = ws + L.mimg;
+    p.dz = reinterpret_cast<float*>(ws + L.dz);
+    p.zf = reinterpret_cast<float*>(ws + L.zf);
+    p.k_scale = a.k_scale;
+    p.eps = a.eps;
+    p.BH = a.B * a.H;
+    p.F = a.F;
+    p.S = a.S;
+    p.D = a.D;
+    p.want_output = a.o != nullptr;
+
+    const uint64_t bhf = (uint64_t)p.BH * p.F;
+    CUtensorMap mK, mV, mQ, mO;
+    if (!make_tmap_bf16_3d(&mK, a.k, a.D, a.S, bhf, 64, kTokG) ||
+        !make_tmap_bf16_3d(&mV, a.v, a.D, a.S, bhf, 64, kTokG))
+        return cudaErrorInvalidValue;
+    if (p.want_output && (!make_tmap_bf16_3d(&mQ, a.q, a.D, a.S, bhf, 64, kTokO) ||
+                          !make_tmap_bf16_3d(&mO, a.o, a.D, a.S, bhf, 64, kTokO)))
+        return cudaErrorInvalidValue;
+
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaFuncSetAttribute(tc_gram_kernel<RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem_gram);
+        cudaFuncSetAttribute(tc_chain_kernel<RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)(RELU ? smem_chain_relu : smem_chain_gdn));
+        cudaFuncSetAttribute(tc_output_kernel<RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem_out);
+        attr_done = true;
+    }
+    const int nsm = sm_count();
+    const int grid_f = (int)std::min<uint64_t>(bhf, (uint64_t)nsm);
+    const int thr = RELU ? 320 : 192;
+    tc_gram_kernel<RELU><<<grid_f, thr, smem_gram, st>>>(p, mK, mV);
+    tc_chain_kernel<RELU><<<p.BH, 192, RELU ? smem_chain_relu : smem_chain_gdn, st>>>(p);
+    if (p.want_output) tc_output_kernel<RELU><<<grid_f, thr, smem_out, st>>>(p, mQ, mO);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_eligible(const ScanArgs& a) {
+    return a.bf16 && a.D >= 64 && a.D <= 128 && a.F > 0;
+}
+
+size_t tc_workspace_bytes(const ScanArgs& a) { return ws_layout(a).total; }
+
+int tc_kernel_count(const ScanArgs& a) { return a.o ? 3 : 2; }
+
+cudaError_t launch_tc(const ScanArgs& a, cudaStream_t st) {
+    return a.mode == LA_MODE_RELU ? launch_tc_mode<true>(a, st) : launch_tc_mode<false>(a, st);
+}
+
+}  // namespace la

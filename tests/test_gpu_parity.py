@@ -133,8 +133,9 @@ def test_streaming_chunks_equal_single_scan():
 # ----------------------------------------------------------------------------
 @pytest.mark.parametrize("mode", ["relu", "gdn"])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("D,S,F", [(16, 1, 3), (48, 17, 2), (64, 130, 3), (112, 200, 2),
-                                   (128, 129, 3), (256, 70, 2)])
+@pytest.mark.parametrize("D,S,F", [(16, 1, 3), (48, 17, 2), (64, 130, 3), (80, 64, 2),
+                                   (96, 300, 2), (112, 200, 2), (128, 129, 3), (128, 1, 4),
+                                   (256, 70, 2)])
 def test_small_shapes(mode, dtype, D, S, F):
     spec = synth.small(B=2, H=2, F=F, S=S, D=D, dtype=dtype, seed=D + S)
     _compare(spec, mode, with_state=True)
@@ -248,3 +249,26 @@ def test_rejects_host_and_overlapping_pointers():
     la.la_scan_gdn(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], 0.1, workspace=ws)
     assert la.la_query_device_status(ws) == la.LA_OK
     del host
+
+
+# ----------------------------------------------------------------------------
+# Both kernel paths agree (tensor-core path vs the float32 SIMT path)
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("mode", ["relu", "gdn"])
+def test_tensor_core_path_matches_simt_path(mode, monkeypatch):
+    spec = synth.small(B=1, H=3, F=5, S=333, D=128, dtype="bf16", seed=31, keys_l2=True)
+    assert la.la_plan(la.LA_MODE_GDN if mode == "gdn" else la.LA_MODE_RELU, la.LA_BF16,
+                      1, 3, 5, 333, 128)[0] == "tcgen05"
+    inp = device_inputs(spec)
+    o_tc, m_tc, _ = _run(spec, mode, inp)
+    monkeypatch.setenv("LA_SCAN_FORCE_SIMT", "1")
+    o_simt, m_simt, _ = _run(spec, mode, inp)
+    torch.cuda.synchronize()
+    assert rel_err(to_np(o_tc), to_np(o_simt)) <= TOL_BF16
+    assert rel_err(to_np(m_tc), to_np(m_simt)) <= TOL_BF16
+
+
+def test_plan_of_the_workloads():
+    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05", 3)
+    assert la.la_plan(la.LA_MODE_RELU, la.LA_BF16, 1, 20, 21, 1560, 112) == ("tcgen05", 3)
+    assert la.la_plan(la.LA_MODE_GDN, la.LA_F32, 1, 2, 8, 64, 32)[0] == "simt_f32"
