@@ -135,6 +135,45 @@ LA_API la_status la_state_step(la_mode mode, const void* k, const void* v, la_dt
                         int B, int H, int F, int S, int D,
                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * Frame-wise GDN scan for callers that cannot allocate device memory.
+ * No counterpart in the pages: it is the same computation as la_scan_gdn,
+ * but its scratch is a fixed area built into the library instead of a
+ * caller-provided workspace.  It exists for callers that cannot call
+ * cudaMalloc: for example a plug-in running inside a host framework that
+ * owns every device allocation and gives its plug-ins no scratch memory, or
+ * a real-time loop whose rules forbid cudaMalloc/cudaFree because they
+ * synchronise the device and can fail mid-run.
+ *
+ * Arguments, layouts and errors are those of la_scan_gdn; there is no
+ * workspace argument.  The caller still owns and passes every input and
+ * output.  This entry point calls no cudaMalloc, cudaFree or other
+ * allocating routine.
+ *
+ * Scratch.  A __device__ array of LA_NOALLOC_SCRATCH_BYTES (64 MiB) that
+ *   every GPU which loads the library holds until the process exits.  A call
+ *   whose la_workspace_size(LA_MODE_GDN, B, H, F, S, D) exceeds it returns
+ *   LA_ERR_UNSUPPORTED before enqueuing anything (for bf16 inputs with
+ *   64 <= D <= 128 that is B*H*F > 511 frames; D > 128 needs only a few
+ *   bytes).
+ * Sharing.  All calls on a device share the one array, and it keeps the
+ *   last call's contents; the library clears what must start at zero at the
+ *   start of every call.  Calls whose GPU work overlaps (on different
+ *   streams, or from different threads) race on the array and give wrong
+ *   results: serialise them, for example on one stream.
+ * Set-up.  The first call on each device looks up the array's device
+ *   address (cudaGetSymbolAddress) with that device current; make that first
+ *   call before any stream capture begins.
+ * Status.  la_query_device_status is not available for this entry point
+ *   (the caller has no workspace pointer); device-side timeouts surface as
+ *   invalid outputs only.
+ */
+#define LA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+LA_API la_status la_scan_gdn_noalloc(const void* q, const void* k, const void* v, void* o,
+                                     la_dtype dt, const float* alpha, const float* beta,
+                                     float k_scale, const float* state_in, float* state_out,
+                                     int B, int H, int F, int S, int D, cudaStream_t stream);
+
 /* Workspace bytes a call of this mode and shape needs (either dtype).
  * Returns 0 for an unsupported shape.  The library has no counterpart in
  * the pages; it exists because the library never allocates. */

@@ -20,7 +20,7 @@ def declared_symbols():
 def test_header_declares_the_abi():
     assert declared_symbols() == sorted([
         "la_scan_relu", "la_scan_gdn", "la_state_step", "la_workspace_size",
-        "la_query_device_status", "la_status_string", "la_plan"])
+        "la_query_device_status", "la_status_string", "la_plan", "la_scan_gdn_noalloc"])
 
 
 def test_library_exports_every_declared_symbol():
