@@ -154,8 +154,8 @@ LA_API la_status la_state_step(la_mode mode, const void* k, const void* v, la_dt
  *   every GPU which loads the library holds until the process exits.  A call
  *   whose la_workspace_size(LA_MODE_GDN, B, H, F, S, D) exceeds it returns
  *   LA_ERR_UNSUPPORTED before enqueuing anything (for bf16 inputs with
- *   64 <= D <= 128 that is B*H*F > 511 frames; D > 128 needs only a few
- *   bytes).
+ *   64 <= D <= 128 the scan needs about 1 MiB per (b, h) pair, so up to
+ *   B*H = 63; D > 128 and float32 inputs need only a few bytes).
  * Sharing.  All calls on a device share the one array, and it keeps the
  *   last call's contents; the library clears what must start at zero at the
  *   start of every call.  Calls whose GPU work overlaps (on different

@@ -65,4 +65,9 @@ size_t tc_workspace_bytes(const ScanArgs& a);
 int tc_kernel_count(const ScanArgs& a);
 cudaError_t launch_tc(const ScanArgs& a, cudaStream_t st);
 
+// Fused persistent tensor-core path (one cooperative launch).
+bool fused_eligible(const ScanArgs& a);
+size_t fused_workspace_bytes(const ScanArgs& a);
+cudaError_t launch_fused(const ScanArgs& a, cudaStream_t st);
+
 }  // namespace la

@@ -57,7 +57,15 @@ bool force_simt() {
 
 bool use_tc(const ScanArgs& a) { return !force_simt() && tc_eligible(a); }
 
+// LA_SCAN_NO_FUSE=1 keeps tensor-core calls on the three-kernel path (tests
+// compare the two).
+bool use_fused(const ScanArgs& a) {
+    const char* e = std::getenv("LA_SCAN_NO_FUSE");
+    return use_tc(a) && !(e && e[0] == '1') && fused_eligible(a);
+}
+
 size_t workspace_needed(const ScanArgs& a) {
+    if (use_fused(a)) return fused_workspace_bytes(a);
     return use_tc(a) ? tc_workspace_bytes(a) : simt_workspace_bytes(a);
 }
 
@@ -99,7 +107,9 @@ la_status run(const ScanArgs& a, cudaStream_t st) {
         cudaGetLastError();
         return LA_ERR_CUDA;
     }
-    cudaError_t e = use_tc(a) ? launch_tc(a, st) : launch_simt(a, st);
+    cudaError_t e = use_fused(a) ? launch_fused(a, st)
+                    : use_tc(a)  ? launch_tc(a, st)
+                                 : launch_simt(a, st);
     if (e != cudaSuccess) { cudaGetLastError(); return LA_ERR_CUDA; }
     return LA_OK;
 }
@@ -200,6 +210,10 @@ extern "C" const char* la_plan(la_mode mode, la_dtype dt, int B, int H, int F, i
     ScanArgs a = base_args(nullptr, nullptr, dt, B, H, F, S, D, nullptr, 0);
     a.mode = mode;
     a.o = reinterpret_cast<void*>(uintptr_t(1));    // a scan (with outputs)
+    if (use_fused(a)) {
+        if (kernels) *kernels = 1;
+        return "tcgen05_fused";
+    }
     if (use_tc(a)) {
         if (kernels) *kernels = tc_kernel_count(a);
         return "tcgen05";

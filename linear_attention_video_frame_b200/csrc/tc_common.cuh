@@ -68,18 +68,24 @@ struct Abort {
 };
 
 // Wait until the phase of `bar` with parity `parity` has completed.  Returns
-// false (and raises the block's abort flag) after kWaitLimitNs, or at once if
-// another thread of the block already gave up.
+// false (and raises the block's abort flag) after kWaitLimitNs, or soon after
+// another thread of the block, or another block of the launch, gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Abort& ab,
                                           uint32_t where) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
-    while (true) {
+    for (uint32_t it = 0;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if (ab.raised()) return false;
-        if (global_timer_ns() - t0 > kWaitLimitNs) {
-            ab.raise(where);
-            return false;
+        if ((it & 15) == 15) {
+            if (*reinterpret_cast<volatile unsigned int*>(ab.status) != 0) {
+                *ab.flag = 1;
+                return false;
+            }
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                ab.raise(where);
+                return false;
+            }
         }
     }
 }
@@ -266,6 +272,90 @@ __host__ __device__ __forceinline__ uint32_t sw128_off(uint32_t r, uint32_t c) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Barrier over a subset of the block's warps (id 1..15, n a multiple of 32).
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// ReLU of two packed bf16 values: clear every element whose sign bit is set.
+__device__ __forceinline__ uint32_t relu_bf16x2(uint32_t w) {
+    const uint32_t m = ((w >> 15) & 0x00010001u) * 0xFFFFu;
+    return w & ~m;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Write 16 consecutive columns [c0, c0+16) of row `row` of a two-block
+// (2 x 64 columns) 128B-swizzled bf16 image.
+__device__ __forceinline__ void store_row16_bf16(uint8_t* img, int row, int c0,
+                                                 const float (&v)[16]) {
+    const int blk = c0 >> 6, ch = (c0 & 63) >> 3;
+    uint4 a = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                         pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+    uint4 b = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
+                         pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+    *reinterpret_cast<uint4*>(img + blk * 16384 + sw128_off(row, ch)) = a;
+    *reinterpret_cast<uint4*>(img + blk * 16384 + sw128_off(row, ch + 1)) = b;
+}
+
+// ----------------------------------------------------------------------------
+// Inter-block hand-off through global memory
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Order this thread's async-proxy (bulk copy) global accesses with its
+// generic-proxy ones.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// 16-byte load that is served by L2 (never a possibly stale L1 line).
+__device__ __forceinline__ float4 ld_cg_f4(const float* p) {
+    float4 v;
+    asm volatile("ld.global.cg.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
+    return v;
+}
+__device__ __forceinline__ float ld_cg_f32(const float* p) {
+    float v;
+    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+
+// Spin until *flag >= target (acquire).  Gives up after kWaitLimitNs, or as
+// soon as this block or any other block of the launch has given up (the
+// status word in global memory is non-zero).
+__device__ __forceinline__ bool wait_flag_ge(const uint32_t* flag, uint32_t target,
+                                             const Abort& ab, uint32_t where) {
+    if (ld_acquire_gpu(flag) >= target) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 0;; ++it) {
+        if (ld_acquire_gpu(flag) >= target) return true;
+        if (ab.raised()) return false;
+        if ((it & 63) == 63) {
+            if (*reinterpret_cast<volatile unsigned int*>(ab.status) != 0) {
+                *ab.flag = 1;
+                return false;
+            }
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                ab.raise(where);
+                return false;
+            }
+        }
+        __nanosleep(64);
+    }
 }
 
 }  // namespace tc

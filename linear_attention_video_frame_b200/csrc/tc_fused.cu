@@ -1,0 +1,1037 @@
+// Fused persistent tensor-core scan (bf16, 64 <= D <= 128): one cooperative
+// launch in which the sequential per-head recurrence runs concurrently with
+// the frame-parallel streaming work, handing per-frame operands through small
+// L2-resident rings instead of HBM round trips.
+//
+// Roles (one block per SM, all blocks co-resident):
+//   chain blocks  (blockIdx < n_chain): each owns up to 4 heads and advances
+//     them frame by frame, interleaved.  The fp32 state of each head lives in
+//     tensor memory; per frame
+//        GDN : M_f = alpha_f (M_{f-1} - G'_f bf16(M_{f-1})) + B_f
+//              (negated-A tcgen05 MMA accumulated onto the state)
+//        ReLU: M_f = M_{f-1} + dM_f,  z_f = z_{f-1} + dz_f
+//     and publishes bf16(M_f) as an MMA operand image.
+//   worker blocks (the rest): take items in ticket order from a global
+//     counter.  A gram item (b,h,f) streams K_f, V_f and produces G'_f, B_f
+//     (GDN) or dM_f, dz_f (ReLU); an output item (b,h,f) streams Q_f and
+//     produces O_f = Q~_f bf16(M_f) (ReLU: / (phi(Q_f) z_f + eps)).
+//
+// Ordering and progress.  Tickets list, for frame step j, the gram items of
+// frame j of every head and then the output items of frame j - lag.  A gram
+// item waits only for its ring slot to be consumed by the chain; an output
+// item waits only for the chain to publish its frame.  Every wait is on an
+// item with a smaller ticket or on a chain block, and chain blocks are always
+// resident, so the smallest unfinished ticket can always proceed.
+//
+// Hand-off protocol (per head, ring of kRG / kRM slots):
+//   gram  -> chain : G' image (bulk store), B_f (plain stores), then
+//                    gram_ready[slot] = f + 1 (release)
+//   chain -> output: M image (bulk store), then chain_done[head] = f + 1
+//   output -> chain: mimg_consumed[slot] = f + 1 once the image is in smem
+//   chain -> gram  : chain_done[head] >= f - kRG + 1 frees gram slot f
+// Every spin is bounded; a block that gives up records LA_ERR_TIMEOUT in the
+// status word, which makes every other block give up too.
+//
+// This is the frame-wise Gated DeltaNet of the SANA-WM paper summary
+// (section 3, "Hybrid GDN/Softmax Attention") in its affine form, and the
+// block-causal ReLU linear attention of the SANA-Video talk (block KV cache
+// segment); the cross-block hand-off of per-frame affine summaries mirrors
+// the composite exchange of the paper's context-parallel training (appendix
+// C.1), applied between blocks of one GPU.
+#include <algorithm>
+#include <cstdlib>
+
+#include "tc_common.cuh"
+#include "tmap.cuh"
+
+namespace la {
+namespace {
+
+using namespace tc;
+
+constexpr int kRG = 16;                 // per-head ring slots: gram -> chain
+constexpr int kRM = 16;                 // per-head ring slots: chain -> output
+constexpr int kWStages = 4;             // worker TMA ring (32 KB stages)
+constexpr int kCStages = 2;             // chain operand ring depth
+constexpr int kIQ = 4;                  // worker item queue depth
+constexpr int kThreads = 352;           // 11 warps
+constexpr int kTokG = 64, kTokO = 128;
+constexpr uint32_t kBoxG = 64 * kTokG * 2;   // 8 KB
+constexpr uint32_t kBoxO = 64 * kTokO * 2;   // 16 KB
+constexpr uint32_t kImg = 32768;             // bf16 128 x 128 operand image
+
+enum : int { kItemStop = 0, kItemGram = 1, kItemOut = 2 };
+
+// Optional event trace (built only with -DLA_TRACE, for tuning).  Each
+// writer (block, role) owns a region of kTraceCap records of two 64-bit
+// words {kind << 56 | block << 40 | aux, %globaltimer}; plain stores only.
+#ifdef LA_TRACE
+constexpr uint32_t kTraceCap = 4096;
+__device__ unsigned long long* g_trace = nullptr;
+__device__ __forceinline__ void trace_event(uint32_t& n, uint32_t writer, uint32_t kind, uint64_t aux) {
+    unsigned long long* t = g_trace;
+    if (!t || n >= kTraceCap) return;
+    unsigned long long* r = t + 2 * ((size_t)(blockIdx.x * 2 + writer) * kTraceCap + n++);
+    r[0] = ((uint64_t)kind << 56) | ((uint64_t)blockIdx.x << 40) | (aux & 0xFFFFFFFFFFull);
+    r[1] = global_timer_ns();
+}
+#define LA_TRACE_EVENT(kind, aux) trace_event(trace_n, trace_w, (kind), (aux))
+#define LA_TRACE_WRITER(w) uint32_t trace_n = 0; const uint32_t trace_w = (w)
+#else
+#define LA_TRACE_EVENT(kind, aux) ((void)0)
+#define LA_TRACE_WRITER(w) ((void)0)
+#endif
+struct Item {
+    int type, bh, f, pad;
+};
+
+struct FusedParams {
+    const float* alpha;
+    const float* beta;
+    const float* state_in;
+    const float* z_in;
+    float* state_out;
+    float* z_out;
+    unsigned int* status;      // header: [0] status, [1] where, [2] ticket
+    uint32_t* chain_done;      // [BH]
+    uint32_t* gram_ready;      // [BH][kRG]
+    uint32_t* mimg_consumed;   // [BH][kRM]
+    uint8_t* gimg;             // [BH][kRG] x kImg  -alpha beta kappa^2 K^T K   (GDN)
+    uint8_t* bimg;             // [BH][kRG] x kImg  beta kappa K^T V  /  phi(K)^T V
+    float* dz;                 // [BH][kRG] x 128   phi(K)^T 1                    (ReLU)
+    uint8_t* mimg;             // [BH][kRM] x kImg
+    float* zf;                 // [BH][kRM] x 128             (ReLU)
+    float k_scale;
+    float eps;
+    int BH, F, S, D;
+    int want_output;
+    int n_chain;
+    int heads_per_chain;
+    int lag;
+    int skip_publish;          // test hook: frame of head 0 whose gram_ready is never set
+};
+
+__device__ __forceinline__ Item decode_ticket(const FusedParams& p, uint32_t t) {
+    const uint32_t BH = p.BH, F = p.F;
+    Item it{kItemStop, 0, 0, 0};
+    if (!p.want_output) {
+        if (t < BH * F) it = Item{kItemGram, (int)(t % BH), (int)(t / BH), 0};
+        return it;
+    }
+    const uint32_t L = p.lag;
+    const uint32_t g0 = min(L, F) * BH;
+    if (t < g0) return Item{kItemGram, (int)(t % BH), (int)(t / BH), 0};
+    uint32_t u = t - g0;
+    const uint32_t nm = F > L ? F - L : 0;
+    if (u < nm * 2 * BH) {
+        const uint32_t j = L + u / (2 * BH), r = u % (2 * BH);
+        if (r < BH) return Item{kItemGram, (int)r, (int)j, 0};
+        return Item{kItemOut, (int)(r - BH), (int)(j - L), 0};
+    }
+    u -= nm * 2 * BH;
+    const uint32_t f0 = F > L ? F - L : 0;
+    if (u < (F - f0) * BH) return Item{kItemOut, (int)(u % BH), (int)(f0 + u / BH), 0};
+    return it;
+}
+
+// ============================================================================
+// worker blocks
+// ============================================================================
+template <bool RELU>
+__device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
+                                            const CUtensorMap* mK, const CUtensorMap* mV,
+                                            const CUtensorMap* mQ, const CUtensorMap* mO) {
+    uint8_t* ring = smem;                                  // kWStages x 32 KB
+    uint8_t* mbuf = ring + kWStages * 32768;               // M image of the current output item
+    uint8_t* stg = mbuf + kImg;                            // 2 x 16 KB epilogue staging
+    uint8_t* ones = stg + 2 * 16384;                       // 2 KB bf16 1.0 (ReLU)
+    float* zbuf = reinterpret_cast<float*>(ones + 2048);   // 128 (ReLU)
+    float* denbuf = zbuf + 128;                            // 4 x 128 (ReLU)
+    float* dzst = denbuf + 4 * 128;                        // 128: dz_f staging (ReLU)
+    Item* items = reinterpret_cast<Item*>(dzst + 128);
+    Item* bc_item = items + kIQ;                           // broadcast slots
+    int* bc_ok = reinterpret_cast<int*>(bc_item + 2);
+    uint64_t* full = reinterpret_cast<uint64_t*>(bc_ok + 4);
+    uint64_t* empty = full + kWStages;
+    uint64_t* xform = empty + kWStages;
+    uint64_t* mfull = xform + kWStages;
+    uint64_t* mempty = mfull + 1;
+    uint64_t* qfull = mempty + 1;
+    uint64_t* qempty = qfull + 4;
+    uint64_t* denready = qempty + 4;
+    uint64_t* iqfull = denready + 4;
+    uint64_t* iqempty = iqfull + kIQ;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(iqempty + kIQ);
+    uint32_t* abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kWStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&xform[s], 4);
+        }
+        mbar_init(mfull, 1);
+        mbar_init(mempty, RELU ? 5 : 1);
+        for (int q = 0; q < 4; ++q) {
+            mbar_init(&qfull[q], 1);
+            mbar_init(&qempty[q], 4);
+            mbar_init(&denready[q], 4);
+        }
+        for (int i = 0; i < kIQ; ++i) {
+            mbar_init(&iqfull[i], 1);
+            mbar_init(&iqempty[i], RELU ? 3 : 2);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (RELU)
+        for (int i = threadIdx.x; i < 2048 / 4; i += blockDim.x)
+            reinterpret_cast<uint32_t*>(ones)[i] = 0x3F803F80u;
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    const Abort ab{abort_flag, p.status};
+    const int F = p.F, D = p.D;
+    const int ntg = (p.S + kTokG - 1) / kTokG, nto = (p.S + kTokO - 1) / kTokO;
+
+    if (warp == 0) {
+        // ---------------- producer: tickets, dependencies, loads ----------------
+        if (lane == 0) {
+            tma_prefetch_desc(mK);
+            tma_prefetch_desc(mV);
+            if (p.want_output) {
+                tma_prefetch_desc(mQ);
+                tma_prefetch_desc(mO);
+            }
+            const uint64_t pol = policy_evict_first();
+            uint32_t iq = 0, nout = 0, ph = 0;
+            int s = 0;
+            bool ok = true;
+            LA_TRACE_WRITER(0);
+            while (true) {
+                Item it{kItemStop, 0, 0, 0};
+                if (ok) it = decode_ticket(p, atomicAdd(&p.status[2], 1u));
+                const int qi = iq % kIQ;
+                ok = ok && mbar_wait(&iqempty[qi], ((iq / kIQ) & 1) ^ 1, ab, 0x401);
+                if (!ok) it.type = kItemStop;
+                items[qi] = it;
+                mbar_arrive(&iqfull[qi]);
+                ++iq;
+                if (it.type == kItemStop) break;
+                const int frame = it.bh * F + it.f;
+                LA_TRACE_EVENT(it.type == kItemGram ? 1 : 2, frame);
+                if (it.type == kItemGram) {
+                    if (it.f >= kRG)
+                        ok = ok && wait_flag_ge(&p.chain_done[it.bh], it.f - kRG + 1, ab, 0x402);
+                    LA_TRACE_EVENT(3, frame);
+                    for (int t = 0; t < ntg; ++t) {
+                        ok = ok && mbar_wait(&empty[s], ph ^ 1, ab, 0x403);
+                        if (ok) {
+                            uint8_t* st = ring + s * 32768;
+                            mbar_expect_tx(&full[s], 4 * kBoxG);
+                            tma_load_3d(st, mK, &full[s], 0, t * kTokG, frame, pol);
+                            tma_load_3d(st + kBoxG, mK, &full[s], 64, t * kTokG, frame, pol);
+                            tma_load_3d(st + 16384, mV, &full[s], 0, t * kTokG, frame, pol);
+                            tma_load_3d(st + 16384 + kBoxG, mV, &full[s], 64, t * kTokG, frame, pol);
+                        }
+                        if (++s == kWStages) { s = 0; ph ^= 1; }
+                    }
+                } else {
+                    ok = ok && wait_flag_ge(&p.chain_done[it.bh], it.f + 1, ab, 0x404);
+                    LA_TRACE_EVENT(4, frame);
+                    fence_proxy_async_global();
+                    ok = ok && mbar_wait(mempty, (nout & 1) ^ 1, ab, 0x405);
+                    ++nout;
+                    if (ok) {
+                        const size_t ms = (size_t)it.bh * kRM + it.f % kRM;
+                        mbar_expect_tx(mfull, kImg + (RELU ? 512 : 0));
+                        bulk_load(mbuf, p.mimg + ms * kImg, kImg, mfull);
+                        if (RELU) bulk_load(zbuf, p.zf + ms * 128, 512, mfull);
+                    }
+                    for (int t = 0; t < nto; ++t) {
+                        ok = ok && mbar_wait(&empty[s], ph ^ 1, ab, 0x406);
+                        if (ok) {
+                            uint8_t* st = ring + s * 32768;
+                            mbar_expect_tx(&full[s], 2 * kBoxO);
+                            tma_load_3d(st, mQ, &full[s], 0, t * kTokO, frame, pol);
+                            tma_load_3d(st + kBoxO, mQ, &full[s], 64, t * kTokO, frame, pol);
+                        }
+                        if (++s == kWStages) { s = 0; ph ^= 1; }
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            const uint32_t idKK = idesc_bf16(128, D, true, true);
+            const uint32_t idZ = idesc_bf16(128, 16, true, false);
+            const uint32_t idO = idesc_bf16(128, D, false, true);
+            const uint64_t ones_d = sdesc_sw128(smem_u32(ones), 16, 1024);
+            uint32_t iq = 0, ph = 0, qctr = 0, nout = 0;
+            int s = 0;
+            bool ok = true;
+            while (ok) {
+                const int qi = iq % kIQ;
+                if (!(ok = mbar_wait(&iqfull[qi], (iq / kIQ) & 1, ab, 0x411))) break;
+                const Item it = items[qi];
+                mbar_arrive(&iqempty[qi]);
+                ++iq;
+                if (it.type == kItemStop) break;
+                if (it.type == kItemGram) {
+                    const uint32_t qa = qctr & 3, qb = (qctr + 1) & 3;
+                    ok = mbar_wait(&qempty[qa], ((qctr >> 2) & 1) ^ 1, ab, 0x412) &&
+                         mbar_wait(&qempty[qb], (((qctr + 1) >> 2) & 1) ^ 1, ab, 0x413);
+                    qctr += 2;
+                    if (!ok) break;
+                    tc_fence_after();
+                    const uint32_t dG = tbase + qa * 128, dW = tbase + qb * 128;
+                    for (int t = 0; t < ntg && ok; ++t) {
+                        if (!(ok = mbar_wait(RELU ? &xform[s] : &full[s], ph, ab, 0x414))) break;
+                        tc_fence_after();
+                        const uint32_t sk = smem_u32(ring + s * 32768), sv = sk + 16384;
+#pragma unroll
+                        for (int k = 0; k < kTokG / 16; ++k) {
+                            const uint64_t ad = sdesc_sw128(sk + k * 2048, kBoxG, 1024);
+                            const uint64_t bv = sdesc_sw128(sv + k * 2048, kBoxG, 1024);
+                            const uint32_t acc = (t | k) ? 1u : 0u;
+                            if (RELU) {
+                                mma_bf16(dW, ad, bv, idKK, acc);
+                                mma_bf16(dG, ad, ones_d, idZ, acc);
+                            } else {
+                                mma_bf16(dG, ad, ad, idKK, acc);
+                                mma_bf16(dW, ad, bv, idKK, acc);
+                            }
+                        }
+                        mma_commit(&empty[s]);
+                        if (++s == kWStages) { s = 0; ph ^= 1; }
+                    }
+                    if (!ok) break;
+                    mma_commit(&qfull[qa]);
+                    mma_commit(&qfull[qb]);
+                } else {
+                    if (!(ok = mbar_wait(mfull, nout & 1, ab, 0x415))) break;
+                    ++nout;
+                    // The image is in shared memory: its ring slot may be rewritten.
+                    st_release_gpu(&p.mimg_consumed[(size_t)it.bh * kRM + it.f % kRM], it.f + 1);
+                    const uint32_t mb = smem_u32(mbuf);
+                    for (int t = 0; t < nto && ok; ++t) {
+                        const uint32_t qa = qctr & 3;
+                        ok = mbar_wait(&qempty[qa], ((qctr >> 2) & 1) ^ 1, ab, 0x416) &&
+                             mbar_wait(RELU ? &xform[s] : &full[s], ph, ab, 0x417);
+                        ++qctr;
+                        if (!ok) break;
+                        tc_fence_after();
+                        const uint32_t qs = smem_u32(ring + s * 32768);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint64_t ad = sdesc_sw128(qs + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                            const uint64_t bd = sdesc_sw128(mb + kk * 2048, 16384, 1024);
+                            mma_bf16(tbase + qa * 128, ad, bd, idO, kk > 0 ? 1u : 0u);
+                        }
+                        mma_commit(&empty[s]);
+                        mma_commit(&qfull[qa]);
+                        if (++s == kWStages) { s = 0; ph ^= 1; }
+                    }
+                    if (!ok) break;
+                    mma_commit(mempty);
+                }
+            }
+        }
+    } else if (warp < 6) {
+        // ---------------- epilogue (4 warps; the leader waits, all follow) ----------------
+        const int q = warp & 3, row = q * 32 + lane;
+        const bool leader = (threadIdx.x == 64);
+        const uint32_t lanebase = uint32_t(q * 32) << 16;
+        uint32_t iq = 0, qctr = 0, sctr = 0;
+        uint32_t dpar = 0;    // bit q: parity of quarter q's next output-tile use (denready)
+        bool ok = true;
+        LA_TRACE_WRITER(1);
+        while (true) {
+            if (leader) {
+                const int qi = iq % kIQ;
+                Item it{kItemStop, 0, 0, 0};
+                ok = ok && mbar_wait(&iqfull[qi], (iq / kIQ) & 1, ab, 0x421);
+                if (ok) {
+                    it = items[qi];
+                    mbar_arrive(&iqempty[qi]);
+                }
+                bc_item[0] = it;
+            }
+            ++iq;
+            named_bar_sync(1, 128);
+            const Item it = bc_item[0];
+            if (it.type == kItemStop) break;
+            const int frame = it.bh * F + it.f;
+            const int nblk = D > 64 ? 2 : 1;
+            if (it.type == kItemGram) {
+                const uint32_t qa = qctr & 3, qb = (qctr + 1) & 3;
+                if (leader) {
+                    ok = ok && mbar_wait(&qfull[qa], (qctr >> 2) & 1, ab, 0x422) &&
+                         mbar_wait(&qfull[qb], ((qctr + 1) >> 2) & 1, ab, 0x423);
+                    if (RELU) bulk_wait_read<0>();     // dz staging free again
+                    *bc_ok = ok;
+                }
+                qctr += 2;
+                named_bar_sync(1, 128);
+                const bool go = *bc_ok;
+                tc_fence_after();
+                const size_t sidx = (size_t)it.bh * kRG + it.f % kRG;
+                // GDN: G'' = -alpha beta kappa^2 K^T K (A operand of the chain's MMA),
+                //      B~  = beta kappa K^T V (added by the chain through an identity MMA).
+                // ReLU: B~ = phi(K)^T V, and dz = phi(K)^T 1 in fp32.
+                const float al = RELU ? 1.f : p.alpha[frame];
+                const float bt = RELU ? 1.f : p.beta[frame];
+                const float sg = -al * bt * p.k_scale * p.k_scale;
+                const float sw = RELU ? 1.f : bt * p.k_scale;
+                for (int im = RELU ? 1 : 0; im < 2; ++im) {
+                    const uint32_t qq = im == 0 ? qa : qb;
+                    const float sc = im == 0 ? sg : sw;
+                    uint8_t* dst = (im == 0 ? p.gimg : p.bimg) + sidx * kImg;
+                    for (int blk = 0; blk < nblk; ++blk) {
+                        if (leader) bulk_wait_read<1>();
+                        named_bar_sync(1, 128);
+                        uint8_t* sb = stg + (sctr & 1) * 16384;
+                        ++sctr;
+                        if (go)
+                            for (int c0 = blk * 64; c0 < min(D, blk * 64 + 64); c0 += 16) {
+                                float v[16];
+                                tmem_ld16(tbase + lanebase + qq * 128 + c0, v);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int e = 0; e < 16; ++e) v[e] *= sc;
+                                store_row16_bf16(sb, row, c0 & 63, v);
+                            }
+                        fence_proxy_async_smem();
+                        named_bar_sync(1, 128);
+                        if (leader && go) {
+                            bulk_store(dst + blk * 16384, sb, 16384);
+                            bulk_commit();
+                        }
+                    }
+                }
+                if (RELU) {
+                    if (go) {
+                        float v[16];
+                        tmem_ld16(tbase + lanebase + qa * 128, v);
+                        tmem_wait_ld();
+                        dzst[row] = v[0];
+                    }
+                    fence_proxy_async_smem();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&qempty[qa]);
+                    mbar_arrive(&qempty[qb]);
+                }
+                named_bar_sync(1, 128);
+                if (leader && go) {
+                    if (RELU) {
+                        bulk_store(p.dz + sidx * 128, dzst, 512);
+                        bulk_commit();
+                    }
+                    bulk_wait_all<0>();
+                    fence_proxy_async_global();
+                    if (!(it.bh == 0 && it.f == p.skip_publish))
+                        st_release_gpu(&p.gram_ready[sidx], it.f + 1);
+                    LA_TRACE_EVENT(5, frame);
+                }
+            } else {
+                for (int t = 0; t < nto; ++t) {
+                    const uint32_t qa = qctr & 3;
+                    if (leader) {
+                        ok = ok && mbar_wait(&qfull[qa], (qctr >> 2) & 1, ab, 0x424);
+                        if (RELU) ok = ok && mbar_wait(&denready[qa], (dpar >> qa) & 1, ab, 0x425);
+                        *bc_ok = ok;
+                    }
+                    dpar ^= 1u << qa;
+                    ++qctr;
+                    named_bar_sync(1, 128);
+                    const bool go = *bc_ok;
+                    tc_fence_after();
+                    const float inv = (RELU && go) ? 1.f / denbuf[qa * 128 + row] : 1.f;
+                    // one 64-column block (16 KB) at a time through staging
+                    for (int blk = 0; blk < nblk; ++blk) {
+                        if (leader) bulk_wait_read<1>();
+                        named_bar_sync(1, 128);
+                        uint8_t* sb = stg + (sctr & 1) * 16384;
+                        ++sctr;
+                        if (go)
+                            for (int c0 = blk * 64; c0 < min(D, blk * 64 + 64); c0 += 16) {
+                                float v[16];
+                                tmem_ld16(tbase + lanebase + qa * 128 + c0, v);
+                                tmem_wait_ld();
+                                if (RELU) {
+#pragma unroll
+                                    for (int e = 0; e < 16; ++e) v[e] *= inv;
+                                }
+                                store_row16_bf16(sb, row, c0 & 63, v);
+                            }
+                        if (blk == nblk - 1) {
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&qempty[qa]);
+                        }
+                        fence_proxy_async_smem();
+                        named_bar_sync(1, 128);
+                        if (leader && go) {
+                            tma_store_3d(mO, sb, blk * 64, t * kTokO, frame);
+                            bulk_commit();
+                            if (t == nto - 1 && blk == nblk - 1) LA_TRACE_EVENT(6, frame);
+                        }
+                    }
+                }
+            }
+        }
+        if (leader) bulk_wait_all<0>();
+    } else if (RELU && warp < 10) {
+        // ---------------- ReLU transforms: phi(K), phi(Q) and denominators ----------------
+        const int tl = threadIdx.x - 192;          // 0..127
+        const bool leader = (tl == 0);
+        uint32_t iq = 0, qctr = 0, nout = 0, ph = 0, bcn = 0;
+        int s = 0;
+        bool ok = true;
+        // The leader's per-tile verdict alternates between two slots: with a
+        // single barrier per tile, a slow warp may still be reading the
+        // previous tile's slot when the leader writes the next one.
+        int* bc2 = bc_ok + 2;
+        while (true) {
+            if (leader) {
+                const int qi = iq % kIQ;
+                Item it{kItemStop, 0, 0, 0};
+                ok = ok && mbar_wait(&iqfull[qi], (iq / kIQ) & 1, ab, 0x431);
+                if (ok) {
+                    it = items[qi];
+                    mbar_arrive(&iqempty[qi]);
+                }
+                bc_item[1] = it;
+            }
+            ++iq;
+            named_bar_sync(2, 128);
+            const Item it = bc_item[1];
+            if (it.type == kItemStop) break;
+            if (it.type == kItemGram) {
+                qctr += 2;
+                for (int t = 0; t < ntg; ++t) {
+                    if (leader) {
+                        ok = ok && mbar_wait(&full[s], ph, ab, 0x432);
+                        bc2[bcn & 1] = ok;
+                    }
+                    named_bar_sync(2, 128);
+                    if (bc2[(bcn++) & 1]) {
+                        uint4* kt = reinterpret_cast<uint4*>(ring + s * 32768);
+                        for (int i = tl; i < 2 * (int)kBoxG / 16; i += 128) {
+                            uint4 x = kt[i];
+                            x.x = relu_bf16x2(x.x); x.y = relu_bf16x2(x.y);
+                            x.z = relu_bf16x2(x.z); x.w = relu_bf16x2(x.w);
+                            kt[i] = x;
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&xform[s]);
+                    if (++s == kWStages) { s = 0; ph ^= 1; }
+                }
+            } else {
+                if (leader) ok = ok && mbar_wait(mfull, nout & 1, ab, 0x433);
+                ++nout;
+                for (int t = 0; t < nto; ++t) {
+                    const uint32_t qa = qctr & 3;
+                    if (leader) {
+                        ok = ok && mbar_wait(&qempty[qa], ((qctr >> 2) & 1) ^ 1, ab, 0x434) &&
+                             mbar_wait(&full[s], ph, ab, 0x435);
+                        bc2[bcn & 1] = ok;
+                    }
+                    ++qctr;
+                    named_bar_sync(2, 128);
+                    if (bc2[(bcn++) & 1]) {
+                        uint8_t* st = ring + s * 32768;
+                        float den = 0.f;
+                        for (int blk = 0; blk < 2 && blk * 64 < D; ++blk) {
+                            for (int c = 0; c < 8; ++c) {
+                                uint4* pch = reinterpret_cast<uint4*>(st + blk * 16384 + sw128_off(tl, c));
+                                uint4 x = *pch;
+                                x.x = relu_bf16x2(x.x); x.y = relu_bf16x2(x.y);
+                                x.z = relu_bf16x2(x.z); x.w = relu_bf16x2(x.w);
+                                *pch = x;
+                                const float* zz = zbuf + blk * 64 + c * 8;
+                                den = fmaf(bf16_lo(x.x), zz[0], den);
+                                den = fmaf(bf16_hi(x.x), zz[1], den);
+                                den = fmaf(bf16_lo(x.y), zz[2], den);
+                                den = fmaf(bf16_hi(x.y), zz[3], den);
+                                den = fmaf(bf16_lo(x.z), zz[4], den);
+                                den = fmaf(bf16_hi(x.z), zz[5], den);
+                                den = fmaf(bf16_lo(x.w), zz[6], den);
+                                den = fmaf(bf16_hi(x.w), zz[7], den);
+                            }
+                        }
+                        denbuf[qa * 128 + tl] = den + p.eps;
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(&xform[s]);
+                        mbar_arrive(&denready[qa]);
+                    }
+                    if (++s == kWStages) { s = 0; ph ^= 1; }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(mempty);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tbase, 512);
+}
+
+// ============================================================================
+// chain blocks (one head each)
+// ============================================================================
+// warp 0: loader -- waits for the gram item of each frame and bulk-copies its
+//         G' image and B_f (ReLU: dz_f, dM_f) into a 2-stage ring, with alpha_f;
+// warp 1: TMEM owner + MMA issuer (GDN);
+// warps 2-9: epilogue -- thread <-> (state row, half of the columns);
+// warp 10: publisher -- stores bf16(M_f) (and z_f) to the head's ring slot once
+//         the slot is free, then releases chain_done.
+// The epilogue's critical path touches only shared and tensor memory.
+template <bool RELU>
+__device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) {
+    // stage s (64 KB): [0, 32 KB) G'' image (GDN) or dz_f (ReLU); [32 KB, 64 KB) B~ image
+    uint8_t* stage = smem;                                  // kCStages x 64 KB
+    uint8_t* ident = stage + kCStages * 2 * kImg;           // identity (K-major A operand)
+    uint8_t* imgs = ident + kImg;                           // 2 x 32 KB bf16 state images
+    float* alph = reinterpret_cast<float*>(imgs + 2 * kImg);   // [kCStages] alpha of the staged frame
+    uint64_t* gfull = reinterpret_cast<uint64_t*>(alph + 4);
+    uint64_t* gempty = gfull + kCStages;
+    uint64_t* mdone = gempty + kCStages;   // MMA of the frame finished
+    uint64_t* mready = mdone + 1;          // TMEM holds alpha_f M_{f-1}, image of M_{f-1} written
+    uint64_t* iready = mready + 1;         // [2] image buffer b holds a frame to publish
+    uint64_t* iread = iready + 2;          // [2] publisher has read image buffer b out
+    int* bc_ok = reinterpret_cast<int*>(iread + 2);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bc_ok + 2);
+    uint32_t* abort_flag = tmem_slot + 1;
+    float* zst = reinterpret_cast<float*>(stage + 8192);   // ReLU: [2][128] z_f staging
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.x;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kCStages; ++s) {
+            mbar_init(&gfull[s], 1);
+            mbar_init(&gempty[s], 2);     // the MMA and the epilogue leader
+        }
+        mbar_init(mdone, 1);
+        mbar_init(mready, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&iready[b], 1);
+            mbar_init(&iread[b], 1);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 128);
+        tmem_relinquish();
+    }
+    if (warp >= 2 && warp < 10)
+        for (int idx = threadIdx.x - 64; idx < 128 * 16; idx += 256) {
+            const int r = idx >> 4, blk = (idx >> 3) & 1, c = idx & 7;
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int k0 = blk * 64 + c * 8 + 2 * e;
+                w[e] = (k0 == r ? 0x3F80u : 0u) | (k0 + 1 == r ? 0x3F800000u : 0u);
+            }
+            *reinterpret_cast<uint4*>(ident + blk * 16384 + sw128_off(r, c)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tM = *tmem_slot;
+    const Abort ab{abort_flag, p.status};
+    const int F = p.F, D = p.D;
+
+    if (warp == 0) {
+        // ---------------- loader ----------------
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            LA_TRACE_WRITER(0);
+            for (int f = 0; f < F; ++f) {
+                const size_t sidx = (size_t)bh * kRG + f % kRG;
+                if (!wait_flag_ge(&p.gram_ready[sidx], f + 1, ab, 0x501)) break;
+                LA_TRACE_EVENT(10, (uint64_t)bh * F + f);
+                fence_proxy_async_global();
+                if (!mbar_wait(&gempty[s], ph ^ 1, ab, 0x502)) break;
+                uint8_t* st = stage + s * 2 * kImg;
+                alph[s] = RELU ? 1.f : p.alpha[(size_t)bh * F + f];
+                if (!RELU) {
+                    mbar_expect_tx(&gfull[s], 2 * kImg);
+                    bulk_load(st, p.gimg + sidx * kImg, kImg, &gfull[s]);
+                } else {
+                    mbar_expect_tx(&gfull[s], kImg + 512);
+                    bulk_load(st, p.dz + sidx * 128, 512, &gfull[s]);
+                }
+                bulk_load(st + kImg, p.bimg + sidx * kImg, kImg, &gfull[s]);
+                if (++s == kCStages) { s = 0; ph ^= 1; }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA: D = alpha M_{f-1} + G'' bf16(M_{f-1}) + I B~ ----------------
+        if (lane == 0) {
+            const uint32_t idM = idesc_bf16(128, D, false, true);
+            const uint32_t ia = smem_u32(ident);
+            int s = 0;
+            uint32_t ph = 0;
+            for (int f = 0; f < F; ++f) {
+                if (!mbar_wait(&gfull[s], ph, ab, 0x503)) break;
+                if (!mbar_wait(mready, f & 1, ab, 0x504)) break;
+                tc_fence_after();
+                const uint32_t sa = smem_u32(stage + s * 2 * kImg);
+                const uint32_t mb = smem_u32(imgs + ((f + 1) & 1) * kImg);   // image of M_{f-1}
+                if (!RELU)
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint64_t ad = sdesc_sw128(sa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                        const uint64_t bd = sdesc_sw128(mb + kk * 2048, 16384, 1024);
+                        mma_bf16(tM, ad, bd, idM, 1u);
+                    }
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t ad = sdesc_sw128(ia + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(sa + kImg + kk * 2048, 16384, 1024);
+                    mma_bf16(tM, ad, bd, idM, 1u);
+                }
+                mma_commit(mdone);
+                mma_commit(&gempty[s]);
+                if (++s == kCStages) { s = 0; ph ^= 1; }
+            }
+        }
+    } else if (warp < 10) {
+        // ---------------- epilogue: thread <-> (state row, column half) ----------------
+        const int q = warp & 3, row = q * 32 + lane, half = (warp - 2) >> 2;
+        const int c_lo = half * 64, c_hi = min(D, c_lo + 64);
+        const bool leader = (threadIdx.x == 64);
+        const uint32_t tl = tM + (uint32_t(q * 32) << 16);
+        const bool live = row < D;
+        LA_TRACE_WRITER(1);
+        // initial state: image of M_0 (buffer 1 = "frame -1") and TMEM alpha_0 M_0
+        if (leader) {
+            bc_ok[0] = F > 0 && mbar_wait(&gfull[0], 0, ab, 0x50c);
+        }
+        named_bar_sync(1, 256);
+        const float a0 = (!RELU && bc_ok[0]) ? alph[0] : 1.f;
+        float z = 0.f;
+        for (int c0 = c_lo; c0 < c_hi; c0 += 16) {
+            float v[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                v[e] = (p.state_in && live) ? p.state_in[((size_t)bh * D + row) * D + c0 + e] : 0.f;
+            store_row16_bf16(imgs + kImg, row, c0, v);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] *= a0;
+            tmem_st16(tl + c0, v);
+        }
+        if (RELU && half == 0 && p.z_in && live) z = p.z_in[(size_t)bh * D + row];
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        named_bar_sync(1, 256);
+        if (leader) mbar_arrive(mready);
+
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int f = 0; f < F; ++f) {
+            const int frame = bh * F + f;
+            const int ib = f & 1;
+            const int s_next = (s + 1 == kCStages) ? 0 : s + 1;
+            const uint32_t ph_next = (s + 1 == kCStages) ? (ph ^ 1) : ph;
+            const bool more = f + 1 < F;
+            if (leader) {
+                ok = ok && mbar_wait(mdone, f & 1, ab, 0x506);
+                // image buffer ib was last used by frame f - 2: read out by the publisher
+                if (f >= 2) ok = ok && mbar_wait(&iread[ib], ((f >> 1) - 1) & 1, ab, 0x507);
+                // alpha_{f+1} (GDN) arrives with the next frame's operands
+                if (!RELU && more) ok = ok && mbar_wait(&gfull[s_next], ph_next, ab, 0x505);
+                bc_ok[0] = ok;
+                LA_TRACE_EVENT(11, frame);
+            }
+            named_bar_sync(1, 256);
+            const bool go = bc_ok[0];
+            tc_fence_after();
+            if (go) {
+                const float an = (!RELU && more) ? alph[s_next] : 1.f;
+                uint8_t* img = imgs + ib * kImg;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int c0 = c_lo + 32 * hh;
+                    if (c0 < c_hi) {
+                        const bool two = c0 + 16 < c_hi;
+                        float v0[16], v1[16];
+                        tmem_ld16(tl + c0, v0);
+                        if (two) tmem_ld16(tl + c0 + 16, v1);
+                        tmem_wait_ld();
+                        store_row16_bf16(img, row, c0, v0);
+                        if (two) store_row16_bf16(img, row, c0 + 16, v1);
+                        if (!more && p.state_out && live) {
+                            float* so = p.state_out + ((size_t)bh * D + row) * D + c0;
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                *reinterpret_cast<float4*>(so + 4 * u) =
+                                    make_float4(v0[4 * u], v0[4 * u + 1], v0[4 * u + 2], v0[4 * u + 3]);
+                            if (two)
+#pragma unroll
+                                for (int u = 0; u < 4; ++u)
+                                    *reinterpret_cast<float4*>(so + 16 + 4 * u) =
+                                        make_float4(v1[4 * u], v1[4 * u + 1], v1[4 * u + 2], v1[4 * u + 3]);
+                        }
+                        if (!RELU && more) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                v0[e] *= an;
+                                v1[e] *= an;
+                            }
+                            tmem_st16(tl + c0, v0);
+                            if (two) tmem_st16(tl + c0 + 16, v1);
+                        }
+                    }
+                }
+                if (RELU && half == 0) {
+                    z += reinterpret_cast<const float*>(stage + s * 2 * kImg)[row];
+                    zst[ib * 128 + row] = z;
+                    if (!more && p.z_out && live) p.z_out[(size_t)bh * D + row] = z;
+                }
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(1, 256);
+            if (leader) {
+                mbar_arrive(&gempty[s]);
+                mbar_arrive(mready);
+                mbar_arrive(&iready[ib]);
+                LA_TRACE_EVENT(12, frame);
+            }
+            s = s_next;
+            ph = ph_next;
+        }
+    } else if (warp == 10) {
+        // ---------------- publisher ----------------
+        // Frame f's stores are issued as soon as its image is written; frame
+        // f - 1 is published (chain_done = f) once all but the newest store
+        // group have completed, so store latency never holds the image buffers.
+        if (lane == 0) {
+            int done = 0;
+            for (int f = 0; f < F; ++f) {
+                const int ib = f & 1;
+                const size_t msidx = (size_t)bh * kRM + f % kRM;
+                // the output item that last used this slot has read it (checked
+                // before the image is ready: it almost always already holds)
+                if (p.want_output && f >= kRM &&
+                    !wait_flag_ge(&p.mimg_consumed[msidx], f - kRM + 1, ab, 0x509))
+                    break;
+                if (!mbar_wait(&iready[ib], (f >> 1) & 1, ab, 0x508)) break;
+                if (p.want_output) {
+                    bulk_store(p.mimg + msidx * kImg, imgs + ib * kImg, kImg);
+                    if (RELU) bulk_store(p.zf + msidx * 128, zst + ib * 128, 512);
+                    bulk_commit();
+                    bulk_wait_read<0>();
+                }
+                mbar_arrive(&iread[ib]);
+                if (p.want_output) {
+                    if (f > 0) {
+                        bulk_wait_all<1>();
+                        fence_proxy_async_global();
+                        st_release_gpu(&p.chain_done[bh], f);
+                        done = f;
+                    }
+                } else {
+                    st_release_gpu(&p.chain_done[bh], f + 1);
+                    done = f + 1;
+                }
+            }
+            if (p.want_output && done < F && !ab.raised()) {
+                bulk_wait_all<0>();
+                fence_proxy_async_global();
+                st_release_gpu(&p.chain_done[bh], F);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tM, 128);
+}
+
+template <bool RELU>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_fused_kernel(const FusedParams p, const __grid_constant__ CUtensorMap mK,
+                const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mQ,
+                const __grid_constant__ CUtensorMap mO) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    if ((int)blockIdx.x < p.n_chain)
+        chain_role<RELU>(p, smem);
+    else
+        worker_role<RELU>(p, smem, &mK, &mV, &mQ, &mO);
+}
+
+// ----------------------------------------------------------------------------
+// Host side
+// ----------------------------------------------------------------------------
+struct FusedLayout {
+    size_t chain_done, gram_ready, mimg_consumed, flags_end;
+    size_t gimg, bimg, dz, mimg, zf, total;
+};
+
+FusedLayout fused_layout(const ScanArgs& a) {
+    const size_t bh = (size_t)a.B * a.H;
+    FusedLayout L;
+    size_t off = kWsHeaderBytes;
+    L.chain_done = off;
+    off += bh * 4;
+    L.gram_ready = off;
+    off += bh * kRG * 4;
+    L.mimg_consumed = off;
+    off += bh * kRM * 4;
+    off = align_up(off, 256);
+    L.flags_end = off;
+    L.gimg = off;
+    if (a.mode == LA_MODE_GDN) off += bh * kRG * kImg;
+    L.bimg = off;
+    off += bh * kRG * kImg;
+    L.dz = off;
+    if (a.mode == LA_MODE_RELU) off += bh * kRG * 512;
+    L.mimg = off;
+    off += bh * kRM * kImg;
+    L.zf = off;
+    if (a.mode == LA_MODE_RELU) off += bh * kRM * 512;
+    L.total = align_up(off, 256);
+    return L;
+}
+
+constexpr size_t kWorkerSmem = kWStages * 32768 + kImg + 2 * 16384 + 2048 + 512 + 2048 + 512 +
+                               (kIQ + 2) * sizeof(Item) + 16 +
+                               (3 * kWStages + 2 + 12 + 2 * kIQ) * 8 + 8;
+constexpr size_t kChainSmem = kCStages * 2 * kImg + kImg + 2 * kImg + 16 + 10 * 8 + 8 + 8;
+constexpr size_t kFusedSmem = 1024 + (kWorkerSmem > kChainSmem ? kWorkerSmem : kChainSmem);
+static_assert(kFusedSmem <= 232448, "fused kernel shared memory");
+
+int sm_count_fused() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+template <bool RELU>
+cudaError_t launch_fused_mode(const ScanArgs& a, cudaStream_t st) {
+    const FusedLayout L = fused_layout(a);
+    uint8_t* ws = reinterpret_cast<uint8_t*>(a.ws);
+    FusedParams p;
+    p.alpha = a.alpha;
+    p.beta = a.beta;
+    p.state_in = a.state_in;
+    p.z_in = a.z_in;
+    p.state_out = a.state_out;
+    p.z_out = a.z_out;
+    p.status = reinterpret_cast<unsigned int*>(ws);
+    p.chain_done = reinterpret_cast<uint32_t*>(ws + L.chain_done);
+    p.gram_ready = reinterpret_cast<uint32_t*>(ws + L.gram_ready);
+    p.mimg_consumed = reinterpret_cast<uint32_t*>(ws + L.mimg_consumed);
+    p.gimg = ws + L.gimg;
+    p.bimg = ws + L.bimg;
+    p.dz = reinterpret_cast<float*>(ws + L.dz);
+    p.mimg = ws + L.mimg;
+    p.zf = reinterpret_cast<float*>(ws + L.zf);
+    p.k_scale = a.k_scale;
+    p.eps = a.eps;
+    p.BH = a.B * a.H;
+    p.F = a.F;
+    p.S = a.S;
+    p.D = a.D;
+    p.want_output = a.o != nullptr;
+    p.lag = 10;
+    if (const char* e = std::getenv("LA_SCAN_LAG")) p.lag = std::max(1, std::min(std::atoi(e), kRG + kRM - 1));
+    p.skip_publish = -1;
+    if (const char* e = std::getenv("LA_SCAN_TEST_SKIP_PUBLISH")) p.skip_publish = std::atoi(e);
+    const int nsm = sm_count_fused();
+    p.n_chain = p.BH;                 // one chain block per (b, h)
+    p.heads_per_chain = 1;
+    if (p.n_chain >= nsm || 2ull * p.BH * p.F >= (1ull << 31)) return cudaErrorInvalidValue;
+
+    const uint64_t bhf = (uint64_t)p.BH * p.F;
+    CUtensorMap mK, mV, mQ, mO;
+    if (!make_tmap_bf16_3d(&mK, a.k, a.D, a.S, bhf, 64, kTokG) ||
+        !make_tmap_bf16_3d(&mV, a.v, a.D, a.S, bhf, 64, kTokG))
+        return cudaErrorInvalidValue;
+    if (p.want_output) {
+        if (!make_tmap_bf16_3d(&mQ, a.q, a.D, a.S, bhf, 64, kTokO) ||
+            !make_tmap_bf16_3d(&mO, a.o, a.D, a.S, bhf, 64, kTokO))
+            return cudaErrorInvalidValue;
+    } else {
+        mQ = mK;
+        mO = mK;
+    }
+    // flags and counters start at zero
+    cudaError_t e = cudaMemsetAsync(a.ws, 0, L.flags_end, st);
+    if (e != cudaSuccess) return e;
+
+    static bool attr_done = false;
+    if (!attr_done) {
+        e = cudaFuncSetAttribute(tc_fused_kernel<RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kFusedSmem);
+        if (e != cudaSuccess) return e;
+        attr_done = true;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(nsm);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kFusedSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, tc_fused_kernel<RELU>, p, mK, mV, mQ, mO);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+#ifdef LA_TRACE
+extern "C" __attribute__((visibility("default"))) int la_trace_install(void* buf) {
+    unsigned long long* p = reinterpret_cast<unsigned long long*>(buf);
+    return (int)cudaMemcpyToSymbol(g_trace, &p, sizeof(p));
+}
+#endif
+
+// One chain block per (b, h) pair, at most a third of the SMs, so that at
+// least two thirds of them stream.
+bool fused_eligible(const ScanArgs& a) {
+    if (!tc_eligible(a)) return false;
+    const int nsm = sm_count_fused();
+    return (long)a.B * a.H <= (long)(nsm / 3);
+}
+
+size_t fused_workspace_bytes(const ScanArgs& a) { return fused_layout(a).total; }
+
+cudaError_t launch_fused(const ScanArgs& a, cudaStream_t st) {
+    return a.mode == LA_MODE_RELU ? launch_fused_mode<true>(a, st)
+                                  : launch_fused_mode<false>(a, st);
+}
+
+}  // namespace la

@@ -70,34 +70,6 @@ struct TcParams {
     int want_output;
 };
 
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
-__device__ __forceinline__ void named_bar_sync(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
-// ReLU of 8 packed bf16 values: clear every element whose sign bit is set.
-__device__ __forceinline__ uint32_t relu_bf16x2(uint32_t w) {
-    const uint32_t m = ((w >> 15) & 0x00010001u) * 0xFFFFu;
-    return w & ~m;
-}
-
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-// Write 16 consecutive columns [c0, c0+16) of row `row` of a 2-block image.
-__device__ __forceinline__ void store_row16_bf16(uint8_t* img, int row, int c0, const float (&v)[16]) {
-    const int blk = c0 >> 6, ch = (c0 & 63) >> 3;
-    uint4 a = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
-                         pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
-    uint4 b = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
-                         pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
-    *reinterpret_cast<uint4*>(img + blk * 16384 + sw128_off(row, ch)) = a;
-    *reinterpret_cast<uint4*>(img + blk * 16384 + sw128_off(row, ch + 1)) = b;
-}
-
 // ============================================================================
 // gram: per-frame contractions over tokens
 // ============================================================================

@@ -27,16 +27,26 @@ def _cuda():
     torch.cuda.init()
 
 
+def _check_status(ws):
+    st = la.la_query_device_status(ws)
+    where = int(ws[4:8].view(torch.int32).item())
+    assert st == la.LA_OK, f"device status {la.la_status_string(st)} at wait 0x{where:x}"
+
+
 def _run(spec, mode, inp, state_in=None, z_in=None, want_state=True):
-    B, H, D = spec.B, spec.H, spec.D
+    B, H, F, S, D = spec.B, spec.H, spec.F, spec.S, spec.D
     so = torch.full((B, H, D, D), float("nan"), device="cuda") if want_state else None
+    m = la.LA_MODE_RELU if mode == "relu" else la.LA_MODE_GDN
+    ws = la.workspace_for(m, B, H, F, S, D)
     if mode == "relu":
         zo = torch.full((B, H, D), float("nan"), device="cuda") if want_state else None
         o = la.la_scan_relu(inp["q"], inp["k"], inp["v"], state_in=state_in, z_in=z_in,
-                            state_out=so, z_out=zo, eps=spec.eps)
+                            state_out=so, z_out=zo, eps=spec.eps, workspace=ws)
+        _check_status(ws)
         return o, so, zo
     o = la.la_scan_gdn(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], spec.k_scale,
-                       state_in=state_in, state_out=so)
+                       state_in=state_in, state_out=so, workspace=ws)
+    _check_status(ws)
     return o, so, None
 
 
@@ -72,6 +82,7 @@ def _compare(spec, mode, heads=None, with_state=False):
             assert rel_err(to_np(zo[b, h]), rz) < 1e-5
     e_o = rel_err(np.stack(got_o), np.stack(ref_o))
     e_m = rel_err(np.stack(got_m), np.stack(ref_m))
+    print(f"\n[parity] {spec.name} {mode}: output {e_o:.3e} state {e_m:.3e} (bar {tol})")
     assert e_o <= tol, f"output error {e_o:.3e} > {tol}"
     assert e_m <= tol, f"state error {e_m:.3e} > {tol}"
     return e_o, e_m
@@ -258,7 +269,7 @@ def test_rejects_host_and_overlapping_pointers():
 def test_tensor_core_path_matches_simt_path(mode, monkeypatch):
     spec = synth.small(B=1, H=3, F=5, S=333, D=128, dtype="bf16", seed=31, keys_l2=True)
     assert la.la_plan(la.LA_MODE_GDN if mode == "gdn" else la.LA_MODE_RELU, la.LA_BF16,
-                      1, 3, 5, 333, 128)[0] == "tcgen05"
+                      1, 3, 5, 333, 128)[0].startswith("tcgen05")
     inp = device_inputs(spec)
     o_tc, m_tc, _ = _run(spec, mode, inp)
     monkeypatch.setenv("LA_SCAN_FORCE_SIMT", "1")
@@ -269,6 +280,64 @@ def test_tensor_core_path_matches_simt_path(mode, monkeypatch):
 
 
 def test_plan_of_the_workloads():
-    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05", 3)
-    assert la.la_plan(la.LA_MODE_RELU, la.LA_BF16, 1, 20, 21, 1560, 112) == ("tcgen05", 3)
+    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05_fused", 1)
+    assert la.la_plan(la.LA_MODE_RELU, la.LA_BF16, 1, 20, 21, 1560, 112) == ("tcgen05_fused", 1)
+    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 4, 20, 8, 880, 128) == ("tcgen05", 3)
     assert la.la_plan(la.LA_MODE_GDN, la.LA_F32, 1, 2, 8, 64, 32)[0] == "simt_f32"
+    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 16, 512, 1024, 256)[0] == "simt_f32"
+
+
+@pytest.mark.parametrize("mode", ["relu", "gdn"])
+def test_fused_kernel_matches_three_kernel_path(mode, monkeypatch):
+    spec = synth.small(B=2, H=5, F=13, S=250, D=112, dtype="bf16", seed=33, keys_l2=True)
+    inp = device_inputs(spec)
+    m0n, z0n = synth.random_state(spec, 0.05)
+    m0, z0 = torch.from_numpy(m0n).cuda(), torch.from_numpy(z0n).cuda()
+    o_f, m_f, z_f = _run(spec, mode, inp, m0, z0 if mode == "relu" else None)
+    monkeypatch.setenv("LA_SCAN_NO_FUSE", "1")
+    o_3, m_3, z_3 = _run(spec, mode, inp, m0, z0 if mode == "relu" else None)
+    torch.cuda.synchronize()
+    # The fused kernel adds each frame's increment as a bf16 operand of the
+    # tensor core (the three-kernel path adds it in fp32), so the two agree to
+    # bf16 rounding of the increments, well inside the bf16 parity bar.
+    assert rel_err(to_np(o_f), to_np(o_3)) <= TOL_BF16
+    assert rel_err(to_np(m_f), to_np(m_3)) <= TOL_BF16
+    if mode == "relu":
+        assert rel_err(to_np(z_f), to_np(z_3)) < 1e-5
+
+
+@pytest.mark.parametrize("mode", ["relu", "gdn"])
+def test_fused_kernel_at_its_head_limit_with_slot_reuse(mode):
+    # 49 (b, h) pairs: one chain block each on a 148-SM B200 (the fused
+    # limit); F = 21 > 8 reuses every per-head hand-off slot.
+    spec = synth.small(B=7, H=7, F=21, S=96, D=128, dtype="bf16", seed=35, keys_l2=True,
+                       alpha=("sigmoid_normal", 3.0, 1.0), beta=("sigmoid_normal", 0.0, 1.0))
+    assert la.la_plan(la.LA_MODE_GDN if mode == "gdn" else la.LA_MODE_RELU, la.LA_BF16,
+                      7, 7, 21, 96, 128)[0] == "tcgen05_fused"
+    _compare(spec, mode, with_state=True, heads=[(0, 0), (3, 4), (6, 6)])
+
+
+def test_many_heads_use_the_three_kernel_path():
+    spec = synth.small(B=15, H=20, F=2, S=64, D=64, dtype="bf16", seed=37)
+    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 15, 20, 2, 64, 64) == ("tcgen05", 3)
+    _compare(spec, "gdn", heads=[(0, 0), (7, 13), (14, 19)])
+
+
+def test_device_wait_timeout_is_reported_and_the_context_stays_usable(monkeypatch):
+    # A gram hand-off flag that nothing sets: the chain block's bounded wait
+    # gives up, every block of the launch stops, the call's workspace records
+    # LA_ERR_TIMEOUT, and the next call works normally.
+    spec = synth.small(B=1, H=2, F=6, S=64, D=64, dtype="bf16", seed=39)
+    inp = device_inputs(spec)
+    ws = la.workspace_for(la.LA_MODE_GDN, 1, 2, 6, 64, 64)
+    monkeypatch.setenv("LA_SCAN_TEST_SKIP_PUBLISH", "3")
+    la.la_scan_gdn(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], spec.k_scale,
+                   workspace=ws)
+    assert la.la_query_device_status(ws) == la.LA_ERR_TIMEOUT
+    monkeypatch.delenv("LA_SCAN_TEST_SKIP_PUBLISH")
+    o = la.la_scan_gdn(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], spec.k_scale,
+                       workspace=ws)
+    assert la.la_query_device_status(ws) == la.LA_OK
+    for h in range(2):
+        ro, _, _ = _oracle(spec, "gdn", 0, h)
+        assert rel_err(to_np(o[0, h]), ro) <= TOL_BF16

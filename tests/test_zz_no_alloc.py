@@ -28,7 +28,7 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
     # 720p-shaped GDN slice on the tensor-core path: 2 x 3 heads x 8 frames per call
     spec = synth.small(B=2, H=3, F=16, S=880, D=128, dtype="bf16", seed=41, keys_l2=True,
                        alpha=("sigmoid_normal", 3.0, 1.0), beta=("sigmoid_normal", 0.0, 1.0))
-    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 2, 3, 8, 880, 128)[0] == "tcgen05"
+    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 2, 3, 8, 880, 128)[0].startswith("tcgen05")
     inp = device_inputs(spec)
     B, H, S, D = spec.B, spec.H, spec.S, spec.D
     stream = torch.cuda.current_stream()
@@ -55,7 +55,7 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls_in_a_row():
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
-    # 4 x 20 x 181 frames of 128 x 128 need far more than 64 MiB of scratch:
+    # 4 x 20 heads of 128 x 128 state need more than 64 MiB of scratch:
     # refused before anything is enqueued (the pointers are never touched).
     fake = ctypes.c_void_p(0x10000)
     st = la.lib.la_scan_gdn_noalloc(fake, fake, fake, fake, la.LA_BF16, fake, fake, 0.01,
