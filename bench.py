@@ -267,6 +267,8 @@ def run_ours(args):
 
     idx, mode = WORKLOADS[args.workload]
     base = synth.config(idx)
+    if args.frames:
+        base = base.with_(F=args.frames, name=f"{base.name}_clip{args.frames}")
     spec = base.with_(seed=base.seed + 1000 * rank) if rank else base   # own data per rank
     B, H, F, S, D = spec.B, spec.H, spec.F, spec.S, spec.D
     tdt = torch.bfloat16 if spec.dtype == "bf16" else torch.float32
@@ -465,6 +467,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true",
                     help="skip the host-buffer end-to-end leg (profiling runs)")
+    ap.add_argument("--frames", type=int, default=0,
+                    help="profiling only: a shorter clip (this many latent frames) of the workload")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

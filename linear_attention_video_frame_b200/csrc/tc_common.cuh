@@ -134,6 +134,27 @@ __device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t 
                  ::"l"(dst), "r"(smem_u32(src)), "r"(bytes) : "memory");
 }
 
+// The same copies with an L2 cache-eviction policy (see createpolicy below).
+__device__ __forceinline__ void bulk_load_hint(void* dst, const void* src, uint32_t bytes,
+                                               uint64_t* bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;"
+        ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy) : "memory");
+}
+__device__ __forceinline__ void bulk_store_hint(void* dst, const void* src, uint32_t bytes,
+                                                uint64_t policy) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;"
+                 ::"l"(dst), "r"(smem_u32(src)), "r"(bytes), "l"(policy) : "memory");
+}
+__device__ __forceinline__ void tma_store_3d_hint(const CUtensorMap* map, const void* src,
+                                                  int x, int y, int z, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group.L2::cache_hint"
+        " [%0, {%1, %2, %3}], [%4], %5;"
+        ::"l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(src)), "l"(policy) : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

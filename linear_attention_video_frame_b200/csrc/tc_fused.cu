@@ -71,7 +71,7 @@ __device__ unsigned long long* g_trace = nullptr;
 __device__ __forceinline__ void trace_event(uint32_t& n, uint32_t writer, uint32_t kind, uint64_t aux) {
     unsigned long long* t = g_trace;
     if (!t || n >= kTraceCap) return;
-    unsigned long long* r = t + 2 * ((size_t)(blockIdx.x * 2 + writer) * kTraceCap + n++);
+    unsigned long long* r = t + 2 * ((size_t)(blockIdx.x * 4 + writer) * kTraceCap + n++);
     r[0] = ((uint64_t)kind << 56) | ((uint64_t)blockIdx.x << 40) | (aux & 0xFFFFFFFFFFull);
     r[1] = global_timer_ns();
 }
@@ -252,8 +252,8 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                     if (ok) {
                         const size_t ms = (size_t)it.bh * kRM + it.f % kRM;
                         mbar_expect_tx(mfull, kImg + (RELU ? 512 : 0));
-                        bulk_load(mbuf, p.mimg + ms * kImg, kImg, mfull);
-                        if (RELU) bulk_load(zbuf, p.zf + ms * 128, 512, mfull);
+                        bulk_load_hint(mbuf, p.mimg + ms * kImg, kImg, mfull, pol);
+                        if (RELU) bulk_load_hint(zbuf, p.zf + ms * 128, 512, mfull, pol);
                     }
                     for (int t = 0; t < nto; ++t) {
                         ok = ok && mbar_wait(&empty[s], ph ^ 1, ab, 0x406);
@@ -352,6 +352,8 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
         uint32_t iq = 0, qctr = 0, sctr = 0;
         uint32_t dpar = 0;    // bit q: parity of quarter q's next output-tile use (denready)
         bool ok = true;
+        const uint64_t pol_keep = policy_evict_last();     // hand-off data: re-read soon
+        const uint64_t pol_stream = policy_evict_first();  // outputs: never re-read
         LA_TRACE_WRITER(1);
         while (true) {
             if (leader) {
@@ -411,7 +413,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                         fence_proxy_async_smem();
                         named_bar_sync(1, 128);
                         if (leader && go) {
-                            bulk_store(dst + blk * 16384, sb, 16384);
+                            bulk_store_hint(dst + blk * 16384, sb, 16384, pol_keep);
                             bulk_commit();
                         }
                     }
@@ -434,7 +436,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                 named_bar_sync(1, 128);
                 if (leader && go) {
                     if (RELU) {
-                        bulk_store(p.dz + sidx * 128, dzst, 512);
+                        bulk_store_hint(p.dz + sidx * 128, dzst, 512, pol_keep);
                         bulk_commit();
                     }
                     bulk_wait_all<0>();
@@ -482,7 +484,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                         fence_proxy_async_smem();
                         named_bar_sync(1, 128);
                         if (leader && go) {
-                            tma_store_3d(mO, sb, blk * 64, t * kTokO, frame);
+                            tma_store_3d_hint(mO, sb, blk * 64, t * kTokO, frame, pol_stream);
                             bulk_commit();
                             if (t == nto - 1 && blk == nblk - 1) LA_TRACE_EVENT(6, frame);
                         }
@@ -606,31 +608,35 @@ template <bool RELU>
 __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) {
     // stage s (64 KB): [0, 32 KB) G'' image (GDN) or dz_f (ReLU); [32 KB, 64 KB) B~ image
     uint8_t* stage = smem;                                  // kCStages x 64 KB
-    uint8_t* ident = stage + kCStages * 2 * kImg;           // identity (K-major A operand)
-    uint8_t* imgs = ident + kImg;                           // 2 x 32 KB bf16 state images
-    float* alph = reinterpret_cast<float*>(imgs + 2 * kImg);   // [kCStages] alpha of the staged frame
-    uint64_t* gfull = reinterpret_cast<uint64_t*>(alph + 4);
+    uint8_t* imgs = stage + kCStages * 2 * kImg;            // 2 x 32 KB bf16 state images
+    float* zst = reinterpret_cast<float*>(imgs + 2 * kImg); // [2][128] z_f staging (ReLU)
+    float* abc = zst + 256;                                 // [2] alpha_{f+1} broadcast per half
+    uint64_t* gfull = reinterpret_cast<uint64_t*>(abc + 2);
     uint64_t* gempty = gfull + kCStages;
-    uint64_t* mdone = gempty + kCStages;   // MMA of the frame finished
-    uint64_t* mready = mdone + 1;          // TMEM holds alpha_f M_{f-1}, image of M_{f-1} written
-    uint64_t* iready = mready + 1;         // [2] image buffer b holds a frame to publish
+    uint64_t* mdone = gempty + kCStages;   // [2] MMA of the frame finished (per column half)
+    uint64_t* mready = mdone + 2;          // [2] TMEM holds alpha_f M_{f-1}, image written (per half)
+    uint64_t* iready = mready + 2;         // [2] image buffer b holds a frame to publish
     uint64_t* iread = iready + 2;          // [2] publisher has read image buffer b out
-    int* bc_ok = reinterpret_cast<int*>(iread + 2);
+    int* bc_ok = reinterpret_cast<int*>(iread + 2);        // [2] per half
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bc_ok + 2);
     uint32_t* abort_flag = tmem_slot + 1;
-    float* zst = reinterpret_cast<float*>(stage + 8192);   // ReLU: [2][128] z_f staging
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.x;
+    const int F = p.F, D = p.D;
+    const int nhalf = D > 64 ? 2 : 1;      // independent column halves of the state
     if (threadIdx.x == 0) {
         for (int s = 0; s < kCStages; ++s) {
             mbar_init(&gfull[s], 1);
-            mbar_init(&gempty[s], 2);     // the MMA and the epilogue leader
+            // the epilogue halves (and, for GDN, the MMA) are done with the stage
+            mbar_init(&gempty[s], nhalf + (RELU ? 0 : 1));
         }
-        mbar_init(mdone, 1);
-        mbar_init(mready, 1);
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(&mdone[h], 1);
+            mbar_init(&mready[h], 1);
+        }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&iready[b], 1);
+            mbar_init(&iready[b], nhalf);
             mbar_init(&iread[b], 1);
         }
         *abort_flag = 0;
@@ -640,31 +646,18 @@ __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) 
         tmem_alloc(tmem_slot, 128);
         tmem_relinquish();
     }
-    if (warp >= 2 && warp < 10)
-        for (int idx = threadIdx.x - 64; idx < 128 * 16; idx += 256) {
-            const int r = idx >> 4, blk = (idx >> 3) & 1, c = idx & 7;
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int k0 = blk * 64 + c * 8 + 2 * e;
-                w[e] = (k0 == r ? 0x3F80u : 0u) | (k0 + 1 == r ? 0x3F800000u : 0u);
-            }
-            *reinterpret_cast<uint4*>(ident + blk * 16384 + sw128_off(r, c)) =
-                make_uint4(w[0], w[1], w[2], w[3]);
-        }
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tM = *tmem_slot;
     const Abort ab{abort_flag, p.status};
-    const int F = p.F, D = p.D;
 
     if (warp == 0) {
         // ---------------- loader ----------------
         if (lane == 0) {
             int s = 0;
             uint32_t ph = 0;
+            const uint64_t pol_last_use = policy_evict_first();
             LA_TRACE_WRITER(0);
             for (int f = 0; f < F; ++f) {
                 const size_t sidx = (size_t)bh * kRG + f % kRG;
@@ -673,192 +666,218 @@ __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) 
                 fence_proxy_async_global();
                 if (!mbar_wait(&gempty[s], ph ^ 1, ab, 0x502)) break;
                 uint8_t* st = stage + s * 2 * kImg;
-                alph[s] = RELU ? 1.f : p.alpha[(size_t)bh * F + f];
                 if (!RELU) {
                     mbar_expect_tx(&gfull[s], 2 * kImg);
-                    bulk_load(st, p.gimg + sidx * kImg, kImg, &gfull[s]);
+                    bulk_load_hint(st, p.gimg + sidx * kImg, kImg, &gfull[s], pol_last_use);
                 } else {
                     mbar_expect_tx(&gfull[s], kImg + 512);
-                    bulk_load(st, p.dz + sidx * 128, 512, &gfull[s]);
+                    bulk_load_hint(st, p.dz + sidx * 128, 512, &gfull[s], pol_last_use);
                 }
-                bulk_load(st + kImg, p.bimg + sidx * kImg, kImg, &gfull[s]);
+                bulk_load_hint(st + kImg, p.bimg + sidx * kImg, kImg, &gfull[s], pol_last_use);
                 if (++s == kCStages) { s = 0; ph ^= 1; }
             }
         }
     } else if (warp == 1) {
-        // ---------------- MMA: D = alpha M_{f-1} + G'' bf16(M_{f-1}) + I B~ ----------------
-        if (lane == 0) {
-            const uint32_t idM = idesc_bf16(128, D, false, true);
-            const uint32_t ia = smem_u32(ident);
+        // ---------------- MMA (GDN): D[:, half] += G'' bf16(M_{f-1})[:, half] ----------------
+        if (!RELU && lane == 0) {
             int s = 0;
             uint32_t ph = 0;
             for (int f = 0; f < F; ++f) {
                 if (!mbar_wait(&gfull[s], ph, ab, 0x503)) break;
-                if (!mbar_wait(mready, f & 1, ab, 0x504)) break;
-                tc_fence_after();
                 const uint32_t sa = smem_u32(stage + s * 2 * kImg);
                 const uint32_t mb = smem_u32(imgs + ((f + 1) & 1) * kImg);   // image of M_{f-1}
-                if (!RELU)
+                bool ok = true;
+                for (int h = 0; h < nhalf; ++h) {
+                    if (!(ok = mbar_wait(&mready[h], f & 1, ab, 0x504))) break;
+                    tc_fence_after();
+                    const int nh = min(64, D - 64 * h);
+                    const uint32_t idH = idesc_bf16(128, nh, false, true);
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint64_t ad = sdesc_sw128(sa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                        const uint64_t bd = sdesc_sw128(mb + kk * 2048, 16384, 1024);
-                        mma_bf16(tM, ad, bd, idM, 1u);
+                        const uint64_t bd = sdesc_sw128(mb + h * 16384 + kk * 2048, 16384, 1024);
+                        mma_bf16(tM + 64 * h, ad, bd, idH, 1u);
                     }
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t ad = sdesc_sw128(ia + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bd = sdesc_sw128(sa + kImg + kk * 2048, 16384, 1024);
-                    mma_bf16(tM, ad, bd, idM, 1u);
+                    mma_commit(&mdone[h]);
                 }
-                mma_commit(mdone);
+                if (!ok) break;
                 mma_commit(&gempty[s]);
                 if (++s == kCStages) { s = 0; ph ^= 1; }
             }
         }
     } else if (warp < 10) {
-        // ---------------- epilogue: thread <-> (state row, column half) ----------------
-        const int q = warp & 3, row = q * 32 + lane, half = (warp - 2) >> 2;
-        const int c_lo = half * 64, c_hi = min(D, c_lo + 64);
-        const bool leader = (threadIdx.x == 64);
+        // ---------------- epilogue: two independent column halves ----------------
+        const int h = (warp - 2) >> 2;                  // column half of this warp
+        const int q = warp & 3, row = q * 32 + lane;
+        const int c_lo = 64 * h, c_hi = min(D, c_lo + 64);
+        const bool active = h < nhalf;
+        const bool leader = ((threadIdx.x & 127) == 0); // first thread of each half group
+        const int bar_id = 1 + h;
         const uint32_t tl = tM + (uint32_t(q * 32) << 16);
         const bool live = row < D;
-        LA_TRACE_WRITER(1);
-        // initial state: image of M_0 (buffer 1 = "frame -1") and TMEM alpha_0 M_0
-        if (leader) {
-            bc_ok[0] = F > 0 && mbar_wait(&gfull[0], 0, ab, 0x50c);
-        }
-        named_bar_sync(1, 256);
-        const float a0 = (!RELU && bc_ok[0]) ? alph[0] : 1.f;
-        float z = 0.f;
-        for (int c0 = c_lo; c0 < c_hi; c0 += 16) {
-            float v[16];
+        LA_TRACE_WRITER(1 + h);
+        if (active) {
+            // alpha_{f+1} is read two frames ahead from the gate array (a read-only input)
+            const float* ap = p.alpha + (size_t)bh * F;
+            float a_cur = (!RELU && F > 0) ? __ldg(ap) : 1.f;       // alpha_0
+            float a_nxt = (!RELU && F > 1) ? __ldg(ap + 1) : 1.f;   // alpha_1
+            // initial state: image of M_0 (buffer 1 = "frame -1") and TMEM alpha_0 M_0
+            float z = 0.f;
+            for (int c0 = c_lo; c0 < c_hi; c0 += 16) {
+                float v[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-                v[e] = (p.state_in && live) ? p.state_in[((size_t)bh * D + row) * D + c0 + e] : 0.f;
-            store_row16_bf16(imgs + kImg, row, c0, v);
+                for (int e = 0; e < 16; ++e)
+                    v[e] = (p.state_in && live) ? p.state_in[((size_t)bh * D + row) * D + c0 + e] : 0.f;
+                store_row16_bf16(imgs + kImg, row, c0, v);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] *= a0;
-            tmem_st16(tl + c0, v);
-        }
-        if (RELU && half == 0 && p.z_in && live) z = p.z_in[(size_t)bh * D + row];
-        tmem_wait_st();
-        fence_proxy_async_smem();
-        tc_fence_before();
-        named_bar_sync(1, 256);
-        if (leader) mbar_arrive(mready);
-
-        int s = 0;
-        uint32_t ph = 0;
-        bool ok = true;
-        for (int f = 0; f < F; ++f) {
-            const int frame = bh * F + f;
-            const int ib = f & 1;
-            const int s_next = (s + 1 == kCStages) ? 0 : s + 1;
-            const uint32_t ph_next = (s + 1 == kCStages) ? (ph ^ 1) : ph;
-            const bool more = f + 1 < F;
-            if (leader) {
-                ok = ok && mbar_wait(mdone, f & 1, ab, 0x506);
-                // image buffer ib was last used by frame f - 2: read out by the publisher
-                if (f >= 2) ok = ok && mbar_wait(&iread[ib], ((f >> 1) - 1) & 1, ab, 0x507);
-                // alpha_{f+1} (GDN) arrives with the next frame's operands
-                if (!RELU && more) ok = ok && mbar_wait(&gfull[s_next], ph_next, ab, 0x505);
-                bc_ok[0] = ok;
-                LA_TRACE_EVENT(11, frame);
+                for (int e = 0; e < 16; ++e) v[e] *= a_cur;
+                tmem_st16(tl + c0, v);
             }
-            named_bar_sync(1, 256);
-            const bool go = bc_ok[0];
-            tc_fence_after();
-            if (go) {
-                const float an = (!RELU && more) ? alph[s_next] : 1.f;
-                uint8_t* img = imgs + ib * kImg;
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int c0 = c_lo + 32 * hh;
-                    if (c0 < c_hi) {
-                        const bool two = c0 + 16 < c_hi;
-                        float v0[16], v1[16];
-                        tmem_ld16(tl + c0, v0);
-                        if (two) tmem_ld16(tl + c0 + 16, v1);
-                        tmem_wait_ld();
-                        store_row16_bf16(img, row, c0, v0);
-                        if (two) store_row16_bf16(img, row, c0 + 16, v1);
-                        if (!more && p.state_out && live) {
-                            float* so = p.state_out + ((size_t)bh * D + row) * D + c0;
-#pragma unroll
-                            for (int u = 0; u < 4; ++u)
-                                *reinterpret_cast<float4*>(so + 4 * u) =
-                                    make_float4(v0[4 * u], v0[4 * u + 1], v0[4 * u + 2], v0[4 * u + 3]);
-                            if (two)
-#pragma unroll
-                                for (int u = 0; u < 4; ++u)
-                                    *reinterpret_cast<float4*>(so + 16 + 4 * u) =
-                                        make_float4(v1[4 * u], v1[4 * u + 1], v1[4 * u + 2], v1[4 * u + 3]);
-                        }
-                        if (!RELU && more) {
-#pragma unroll
-                            for (int e = 0; e < 16; ++e) {
-                                v0[e] *= an;
-                                v1[e] *= an;
-                            }
-                            tmem_st16(tl + c0, v0);
-                            if (two) tmem_st16(tl + c0 + 16, v1);
-                        }
-                    }
-                }
-                if (RELU && half == 0) {
-                    z += reinterpret_cast<const float*>(stage + s * 2 * kImg)[row];
-                    zst[ib * 128 + row] = z;
-                    if (!more && p.z_out && live) p.z_out[(size_t)bh * D + row] = z;
-                }
-            }
+            if (RELU && h == 0 && p.z_in && live) z = p.z_in[(size_t)bh * D + row];
             tmem_wait_st();
             fence_proxy_async_smem();
             tc_fence_before();
-            named_bar_sync(1, 256);
-            if (leader) {
-                mbar_arrive(&gempty[s]);
-                mbar_arrive(mready);
-                mbar_arrive(&iready[ib]);
-                LA_TRACE_EVENT(12, frame);
+            named_bar_sync(bar_id, 128);
+            if (leader) mbar_arrive(&mready[h]);
+
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int f = 0; f < F; ++f) {
+                const int frame = bh * F + f;
+                const int ib = f & 1;
+                const bool more = f + 1 < F;
+                if (leader) {
+                    ok = ok && mbar_wait(&gfull[s], ph, ab, 0x505);
+                    if (!RELU) ok = ok && mbar_wait(&mdone[h], f & 1, ab, 0x506);
+                    LA_TRACE_EVENT(16 + 20 * h, frame);
+                    // image buffer ib was last used by frame f - 2: read out by the publisher
+                    if (f >= 2) ok = ok && mbar_wait(&iread[ib], ((f >> 1) - 1) & 1, ab, 0x507);
+                    bc_ok[h] = ok;
+                    abc[h] = a_nxt;
+                    LA_TRACE_EVENT(11 + 20 * h, frame);
+                }
+                named_bar_sync(bar_id, 128);
+                const bool go = bc_ok[h];
+                const float an = abc[h];
+                tc_fence_after();
+                if (leader) a_nxt = (!RELU && f + 2 < F) ? __ldg(ap + f + 2) : 1.f;
+                if (go) {
+                    const uint8_t* bimg = stage + s * 2 * kImg + kImg + h * 16384;
+                    uint8_t* img = imgs + ib * kImg;
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const int c0 = c_lo + 32 * cc;
+                        if (c0 < c_hi) {
+                            const bool two = c0 + 16 < c_hi;
+                            float v0[16], v1[16];
+                            tmem_ld16(tl + c0, v0);
+                            if (two) tmem_ld16(tl + c0 + 16, v1);
+                            // B~ (bf16) columns c0 .. c0+31 of this row
+                            uint4 bw[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                bw[u] = *reinterpret_cast<const uint4*>(
+                                    bimg + sw128_off(row, ((c0 & 63) >> 3) + u));
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                v0[8 * u + 0] += bf16_lo(bw[u].x); v0[8 * u + 1] += bf16_hi(bw[u].x);
+                                v0[8 * u + 2] += bf16_lo(bw[u].y); v0[8 * u + 3] += bf16_hi(bw[u].y);
+                                v0[8 * u + 4] += bf16_lo(bw[u].z); v0[8 * u + 5] += bf16_hi(bw[u].z);
+                                v0[8 * u + 6] += bf16_lo(bw[u].w); v0[8 * u + 7] += bf16_hi(bw[u].w);
+                                v1[8 * u + 0] += bf16_lo(bw[u + 2].x); v1[8 * u + 1] += bf16_hi(bw[u + 2].x);
+                                v1[8 * u + 2] += bf16_lo(bw[u + 2].y); v1[8 * u + 3] += bf16_hi(bw[u + 2].y);
+                                v1[8 * u + 4] += bf16_lo(bw[u + 2].z); v1[8 * u + 5] += bf16_hi(bw[u + 2].z);
+                                v1[8 * u + 6] += bf16_lo(bw[u + 2].w); v1[8 * u + 7] += bf16_hi(bw[u + 2].w);
+                            }
+                            store_row16_bf16(img, row, c0, v0);
+                            if (two) store_row16_bf16(img, row, c0 + 16, v1);
+                            if (!more && p.state_out && live) {
+                                float* so = p.state_out + ((size_t)bh * D + row) * D + c0;
+#pragma unroll
+                                for (int u = 0; u < 4; ++u)
+                                    *reinterpret_cast<float4*>(so + 4 * u) =
+                                        make_float4(v0[4 * u], v0[4 * u + 1], v0[4 * u + 2], v0[4 * u + 3]);
+                                if (two)
+#pragma unroll
+                                    for (int u = 0; u < 4; ++u)
+                                        *reinterpret_cast<float4*>(so + 16 + 4 * u) =
+                                            make_float4(v1[4 * u], v1[4 * u + 1], v1[4 * u + 2], v1[4 * u + 3]);
+                            }
+                            if (more) {
+                                if (!RELU)
+#pragma unroll
+                                    for (int e = 0; e < 16; ++e) {
+                                        v0[e] *= an;
+                                        v1[e] *= an;
+                                    }
+                                tmem_st16(tl + c0, v0);
+                                if (two) tmem_st16(tl + c0 + 16, v1);
+                            }
+                        }
+                    }
+                    if (RELU && h == 0) {
+                        z += reinterpret_cast<const float*>(stage + s * 2 * kImg)[row];
+                        zst[ib * 128 + row] = z;
+                        if (!more && p.z_out && live) p.z_out[(size_t)bh * D + row] = z;
+                    }
+                }
+                tmem_wait_st();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar_sync(bar_id, 128);
+                if (leader) {
+                    mbar_arrive(&gempty[s]);
+                    mbar_arrive(&mready[h]);
+                    mbar_arrive(&iready[ib]);
+                    LA_TRACE_EVENT(12 + 20 * h, frame);
+                }
+                if (++s == kCStages) { s = 0; ph ^= 1; }
             }
-            s = s_next;
-            ph = ph_next;
         }
     } else if (warp == 10) {
         // ---------------- publisher ----------------
-        // Frame f's stores are issued as soon as its image is written; frame
-        // f - 1 is published (chain_done = f) once all but the newest store
-        // group have completed, so store latency never holds the image buffers.
+        // Frame f's stores are issued as soon as its image is written and its
+        // ring slot is free.  Up to kPubLag store groups stay in flight; frame
+        // g is published (chain_done = g + 1) once its stores have completed,
+        // so store latency never holds back the image buffers.  The slot-free
+        // flag of the next frame is read one frame ahead.
         if (lane == 0) {
-            int done = 0;
+            constexpr int kPubLag = 3;
+            const uint64_t pol_keep = policy_evict_last();
+            int published = 0;            // frames published so far
+            uint32_t seen = 0;            // last value read from the next slot's flag
             for (int f = 0; f < F; ++f) {
                 const int ib = f & 1;
                 const size_t msidx = (size_t)bh * kRM + f % kRM;
-                // the output item that last used this slot has read it (checked
-                // before the image is ready: it almost always already holds)
-                if (p.want_output && f >= kRM &&
+                if (p.want_output && f >= kRM && seen < (uint32_t)(f - kRM + 1) &&
                     !wait_flag_ge(&p.mimg_consumed[msidx], f - kRM + 1, ab, 0x509))
                     break;
                 if (!mbar_wait(&iready[ib], (f >> 1) & 1, ab, 0x508)) break;
                 if (p.want_output) {
-                    bulk_store(p.mimg + msidx * kImg, imgs + ib * kImg, kImg);
-                    if (RELU) bulk_store(p.zf + msidx * 128, zst + ib * 128, 512);
+                    bulk_store_hint(p.mimg + msidx * kImg, imgs + ib * kImg, kImg, pol_keep);
+                    if (RELU) bulk_store_hint(p.zf + msidx * 128, zst + ib * 128, 512, pol_keep);
                     bulk_commit();
                     bulk_wait_read<0>();
                 }
                 mbar_arrive(&iread[ib]);
+                // look at the next frame's slot while this frame's stores drain
+                seen = (p.want_output && f + 1 < F && f + 1 >= kRM)
+                           ? ld_acquire_gpu(&p.mimg_consumed[(size_t)bh * kRM + (f + 1) % kRM])
+                           : 0u;
                 if (p.want_output) {
-                    if (f > 0) {
-                        bulk_wait_all<1>();
+                    if (f + 1 - published > kPubLag) {
+                        bulk_wait_all<kPubLag>();
                         fence_proxy_async_global();
-                        st_release_gpu(&p.chain_done[bh], f);
-                        done = f;
+                        published = f + 1 - kPubLag;
+                        st_release_gpu(&p.chain_done[bh], published);
                     }
                 } else {
-                    st_release_gpu(&p.chain_done[bh], f + 1);
-                    done = f + 1;
+                    published = f + 1;
+                    st_release_gpu(&p.chain_done[bh], published);
                 }
             }
-            if (p.want_output && done < F && !ab.raised()) {
+            if (p.want_output && published < F && !ab.raised()) {
                 bulk_wait_all<0>();
                 fence_proxy_async_global();
                 st_release_gpu(&p.chain_done[bh], F);
@@ -920,7 +939,7 @@ FusedLayout fused_layout(const ScanArgs& a) {
 constexpr size_t kWorkerSmem = kWStages * 32768 + kImg + 2 * 16384 + 2048 + 512 + 2048 + 512 +
                                (kIQ + 2) * sizeof(Item) + 16 +
                                (3 * kWStages + 2 + 12 + 2 * kIQ) * 8 + 8;
-constexpr size_t kChainSmem = kCStages * 2 * kImg + kImg + 2 * kImg + 16 + 10 * 8 + 8 + 8;
+constexpr size_t kChainSmem = kCStages * 2 * kImg + 2 * kImg + 1024 + 8 + 12 * 8 + 8 + 8;
 constexpr size_t kFusedSmem = 1024 + (kWorkerSmem > kChainSmem ? kWorkerSmem : kChainSmem);
 static_assert(kFusedSmem <= 232448, "fused kernel shared memory");
 
