@@ -125,6 +125,25 @@ def traffic_record(workload: str):
 
 
 # ----------------------------------------------------------------------------
+# Multi-rank host logic (weak scaling: one replica per rank, own data)
+# ----------------------------------------------------------------------------
+def rank_spec(base, rank: int):
+    """Rank r > 0 scans its own batch: the same workload with seed + 1000 r."""
+    return base.with_(seed=base.seed + 1000 * rank) if rank else base
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """The slowest rank's time (the job's time); plumbing only, not on the data path."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------
 # Clock sampling during the timed region (NVML; read-only)
 # ----------------------------------------------------------------------------
 class ClockSampler:
@@ -269,7 +288,7 @@ def run_ours(args):
     base = synth.config(idx)
     if args.frames:
         base = base.with_(F=args.frames, name=f"{base.name}_clip{args.frames}")
-    spec = base.with_(seed=base.seed + 1000 * rank) if rank else base   # own data per rank
+    spec = rank_spec(base, rank)   # own data per rank
     B, H, F, S, D = spec.B, spec.H, spec.F, spec.S, spec.D
     tdt = torch.bfloat16 if spec.dtype == "bf16" else torch.float32
     dtc = la.LA_BF16 if spec.dtype == "bf16" else la.LA_F32
@@ -354,11 +373,7 @@ def run_ours(args):
     barrier()
     t_local = t0.elapsed_time(t1) / 1e3
     call_ms = [s.elapsed_time(e) / len(plan) for s, e in evs]
-    t_max = t_local
-    if world > 1:
-        tt = torch.tensor([t_local], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max = float(tt.item())
+    t_max = max_over_ranks(t_local, dev)
 
     byts, flops = step_counts(spec, mode)
     frames_all = B * F * K * world
@@ -398,11 +413,7 @@ def run_ours(args):
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        te = e0.elapsed_time(e1) / 1e3
-        if world > 1:
-            tt = torch.tensor([te], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            te = float(tt.item())
+        te = max_over_ranks(e0.elapsed_time(e1) / 1e3, dev)
         e2e_value = B * F * Ke * world / te
     status = la.la_query_device_status(ws)
 
