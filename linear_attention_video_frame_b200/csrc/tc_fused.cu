@@ -49,9 +49,23 @@ namespace {
 
 using namespace tc;
 
+// Tuning knobs (compile-time; the defaults are the measured best).
+#ifndef LA_FUSED_WSTAGES
+#define LA_FUSED_WSTAGES 4
+#endif
+#ifndef LA_FUSED_EARLY_Q
+#define LA_FUSED_EARLY_Q 1
+#endif
+#ifndef LA_FUSED_LAG
+#define LA_FUSED_LAG 14
+#endif
+#ifndef LA_FUSED_PUBLAG
+#define LA_FUSED_PUBLAG 1
+#endif
+
 constexpr int kRG = 16;                 // per-head ring slots: gram -> chain
 constexpr int kRM = 16;                 // per-head ring slots: chain -> output
-constexpr int kWStages = 4;             // worker TMA ring (32 KB stages)
+constexpr int kWStages = LA_FUSED_WSTAGES;   // worker TMA ring (32 KB stages)
 constexpr int kCStages = 2;             // chain operand ring depth
 constexpr int kIQ = 4;                  // worker item queue depth
 constexpr int kThreads = 352;           // 11 warps
@@ -244,18 +258,24 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                         if (++s == kWStages) { s = 0; ph ^= 1; }
                     }
                 } else {
-                    ok = ok && wait_flag_ge(&p.chain_done[it.bh], it.f + 1, ab, 0x404);
-                    LA_TRACE_EVENT(4, frame);
-                    fence_proxy_async_global();
-                    ok = ok && mbar_wait(mempty, (nout & 1) ^ 1, ab, 0x405);
-                    ++nout;
-                    if (ok) {
-                        const size_t ms = (size_t)it.bh * kRM + it.f % kRM;
-                        mbar_expect_tx(mfull, kImg + (RELU ? 512 : 0));
-                        bulk_load_hint(mbuf, p.mimg + ms * kImg, kImg, mfull, pol);
-                        if (RELU) bulk_load_hint(zbuf, p.zf + ms * 128, 512, mfull, pol);
-                    }
+                    // Q does not depend on the chain: fill the ring with Q tiles first,
+                    // then wait for the state image of the frame and fetch it.
+                    auto fetch_state = [&]() {
+                        ok = ok && wait_flag_ge(&p.chain_done[it.bh], it.f + 1, ab, 0x404);
+                        LA_TRACE_EVENT(4, frame);
+                        fence_proxy_async_global();
+                        ok = ok && mbar_wait(mempty, (nout & 1) ^ 1, ab, 0x405);
+                        ++nout;
+                        if (ok) {
+                            const size_t ms = (size_t)it.bh * kRM + it.f % kRM;
+                            mbar_expect_tx(mfull, kImg + (RELU ? 512 : 0));
+                            bulk_load_hint(mbuf, p.mimg + ms * kImg, kImg, mfull, pol);
+                            if (RELU) bulk_load_hint(zbuf, p.zf + ms * 128, 512, mfull, pol);
+                        }
+                    };
+                    const int early = LA_FUSED_EARLY_Q ? min(nto, kWStages) : 0;
                     for (int t = 0; t < nto; ++t) {
+                        if (t == early) fetch_state();
                         ok = ok && mbar_wait(&empty[s], ph ^ 1, ab, 0x406);
                         if (ok) {
                             uint8_t* st = ring + s * 32768;
@@ -265,6 +285,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                         }
                         if (++s == kWStages) { s = 0; ph ^= 1; }
                     }
+                    if (early == nto) fetch_state();
                 }
             }
         }
@@ -665,6 +686,7 @@ __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) 
                 LA_TRACE_EVENT(10, (uint64_t)bh * F + f);
                 fence_proxy_async_global();
                 if (!mbar_wait(&gempty[s], ph ^ 1, ab, 0x502)) break;
+                LA_TRACE_EVENT(18, (uint64_t)bh * F + f);
                 uint8_t* st = stage + s * 2 * kImg;
                 if (!RELU) {
                     mbar_expect_tx(&gfull[s], 2 * kImg);
@@ -682,13 +704,16 @@ __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) 
         if (!RELU && lane == 0) {
             int s = 0;
             uint32_t ph = 0;
+            LA_TRACE_WRITER(3);
             for (int f = 0; f < F; ++f) {
                 if (!mbar_wait(&gfull[s], ph, ab, 0x503)) break;
+                LA_TRACE_EVENT(19, (uint64_t)bh * F + f);
                 const uint32_t sa = smem_u32(stage + s * 2 * kImg);
                 const uint32_t mb = smem_u32(imgs + ((f + 1) & 1) * kImg);   // image of M_{f-1}
                 bool ok = true;
                 for (int h = 0; h < nhalf; ++h) {
                     if (!(ok = mbar_wait(&mready[h], f & 1, ab, 0x504))) break;
+                    LA_TRACE_EVENT(22 + h, (uint64_t)bh * F + f);
                     tc_fence_after();
                     const int nh = min(64, D - 64 * h);
                     const uint32_t idH = idesc_bf16(128, nh, false, true);
@@ -843,7 +868,7 @@ __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) 
         // so store latency never holds back the image buffers.  The slot-free
         // flag of the next frame is read one frame ahead.
         if (lane == 0) {
-            constexpr int kPubLag = 3;
+            constexpr int kPubLag = LA_FUSED_PUBLAG;
             const uint64_t pol_keep = policy_evict_last();
             int published = 0;            // frames published so far
             uint32_t seen = 0;            // last value read from the next slot's flag
@@ -981,7 +1006,7 @@ cudaError_t launch_fused_mode(const ScanArgs& a, cudaStream_t st) {
     p.S = a.S;
     p.D = a.D;
     p.want_output = a.o != nullptr;
-    p.lag = 10;
+    p.lag = LA_FUSED_LAG;
     if (const char* e = std::getenv("LA_SCAN_LAG")) p.lag = std::max(1, std::min(std::atoi(e), kRG + kRM - 1));
     p.skip_publish = -1;
     if (const char* e = std::getenv("LA_SCAN_TEST_SKIP_PUBLISH")) p.skip_publish = std::atoi(e);
