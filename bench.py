@@ -102,10 +102,21 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# Sources the dominant (fused) kernel is compiled from.
+KERNEL_SOURCES = ("tc_fused.cu", "tc_common.cuh", "tmap.cuh", "common.cuh")
+
+
 def kernel_source_hash() -> str:
+    """Hash of the fused kernel's sources, so a committed DRAM-traffic figure
+    is used only while the kernel it was measured on is unchanged.  Lines of
+    the optional event trace are left out: without -DLA_TRACE they compile
+    to nothing."""
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "linear_attention_video_frame_b200", "csrc", "*"))):
-        h.update(open(p, "rb").read())
+    for name in KERNEL_SOURCES:
+        p = os.path.join(ROOT, "linear_attention_video_frame_b200", "csrc", name)
+        for line in open(p, "rb").read().splitlines(keepends=True):
+            if b"LA_TRACE" not in line:
+                h.update(line)
     return h.hexdigest()[:16]
 
 
@@ -381,24 +392,27 @@ def run_ours(args):
     ms_per_step = 1e3 * t_max / K
     tflops = flops * K * world / t_max / 1e12
 
-    # ---- e2e: host buffers, H2D of inputs and D2H of the output inside the timed region ----
+    # ---- e2e: the C-ABI host-buffer call (la_scan_host): H2D of the inputs, the
+    # scan and D2H of the output and final state all inside the timed region,
+    # pipelined chunk by chunk over the library's copy streams ----
     Ke = max(3, min(K, 10))
+    mode_c = la.LA_MODE_GDN if mode == "gdn" else la.LA_MODE_RELU
+    chunk = spec.chunk_frames or 0
     o_host = torch.empty_like(host["q"], pin_memory=True)
-    h2d = sum(host[x].numel() * host[x].element_size() for x in ("q", "k", "v", "alpha", "beta"))
-    d2h = o_host.numel() * o_host.element_size()
+    so_host = torch.empty((B, H, D, D), dtype=torch.float32, pin_memory=True)
+    zo_host = torch.empty((B, H, D), dtype=torch.float32, pin_memory=True) \
+        if mode == "relu" else None
+    ins = ("q", "k", "v", "alpha", "beta") if mode == "gdn" else ("q", "k", "v")
+    h2d = sum(host[x].numel() * host[x].element_size() for x in ins)
+    d2h = sum(t.numel() * t.element_size() for t in (o_host, so_host, zo_host) if t is not None)
+    hws = None if args.no_e2e else la.host_workspace_for(mode_c, dtc, B, H, F, S, D, chunk, dev)
 
     def e2e_step():
-        for x in ("q", "k", "v", "alpha", "beta"):
-            dev_in[x].copy_(host[x], non_blocking=True)
-        if len(views) > 1:   # chunked: re-slice from the freshly copied tensors
-            for j, (f0, n, si) in enumerate(plan):
-                sl = slice(f0, f0 + n)
-                for i, x in enumerate(("q", "k", "v", "alpha", "beta")):
-                    views[j][i].copy_(dev_in[x][:, :, sl])
-        one_step()
-        if len(views) > 1:
-            o.copy_(torch.cat([vw[5] for vw in views], dim=2))
-        o_host.copy_(o, non_blocking=True)
+        la.la_scan_host(mode_c, host["q"], host["k"], host["v"], o=o_host,
+                        alpha=host["alpha"] if mode == "gdn" else None,
+                        beta=host["beta"] if mode == "gdn" else None,
+                        k_scale=spec.k_scale, eps=spec.eps, state_out=so_host, z_out=zo_host,
+                        chunk_frames=chunk, workspace=hws, stream=stream)
 
     e2e_value = None
     if not args.no_e2e:
@@ -416,6 +430,8 @@ def run_ours(args):
         te = max_over_ranks(e0.elapsed_time(e1) / 1e3, dev)
         e2e_value = B * F * Ke * world / te
     status = la.la_query_device_status(ws)
+    if status == la.LA_OK and hws is not None:
+        status = la.la_query_device_status(hws)
 
     # ---- roofline of the dominant kernel ----
     peaks, peak_src = load_peaks()
@@ -427,6 +443,8 @@ def run_ours(args):
                 "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
                 "peak_source": f"{peak_src} (hbm_gbs, STREAM-style copy)",
                 "kernel": path, "kernel_ms": kern_s * 1e3,
+                "kernel_ms_min": min(call_ms), "kernel_ms_median": statistics.median(call_ms),
+                "kernel_ms_max": max(call_ms),
                 "alg_bytes_per_launch": per_call_bytes,
                 "tensor_tflops_achieved": flops / len(plan) / kern_s / 1e12,
                 "tensor_frac_of_bf16_peak": flops / len(plan) / kern_s / 1e12 /
@@ -454,7 +472,9 @@ def run_ours(args):
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "latent frames/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": Ke},
+                "d2h_bytes_per_step": d2h, "steps": Ke, "call": "la_scan_host",
+                "chunk_frames": la.la_host_chunk_frames(F, chunk),
+                "host_memory": "pinned"},
         "clocks": clocks.summary(),
         "device_status": la.la_status_string(status),
     }

@@ -174,6 +174,60 @@ LA_API la_status la_scan_gdn_noalloc(const void* q, const void* k, const void* v
                                      float k_scale, const float* state_in, float* state_out,
                                      int B, int H, int F, int S, int D, cudaStream_t stream);
 
+/*
+ * The scan of a clip held in HOST memory, streamed through the GPU in chunks
+ * of frames.  Source: SANA-WM paper summary (paperlayer), section 3,
+ * "Chunk-causal deployment", and the SANA-Video talk, block KV cache
+ * segment -- the recurrent state carries everything a later chunk needs
+ * from the earlier ones, so a clip can be processed chunk by chunk.
+ * The computation is that of la_scan_relu (mode LA_MODE_RELU) or
+ * la_scan_gdn (mode LA_MODE_GDN) on the whole clip; the chunking changes
+ * only where the data is while it runs.
+ *
+ * Pipeline.  Chunk c+1 is copied in (host to device) while chunk c is
+ *   scanned on `stream` and chunk c-1's output is copied out, on two copy
+ *   streams of the library's own, over a ring of three chunk slots in the
+ *   workspace.  The state stays on the device between chunks.
+ * Memory.  q, k, v, o, alpha, beta, state_in, z_in, state_out and z_out
+ *   are HOST pointers with the layouts of the shared conventions above
+ *   (device or managed pointers are rejected with LA_ERR_INVALID_ARG).
+ *   Page-locked (pinned) host memory lets the copies overlap the scan and
+ *   each other; pageable memory is accepted, but the driver stages its
+ *   copies and the call may return only after them.  `workspace` is device
+ *   memory of the current device, 256-byte aligned, of at least
+ *   la_host_workspace_size(mode, dt, B, H, F, S, D, chunk_frames) bytes;
+ *   la_query_device_status accepts it.
+ * Chunking.  chunk_frames > 0 sets the frames per chunk (the last chunk may
+ *   be shorter); chunk_frames <= 0 picks about 16 chunks
+ *   (la_host_chunk_frames reports the choice).
+ * Mode.    LA_MODE_GDN uses alpha, beta, k_scale and ignores eps, z_in and
+ *   z_out; LA_MODE_RELU uses eps, z_in and z_out and ignores the gates.
+ * Asynchrony.  Nothing starts before the work already queued on `stream`,
+ *   and work queued on `stream` after the call starts after every copy of
+ *   the call (host buffers may be read or reused once `stream` reaches that
+ *   point).  Argument errors return before anything is enqueued; a later
+ *   failure returns LA_ERR_CUDA (or the chunk scan's status) with the chunks
+ *   enqueued so far still ordered on `stream`.
+ * Resources.  The first call on a device creates two non-blocking streams
+ *   and a few events for it, kept until the process exits; calls on one
+ *   device serialise their enqueueing on a lock and share the copy streams.
+ */
+LA_API la_status la_scan_host(la_mode mode, const void* q, const void* k, const void* v, void* o,
+                              la_dtype dt, const float* alpha, const float* beta, float k_scale,
+                              float eps, const float* state_in, const float* z_in,
+                              float* state_out, float* z_out,
+                              int B, int H, int F, int S, int D, int chunk_frames,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Device workspace bytes la_scan_host needs for this mode, dtype, shape and
+ * chunking; 0 for an unsupported or invalid combination. */
+LA_API size_t la_host_workspace_size(la_mode mode, la_dtype dt, int B, int H, int F, int S, int D,
+                                     int chunk_frames);
+
+/* Frames per chunk that la_scan_host uses for F frames and this
+ * chunk_frames argument (0 when F < 0). */
+LA_API int la_host_chunk_frames(int F, int chunk_frames);
+
 /* Workspace bytes a call of this mode and shape needs (either dtype).
  * Returns 0 for an unsupported shape.  The library has no counterpart in
  * the pages; it exists because the library never allocates. */

@@ -23,7 +23,8 @@ __all__ = [
     "LA_F32", "LA_BF16", "LA_MODE_RELU", "LA_MODE_GDN", "LaScanError", "lib", "LIB_PATH",
     "la_scan_relu", "la_scan_gdn", "la_state_step", "la_workspace_size",
     "la_query_device_status", "la_status_string", "la_plan", "workspace_for",
-    "la_scan_gdn_noalloc", "LA_NOALLOC_SCRATCH_BYTES",
+    "la_scan_gdn_noalloc", "LA_NOALLOC_SCRATCH_BYTES", "la_scan_host",
+    "la_host_workspace_size", "la_host_chunk_frames", "host_workspace_for",
 ]
 
 LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CUDA, LA_ERR_TIMEOUT = 0, 1, 2, 3, 4
@@ -61,6 +62,13 @@ def _load() -> ctypes.CDLL:
     L.la_scan_gdn_noalloc.restype = I
     L.la_plan.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(ctypes.c_int)]
     L.la_plan.restype = ctypes.c_char_p
+    L.la_scan_host.argtypes = [I, P, P, P, P, I, P, P, F, F, P, P, P, P,
+                               I, I, I, I, I, I, P, Z, P]
+    L.la_scan_host.restype = I
+    L.la_host_workspace_size.argtypes = [I, I, I, I, I, I, I, I]
+    L.la_host_workspace_size.restype = Z
+    L.la_host_chunk_frames.argtypes = [I, I]
+    L.la_host_chunk_frames.restype = I
     L.la_status_string.argtypes = [I]
     L.la_status_string.restype = ctypes.c_char_p
     return L
@@ -211,3 +219,63 @@ def la_state_step(mode: int, k, v, alpha=None, beta=None, k_scale: float = 1.0,
 
 def la_query_device_status(workspace, stream=None) -> int:
     return int(lib.la_query_device_status(_ptr(workspace), _stream(stream)))
+
+
+def la_host_workspace_size(mode: int, dt: int, B: int, H: int, F: int, S: int, D: int,
+                           chunk_frames: int = 0) -> int:
+    return int(lib.la_host_workspace_size(mode, dt, B, H, F, S, D, int(chunk_frames)))
+
+
+def la_host_chunk_frames(F: int, chunk_frames: int = 0) -> int:
+    return int(lib.la_host_chunk_frames(int(F), int(chunk_frames)))
+
+
+def host_workspace_for(mode: int, dt: int, B: int, H: int, F: int, S: int, D: int,
+                       chunk_frames: int = 0, device=None) -> torch.Tensor:
+    """Device workspace of the size la_scan_host asks for."""
+    n = la_host_workspace_size(mode, dt, B, H, F, S, D, chunk_frames)
+    if n == 0:
+        raise LaScanError(LA_ERR_UNSUPPORTED, "la_host_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def _check_host(t: Optional[torch.Tensor], name: str, shape=None, dtype=None):
+    if t is None:
+        return
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+
+
+def la_scan_host(mode: int, q, k, v, o=None, alpha=None, beta=None, k_scale: float = 1.0,
+                 eps: float = 1e-6, state_in=None, z_in=None, state_out=None, z_out=None,
+                 chunk_frames: int = 0, workspace=None, stream=None):
+    """The scan of host-resident q, k, v into host o, streamed through the GPU
+    chunk by chunk (pinned tensors let the copies overlap the scan).  The call
+    is asynchronous on `stream`: synchronise it before reading o."""
+    B, H, F, S, D = k.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _check_host(t, n, (B, H, F, S, D), k.dtype)
+    for t, n in ((alpha, "alpha"), (beta, "beta")):
+        _check_host(t, n, (B, H, F), torch.float32)
+    for t, n in ((state_in, "state_in"), (state_out, "state_out")):
+        _check_host(t, n, (B, H, D, D), torch.float32)
+    for t, n in ((z_in, "z_in"), (z_out, "z_out")):
+        _check_host(t, n, (B, H, D), torch.float32)
+    if workspace is None:
+        raise ValueError("la_scan_host needs a device workspace (see host_workspace_for)")
+    if not workspace.is_cuda:
+        raise ValueError("the workspace must be a CUDA tensor")
+    if o is None:
+        o = torch.empty_like(q, pin_memory=q.is_pinned())
+    st = lib.la_scan_host(int(mode), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _dtype_code(k),
+                          _ptr(alpha), _ptr(beta), float(k_scale), float(eps), _ptr(state_in),
+                          _ptr(z_in), _ptr(state_out), _ptr(z_out), B, H, F, S, D,
+                          int(chunk_frames), _ptr(workspace), workspace.numel(), _stream(stream))
+    _raise(st, "la_scan_host")
+    return o

@@ -20,7 +20,8 @@ def declared_symbols():
 def test_header_declares_the_abi():
     assert declared_symbols() == sorted([
         "la_scan_relu", "la_scan_gdn", "la_state_step", "la_workspace_size",
-        "la_query_device_status", "la_status_string", "la_plan", "la_scan_gdn_noalloc"])
+        "la_query_device_status", "la_status_string", "la_plan", "la_scan_gdn_noalloc",
+        "la_scan_host", "la_host_workspace_size", "la_host_chunk_frames"])
 
 
 def test_library_exports_every_declared_symbol():
@@ -96,6 +97,55 @@ def test_argument_errors_return_before_any_cuda_call():
                           1, 1, 2, 8, 32, 1e-6, P(), ws, None) == la.LA_ERR_INVALID_ARG
     assert L.la_state_step(5, P(), P(), la.LA_BF16, None, None, 1.0, None, None, None, None,
                            1, 1, 2, 8, 32, P(), ws, None) == la.LA_ERR_INVALID_ARG
+
+
+def test_host_chunking_rule():
+    assert la.la_host_chunk_frames(181) == 12          # about 16 chunks
+    assert la.la_host_chunk_frames(8) == 1
+    assert la.la_host_chunk_frames(0) == 1
+    assert la.la_host_chunk_frames(21, 4) == 4
+    assert la.la_host_chunk_frames(6, 50) == 6          # never longer than the clip
+    assert la.la_host_chunk_frames(-1) == 0
+
+
+def test_host_workspace_size():
+    G, R = la.LA_MODE_GDN, la.LA_MODE_RELU
+    n = la.la_host_workspace_size(G, la.LA_BF16, 1, 20, 181, 880, 128, 0)
+    # three slots of q, k, v, o chunks (12 frames) dominate
+    slot_q = 20 * 12 * 880 * 128 * 2
+    assert n >= 3 * 4 * slot_q and n % 256 == 0
+    assert n >= la.la_workspace_size(G, 1, 20, 12, 880, 128) + 3 * 4 * slot_q
+    assert la.la_host_workspace_size(G, la.LA_F32, 1, 20, 181, 880, 128, 0) > n
+    assert la.la_host_workspace_size(G, la.LA_BF16, 1, 20, 181, 880, 128, 24) > n
+    assert la.la_host_workspace_size(R, la.LA_BF16, 1, 20, 21, 1560, 112, 0) > 0
+    assert la.la_host_workspace_size(G, la.LA_BF16, 1, 1, 4, 64, 24, 0) == 0
+    assert la.la_host_workspace_size(G, 5, 1, 1, 4, 64, 32, 0) == 0
+    assert la.la_host_workspace_size(7, la.LA_BF16, 1, 1, 4, 64, 32, 0) == 0
+    assert la.la_host_workspace_size(G, la.LA_BF16, 0, 1, 4, 64, 32, 0) == 0
+
+
+def test_host_scan_argument_errors_return_before_any_cuda_call():
+    L = la.lib
+    P = _fake
+    B, H, F, S, D = 1, 1, 4, 16, 32
+    ws = la.la_host_workspace_size(la.LA_MODE_GDN, la.LA_BF16, B, H, F, S, D, 0)
+
+    def call(mode=la.LA_MODE_GDN, dt=la.LA_BF16, shape=(B, H, F, S, D), w=P(), n=ws,
+             ks=0.1, eps=1e-6, q=P()):
+        return L.la_scan_host(mode, q, P(), P(), P(0x20000), dt, P(), P(), ks, eps,
+                              None, None, None, None, *shape, 0, w, n, None)
+
+    assert call(dt=3) == la.LA_ERR_INVALID_ARG
+    assert call(mode=9) == la.LA_ERR_INVALID_ARG
+    assert call(shape=(1, 1, 4, 16, 24)) == la.LA_ERR_UNSUPPORTED
+    assert call(shape=(1, 0, 4, 16, 32)) == la.LA_ERR_INVALID_ARG
+    assert call(shape=(1, 1, -1, 16, 32)) == la.LA_ERR_INVALID_ARG
+    assert call(ks=float("inf")) == la.LA_ERR_INVALID_ARG
+    assert call(mode=la.LA_MODE_RELU, eps=-1.0) == la.LA_ERR_INVALID_ARG
+    assert call(w=None) == la.LA_ERR_INVALID_ARG
+    assert call(w=P(0x10080)) == la.LA_ERR_INVALID_ARG
+    assert call(n=ws - 1) == la.LA_ERR_INVALID_ARG
+    assert call(q=None) == la.LA_ERR_INVALID_ARG
 
 
 def test_python_binding_refuses_cpu_tensors():
