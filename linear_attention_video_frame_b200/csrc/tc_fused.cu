@@ -4,17 +4,17 @@
 // L2-resident rings instead of HBM round trips.
 //
 // Roles (one block per SM, all blocks co-resident):
-//   chain blocks  (blockIdx < n_chain): each owns up to 4 heads and advances
-//     them frame by frame, interleaved.  The fp32 state of each head lives in
-//     tensor memory; per frame
-//        GDN : M_f = alpha_f (M_{f-1} - G'_f bf16(M_{f-1})) + B_f
-//              (negated-A tcgen05 MMA accumulated onto the state)
-//        ReLU: M_f = M_{f-1} + dM_f,  z_f = z_{f-1} + dz_f
+//   chain blocks  (blockIdx < n_chain): one per head; advances its head frame
+//     by frame.  The fp32 state lives in tensor memory; per frame
+//        GDN : M_f = alpha_f M_{f-1} + G''_f bf16(M_{f-1}) + B~_f
+//              (G''_f = -alpha_f beta_f kappa^2 K_f^T K_f, B~_f = beta_f kappa K_f^T V_f)
+//        ReLU: M_f = M_{f-1} + B~_f,  z_f = z_{f-1} + dz_f
+//              (B~_f = phi(K_f)^T V_f, dz_f = column sums of phi(K_f))
 //     and publishes bf16(M_f) as an MMA operand image.
 //   worker blocks (the rest): take items in ticket order from a global
-//     counter.  A gram item (b,h,f) streams K_f, V_f and produces G'_f, B_f
-//     (GDN) or dM_f, dz_f (ReLU); an output item (b,h,f) streams Q_f and
-//     produces O_f = Q~_f bf16(M_f) (ReLU: / (phi(Q_f) z_f + eps)).
+//     counter.  A gram item (b,h,f) streams K_f, V_f and produces the bf16
+//     images of G''_f and B~_f (ReLU: B~_f and dz_f); an output item (b,h,f)
+//     streams Q_f and produces O_f = Q~_f bf16(M_f) (ReLU: / (phi(Q_f) z_f + eps)).
 //
 // Ordering and progress.  Tickets list, for frame step j, the gram items of
 // frame j of every head and then the output items of frame j - lag.  A gram
@@ -24,11 +24,15 @@
 // resident, so the smallest unfinished ticket can always proceed.
 //
 // Hand-off protocol (per head, ring of kRG / kRM slots):
-//   gram  -> chain : G' image (bulk store), B_f (plain stores), then
+//   gram  -> chain : G'' and B~ images (bulk stores), then
 //                    gram_ready[slot] = f + 1 (release)
-//   chain -> output: M image (bulk store), then chain_done[head] = f + 1
+//   chain -> output: M image (bulk store), then chain_done[head][f & 1] = f + 1
+//                    (even and odd frames are published by two threads, each
+//                    in frame order, so frame f is out once the flag of its
+//                    parity reaches f + 1)
 //   output -> chain: mimg_consumed[slot] = f + 1 once the image is in smem
-//   chain -> gram  : chain_done[head] >= f - kRG + 1 frees gram slot f
+//   chain -> gram  : chain_done[head][g & 1] >= g + 1, g = f - kRG, frees gram
+//                    slot f (frame g was consumed before it was published)
 // Every spin is bounded; a block that gives up records LA_ERR_TIMEOUT in the
 // status word, which makes every other block give up too.
 //
@@ -59,6 +63,19 @@ using namespace tc;
 #ifndef LA_FUSED_LAG
 #define LA_FUSED_LAG 14
 #endif
+#ifndef LA_FUSED_L2_HINTS
+#define LA_FUSED_L2_HINTS 1
+#endif
+#if LA_FUSED_L2_HINTS
+#define LA_POL_KEEP policy_evict_last
+#define LA_POL_STREAM policy_evict_first
+#else
+#define LA_POL_KEEP policy_evict_normal
+#define LA_POL_STREAM policy_evict_normal
+#endif
+#ifndef LA_FUSED_PUB_EVICT_LAST
+#define LA_FUSED_PUB_EVICT_LAST 1
+#endif
 #ifndef LA_FUSED_PUBLAG
 #define LA_FUSED_PUBLAG 1
 #endif
@@ -68,7 +85,7 @@ constexpr int kRM = 16;                 // per-head ring slots: chain -> output
 constexpr int kWStages = LA_FUSED_WSTAGES;   // worker TMA ring (32 KB stages)
 constexpr int kCStages = 2;             // chain operand ring depth
 constexpr int kIQ = 4;                  // worker item queue depth
-constexpr int kThreads = 352;           // 11 warps
+constexpr int kThreads = 384;           // 12 warps
 constexpr int kTokG = 64, kTokO = 128;
 constexpr uint32_t kBoxG = 64 * kTokG * 2;   // 8 KB
 constexpr uint32_t kBoxO = 64 * kTokO * 2;   // 16 KB
@@ -81,11 +98,12 @@ enum : int { kItemStop = 0, kItemGram = 1, kItemOut = 2 };
 // words {kind << 56 | block << 40 | aux, %globaltimer}; plain stores only.
 #ifdef LA_TRACE
 constexpr uint32_t kTraceCap = 4096;
+constexpr uint32_t kTraceWriters = 6;
 __device__ unsigned long long* g_trace = nullptr;
 __device__ __forceinline__ void trace_event(uint32_t& n, uint32_t writer, uint32_t kind, uint64_t aux) {
     unsigned long long* t = g_trace;
     if (!t || n >= kTraceCap) return;
-    unsigned long long* r = t + 2 * ((size_t)(blockIdx.x * 4 + writer) * kTraceCap + n++);
+    unsigned long long* r = t + 2 * ((size_t)(blockIdx.x * kTraceWriters + writer) * kTraceCap + n++);
     r[0] = ((uint64_t)kind << 56) | ((uint64_t)blockIdx.x << 40) | (aux & 0xFFFFFFFFFFull);
     r[1] = global_timer_ns();
 }
@@ -107,7 +125,7 @@ struct FusedParams {
     float* state_out;
     float* z_out;
     unsigned int* status;      // header: [0] status, [1] where, [2] ticket
-    uint32_t* chain_done;      // [BH]
+    uint32_t* chain_done;      // [BH][2]: frames published, per frame parity
     uint32_t* gram_ready;      // [BH][kRG]
     uint32_t* mimg_consumed;   // [BH][kRM]
     uint8_t* gimg;             // [BH][kRG] x kImg  -alpha beta kappa^2 K^T K   (GDN)
@@ -224,7 +242,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                 tma_prefetch_desc(mQ);
                 tma_prefetch_desc(mO);
             }
-            const uint64_t pol = policy_evict_first();
+            const uint64_t pol = LA_POL_STREAM();
             uint32_t iq = 0, nout = 0, ph = 0;
             int s = 0;
             bool ok = true;
@@ -243,7 +261,8 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                 LA_TRACE_EVENT(it.type == kItemGram ? 1 : 2, frame);
                 if (it.type == kItemGram) {
                     if (it.f >= kRG)
-                        ok = ok && wait_flag_ge(&p.chain_done[it.bh], it.f - kRG + 1, ab, 0x402);
+                        ok = ok && wait_flag_ge(&p.chain_done[2 * it.bh + ((it.f - kRG) & 1)],
+                                                it.f - kRG + 1, ab, 0x402);
                     LA_TRACE_EVENT(3, frame);
                     for (int t = 0; t < ntg; ++t) {
                         ok = ok && mbar_wait(&empty[s], ph ^ 1, ab, 0x403);
@@ -261,7 +280,8 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                     // Q does not depend on the chain: fill the ring with Q tiles first,
                     // then wait for the state image of the frame and fetch it.
                     auto fetch_state = [&]() {
-                        ok = ok && wait_flag_ge(&p.chain_done[it.bh], it.f + 1, ab, 0x404);
+                        ok = ok && wait_flag_ge(&p.chain_done[2 * it.bh + (it.f & 1)], it.f + 1, ab,
+                                                0x404);
                         LA_TRACE_EVENT(4, frame);
                         fence_proxy_async_global();
                         ok = ok && mbar_wait(mempty, (nout & 1) ^ 1, ab, 0x405);
@@ -373,8 +393,8 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
         uint32_t iq = 0, qctr = 0, sctr = 0;
         uint32_t dpar = 0;    // bit q: parity of quarter q's next output-tile use (denready)
         bool ok = true;
-        const uint64_t pol_keep = policy_evict_last();     // hand-off data: re-read soon
-        const uint64_t pol_stream = policy_evict_first();  // outputs: never re-read
+        const uint64_t pol_keep = LA_POL_KEEP();          // hand-off data: re-read soon
+        const uint64_t pol_stream = LA_POL_STREAM();       // outputs: never re-read
         LA_TRACE_WRITER(1);
         while (true) {
             if (leader) {
@@ -619,11 +639,14 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
 // chain blocks (one head each)
 // ============================================================================
 // warp 0: loader -- waits for the gram item of each frame and bulk-copies its
-//         G' image and B_f (ReLU: dz_f, dM_f) into a 2-stage ring, with alpha_f;
+//         G'' and B~ images (ReLU: dz_f and B~) into a 2-stage ring;
 // warp 1: TMEM owner + MMA issuer (GDN);
 // warps 2-9: epilogue -- thread <-> (state row, half of the columns);
-// warp 10: publisher -- stores bf16(M_f) (and z_f) to the head's ring slot once
-//         the slot is free, then releases chain_done.
+// warps 10, 11: publishers of the even and the odd frames -- store bf16(M_f)
+//         (and z_f) to the head's ring slot once the slot is free, then release
+//         the progress flag of their parity.  Image buffer b holds the frames
+//         of parity b, so each publisher owns one buffer; two of them keep the
+//         per-frame store and flag latencies off the recurrence.
 // The epilogue's critical path touches only shared and tensor memory.
 template <bool RELU>
 __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) {
@@ -678,7 +701,7 @@ __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) 
         if (lane == 0) {
             int s = 0;
             uint32_t ph = 0;
-            const uint64_t pol_last_use = policy_evict_first();
+            const uint64_t pol_last_use = LA_POL_STREAM();
             LA_TRACE_WRITER(0);
             for (int f = 0; f < F; ++f) {
                 const size_t sidx = (size_t)bh * kRG + f % kRG;
@@ -769,6 +792,7 @@ __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) 
             bool ok = true;
             for (int f = 0; f < F; ++f) {
                 const int frame = bh * F + f;
+                (void)frame;                       // used by the optional trace only
                 const int ib = f & 1;
                 const bool more = f + 1 < F;
                 if (leader) {
@@ -860,52 +884,64 @@ __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) 
                 if (++s == kCStages) { s = 0; ph ^= 1; }
             }
         }
-    } else if (warp == 10) {
-        // ---------------- publisher ----------------
+    } else if (warp >= 10) {
+        // ---------------- publishers (frames of parity par = warp - 10) ----------------
         // Frame f's stores are issued as soon as its image is written and its
-        // ring slot is free.  Up to kPubLag store groups stay in flight; frame
-        // g is published (chain_done = g + 1) once its stores have completed,
-        // so store latency never holds back the image buffers.  The slot-free
-        // flag of the next frame is read one frame ahead.
+        // ring slot is free.  Up to kPubLag store groups stay in flight; a
+        // frame is published (flag = f + 1) once its stores have completed,
+        // so store latency never holds back the image buffer.  The slot-free
+        // flag of the publisher's next frame is read one frame ahead.
+        const int par = warp - 10;
         if (lane == 0) {
             constexpr int kPubLag = LA_FUSED_PUBLAG;
-            const uint64_t pol_keep = policy_evict_last();
-            int published = 0;            // frames published so far
+            const uint64_t pol_keep = LA_POL_KEEP();
+            uint32_t* flag = &p.chain_done[2 * bh + par];
+            LA_TRACE_WRITER(4 + par);
+            int published = 0;            // frames of this parity published so far
             uint32_t seen = 0;            // last value read from the next slot's flag
-            for (int f = 0; f < F; ++f) {
-                const int ib = f & 1;
+            int i = 0;                    // this frame is the i-th of its parity
+            for (int f = par; f < F; f += 2, ++i) {
                 const size_t msidx = (size_t)bh * kRM + f % kRM;
                 if (p.want_output && f >= kRM && seen < (uint32_t)(f - kRM + 1) &&
                     !wait_flag_ge(&p.mimg_consumed[msidx], f - kRM + 1, ab, 0x509))
                     break;
-                if (!mbar_wait(&iready[ib], (f >> 1) & 1, ab, 0x508)) break;
+                LA_TRACE_EVENT(24, (uint64_t)bh * F + f);
+                if (!mbar_wait(&iready[par], i & 1, ab, 0x508)) break;
+                LA_TRACE_EVENT(25, (uint64_t)bh * F + f);
                 if (p.want_output) {
-                    bulk_store_hint(p.mimg + msidx * kImg, imgs + ib * kImg, kImg, pol_keep);
-                    if (RELU) bulk_store_hint(p.zf + msidx * 128, zst + ib * 128, 512, pol_keep);
+#if LA_FUSED_PUB_EVICT_LAST
+                    bulk_store_hint(p.mimg + msidx * kImg, imgs + par * kImg, kImg, pol_keep);
+#else
+                    bulk_store(p.mimg + msidx * kImg, imgs + par * kImg, kImg);
+#endif
+                    if (RELU) bulk_store_hint(p.zf + msidx * 128, zst + par * 128, 512, pol_keep);
                     bulk_commit();
                     bulk_wait_read<0>();
                 }
-                mbar_arrive(&iread[ib]);
+                LA_TRACE_EVENT(26, (uint64_t)bh * F + f);
+                mbar_arrive(&iread[par]);
                 // look at the next frame's slot while this frame's stores drain
-                seen = (p.want_output && f + 1 < F && f + 1 >= kRM)
-                           ? ld_acquire_gpu(&p.mimg_consumed[(size_t)bh * kRM + (f + 1) % kRM])
+                seen = (p.want_output && f + 2 < F && f + 2 >= kRM)
+                           ? ld_acquire_gpu(&p.mimg_consumed[(size_t)bh * kRM + (f + 2) % kRM])
                            : 0u;
                 if (p.want_output) {
-                    if (f + 1 - published > kPubLag) {
+                    if (i + 1 - published > kPubLag) {
                         bulk_wait_all<kPubLag>();
                         fence_proxy_async_global();
-                        published = f + 1 - kPubLag;
-                        st_release_gpu(&p.chain_done[bh], published);
+                        published = i + 1 - kPubLag;
+                        const int g = par + 2 * (published - 1);     // newest completed frame
+                        st_release_gpu(flag, g + 1);
+                        LA_TRACE_EVENT(27, (uint64_t)bh * F + g);
                     }
                 } else {
-                    published = f + 1;
-                    st_release_gpu(&p.chain_done[bh], published);
+                    published = i + 1;
+                    st_release_gpu(flag, f + 1);
                 }
             }
-            if (p.want_output && published < F && !ab.raised()) {
+            if (p.want_output && published < i && !ab.raised()) {
                 bulk_wait_all<0>();
                 fence_proxy_async_global();
-                st_release_gpu(&p.chain_done[bh], F);
+                st_release_gpu(flag, par + 2 * (i - 1) + 1);
             }
         }
     }
@@ -940,7 +976,7 @@ FusedLayout fused_layout(const ScanArgs& a) {
     FusedLayout L;
     size_t off = kWsHeaderBytes;
     L.chain_done = off;
-    off += bh * 4;
+    off += bh * 2 * 4;
     L.gram_ready = off;
     off += bh * kRG * 4;
     L.mimg_consumed = off;
