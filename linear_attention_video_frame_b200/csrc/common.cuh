@@ -65,6 +65,12 @@ size_t tc_workspace_bytes(const ScanArgs& a);
 int tc_kernel_count(const ScanArgs& a);
 cudaError_t launch_tc(const ScanArgs& a, cudaStream_t st);
 
+// Wide-head tensor-core path: bf16 inputs, 128 < D <= 256, F > 0.
+bool wide_eligible(const ScanArgs& a);
+size_t wide_workspace_bytes(const ScanArgs& a);
+int wide_kernel_count(const ScanArgs& a);
+cudaError_t launch_wide(const ScanArgs& a, cudaStream_t st);
+
 // Fused persistent tensor-core path (one cooperative launch).
 bool fused_eligible(const ScanArgs& a);
 size_t fused_workspace_bytes(const ScanArgs& a);

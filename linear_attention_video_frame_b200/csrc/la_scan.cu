@@ -57,6 +57,8 @@ bool force_simt() {
 
 bool use_tc(const ScanArgs& a) { return !force_simt() && tc_eligible(a); }
 
+bool use_wide(const ScanArgs& a) { return !force_simt() && wide_eligible(a); }
+
 // LA_SCAN_NO_FUSE=1 keeps tensor-core calls on the three-kernel path (tests
 // compare the two).
 bool use_fused(const ScanArgs& a) {
@@ -66,7 +68,8 @@ bool use_fused(const ScanArgs& a) {
 
 size_t workspace_needed(const ScanArgs& a) {
     if (use_fused(a)) return fused_workspace_bytes(a);
-    return use_tc(a) ? tc_workspace_bytes(a) : simt_workspace_bytes(a);
+    if (use_tc(a)) return tc_workspace_bytes(a);
+    return use_wide(a) ? wide_workspace_bytes(a) : simt_workspace_bytes(a);
 }
 
 // Validation common to every entry point.  `need_q` is false for a state step.
@@ -109,7 +112,8 @@ la_status run(const ScanArgs& a, cudaStream_t st) {
     }
     cudaError_t e = use_fused(a) ? launch_fused(a, st)
                     : use_tc(a)  ? launch_tc(a, st)
-                                 : launch_simt(a, st);
+                    : use_wide(a) ? launch_wide(a, st)
+                                  : launch_simt(a, st);
     if (e != cudaSuccess) { cudaGetLastError(); return LA_ERR_CUDA; }
     return LA_OK;
 }
@@ -217,6 +221,10 @@ extern "C" const char* la_plan(la_mode mode, la_dtype dt, int B, int H, int F, i
     if (use_tc(a)) {
         if (kernels) *kernels = tc_kernel_count(a);
         return "tcgen05";
+    }
+    if (use_wide(a)) {
+        if (kernels) *kernels = wide_kernel_count(a);
+        return "tcgen05_wide";
     }
     if (kernels) *kernels = 1;
     return "simt_f32";

@@ -1,0 +1,901 @@
+// Tensor-core (tcgen05) scan for wide heads: bf16 inputs, 128 < D <= 256.
+//
+// A D x D state of up to 256 x 256 fp32 is as large as a whole SM's tensor
+// memory, so the work is cut into 128-row / 128-column blocks (dimensions
+// beyond D are zero padding that the TMA fills and the math keeps at zero):
+//
+//   gram   (frame-parallel) one CTA per (b, h, f, key-row block r):
+//            GDN : G''_f[r] = -alpha_f beta_f kappa^2 K[:, r]^T K   (bf16 image)
+//                  B~_f[r]  =  beta_f kappa     K[:, r]^T V         (bf16 tiles)
+//            ReLU: dM_f[r] = phi(K)[:, r]^T V (fp32), dz_f[r] = phi(K)[:, r]^T 1
+//   chain  (sequential per (b, h)); column blocks of the state evolve
+//          independently, so each column half c has its own CTA:
+//            GDN : M_f[:, c] = alpha_f M_{f-1}[:, c] + G''_f bf16(M_{f-1})[:, c]
+//                              + B~_f[:, c]   (fp32 state in tensor memory)
+//            ReLU: M_f = M_{f-1} + dM_f, z_f = z_{f-1} + dz_f (a plain prefix
+//                  sum, held in registers, one CTA per 32 state columns)
+//          and writes bf16(M_f)[:, c] as an MMA operand image.
+//   output (frame-parallel) one CTA per (b, h, f, value-column half c):
+//            O_f[:, c] = Q~_f bf16(M_f)[:, c]  (ReLU: / (phi(Q_f) z_f + eps))
+//
+// Equations: the frame-wise Gated DeltaNet of the SANA-WM paper summary
+// (section 3, "Hybrid GDN/Softmax Attention") in its affine form, and the
+// block-causal ReLU linear attention of the SANA-Video talk (block KV cache
+// segment).  The split of the state into independent column blocks is plain
+// linear algebra: M_f[:, c] depends only on M_{f-1}[:, c].
+//
+// Operand images (128-byte swizzle, 16-byte chunk j of row r at j ^ (r % 8)):
+//   G''[r] image : 128 rows (key i in block r) x 256 columns (key j), K-major,
+//                  four 64-column blocks of 16 KB.
+//   M[:, c] image: 256 rows (key i) x 128 columns (value j in half c),
+//                  MN-major, two 64-column blocks of 32 KB.
+// dM blocks (ReLU) are fp32 [128 x 256] "quad-interleaved": element (i, j) at
+// ((j / 4) * 128 + i) * 4 + j % 4; B~ tiles (GDN) are bf16 [128 x 128] per
+// (frame, r, c), 16-byte chunk jc (columns 8 jc .. 8 jc + 7) of row i at
+// (jc * 128 + i) * 16 bytes.  Either way a warp's 32 rows touch 512
+// contiguous bytes.  B~ is kept in bf16 like the state image; the state
+// itself and all accumulation stay fp32.
+#include <algorithm>
+
+#include "tc_common.cuh"
+#include "tmap.cuh"
+
+namespace la {
+namespace {
+
+using namespace tc;
+
+constexpr int kDW = 256;                      // padded head dimension
+constexpr int kTokG = 64;                     // tokens per gram tile
+constexpr int kTokO = 128;                    // tokens per output tile
+constexpr uint32_t kBoxG = 64 * kTokG * 2;    // 8 KB: 64 columns x 64 tokens
+constexpr uint32_t kBoxO = 64 * kTokO * 2;    // 16 KB: 64 columns x 128 tokens
+constexpr uint32_t kGTile = 4 * kBoxG;        // 32 KB: one 256-wide gram tile of K or V
+constexpr uint32_t kOTile = 4 * kBoxO;        // 64 KB: one 256-wide output tile of Q
+constexpr uint32_t kGImg = 65536;             // G''[r] image
+constexpr uint32_t kMImg = 65536;             // M[:, c] image
+constexpr uint32_t kQuad = 128 * 256;         // floats of one fp32 [128 x 256] block
+constexpr uint32_t kBTile = 16 * 128;         // 16-byte chunks of one bf16 [128 x 128] B~ tile
+constexpr int kOAcc = 4;                      // output accumulator slots (128 columns each)
+
+struct WideParams {
+    const float* alpha;
+    const float* beta;
+    const float* state_in;
+    const float* z_in;
+    float* state_out;
+    float* z_out;
+    unsigned int* status;   // workspace header (status, where)
+    uint8_t* gimg;          // [BHF][2] x kGImg                 (GDN)
+    uint4* btil;            // [BHF][2][2] x kBTile bf16 B~     (GDN)
+    float* bmat;            // [BHF][2] x kQuad fp32 dM          (ReLU)
+    float* dz;              // [BHF][2] x 128                   (ReLU)
+    uint8_t* mimg;          // [BHF][2] x kMImg
+    float* zf;              // [BHF] x 256                      (ReLU)
+    float k_scale;
+    float eps;
+    int BH, F, S, D;
+    int want_output;
+};
+
+// Write 16 consecutive columns [c0, c0 + 16) of row `row` of a swizzled bf16
+// image whose 64-column blocks are `blk_bytes` apart.
+__device__ __forceinline__ void store_row16(uint8_t* img, uint32_t blk_bytes, int row, int c0,
+                                            const float (&v)[16]) {
+    const int blk = c0 >> 6, ch = (c0 & 63) >> 3;
+    uint4 a = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                         pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+    uint4 b = make_uint4(pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
+                         pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+    *reinterpret_cast<uint4*>(img + blk * blk_bytes + sw128_off(row, ch)) = a;
+    *reinterpret_cast<uint4*>(img + blk * blk_bytes + sw128_off(row, ch + 1)) = b;
+}
+
+// Offset (in floats) of element (row, col) of a quad-interleaved fp32 block.
+__device__ __forceinline__ uint32_t quad_off(int row, int col) {
+    return ((uint32_t)(col >> 2) * 128u + (uint32_t)row) * 4u + (uint32_t)(col & 3);
+}
+
+// ============================================================================
+// gram: per-frame contractions over tokens, one key-row block per CTA
+// ============================================================================
+// warp 0: TMA producer; warp 1: TMEM owner + MMA issuer; warps 2-5: epilogue;
+// warps 6-9 (ReLU): phi(K) in place before the MMA.
+template <bool RELU>
+__global__ void __launch_bounds__(RELU ? 320 : 192, 1)
+wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
+                 const __grid_constant__ CUtensorMap mapV) {
+    constexpr int kStages = RELU ? 3 : 2;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* ring = smem;                                  // kStages x (K 32 KB | V 32 KB)
+    uint8_t* stage_img = ring + kStages * 2 * kGTile;      // G''[r] image staging (GDN)
+    uint8_t* ones = stage_img + (RELU ? 0 : kGImg);        // 2 KB of bf16 1.0 (ReLU)
+    uint64_t* full = reinterpret_cast<uint64_t*>(ones + 2048);
+    uint64_t* empty = full + kStages;
+    uint64_t* xform = empty + kStages;
+    uint64_t* accfull = xform + kStages;
+    uint64_t* accempty = accfull + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + 1);
+    uint32_t* abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int D = p.D;
+    const int nbx = (D + 63) / 64;                         // column boxes that hold data
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&xform[s], 4);
+        }
+        mbar_init(accfull, 1);
+        mbar_init(accempty, 4);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    // Column boxes past D are never loaded: zero them once.
+    for (int s = 0; s < kStages; ++s)
+        for (int t = 0; t < 2; ++t)
+            for (int b = nbx; b < 4; ++b) {
+                uint4* z = reinterpret_cast<uint4*>(ring + s * 2 * kGTile + t * kGTile + b * kBoxG);
+                for (int i = threadIdx.x; i < (int)(kBoxG / 16); i += blockDim.x)
+                    z[i] = make_uint4(0, 0, 0, 0);
+            }
+    if (RELU)
+        for (int i = threadIdx.x; i < 2048 / 4; i += blockDim.x)
+            reinterpret_cast<uint32_t*>(ones)[i] = 0x3F803F80u;
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    const Abort ab{abort_flag, p.status};
+    const int nitems = p.BH * p.F * 2;
+    const int nt = (p.S + kTokG - 1) / kTokG;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&mapK);
+            tma_prefetch_desc(&mapV);
+            const uint64_t pol = policy_evict_first();
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x) {
+                const int frame = item >> 1;
+                for (int t = 0; t < nt; ++t) {
+                    if (!(ok = mbar_wait(&empty[s], ph ^ 1, ab, 0x601))) break;
+                    uint8_t* st = ring + s * 2 * kGTile;
+                    mbar_expect_tx(&full[s], 2 * nbx * kBoxG);
+                    for (int b = 0; b < nbx; ++b) {
+                        tma_load_3d(st + b * kBoxG, &mapK, &full[s], 64 * b, t * kTokG, frame, pol);
+                        tma_load_3d(st + kGTile + b * kBoxG, &mapV, &full[s], 64 * b, t * kTokG,
+                                    frame, pol);
+                    }
+                    if (++s == kStages) { s = 0; ph ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idW = idesc_bf16(128, kDW, true, true);
+            const uint32_t idZ = idesc_bf16(128, 16, true, false);
+            const uint64_t ones_d = sdesc_sw128(smem_u32(ones), 16, 1024);
+            // GDN: G at columns [0, 256), B~ at [256, 512); ReLU: dM at [0, 256), dz at 256.
+            const uint32_t dA = tbase, dB = tbase + 256;
+            int s = 0, li = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
+                const int r = item & 1;
+                if (!(ok = mbar_wait(accempty, (li & 1) ^ 1, ab, 0x602))) break;
+                tc_fence_after();
+                for (int t = 0; t < nt; ++t) {
+                    if (!(ok = mbar_wait(RELU ? &xform[s] : &full[s], ph, ab, 0x603))) break;
+                    tc_fence_after();
+                    const uint32_t sk = smem_u32(ring + s * 2 * kGTile), sv = sk + kGTile;
+#pragma unroll
+                    for (int k = 0; k < kTokG / 16; ++k) {
+                        // A = K[:, block r]^T (MN-major), B = K or V (MN-major, N = 256)
+                        const uint64_t ad = sdesc_sw128(sk + 2 * r * kBoxG + k * 2048, kBoxG, 1024);
+                        const uint64_t bk = sdesc_sw128(sk + k * 2048, kBoxG, 1024);
+                        const uint64_t bv = sdesc_sw128(sv + k * 2048, kBoxG, 1024);
+                        const uint32_t acc = (t | k) ? 1u : 0u;
+                        if (RELU) {
+                            mma_bf16(dA, ad, bv, idW, acc);
+                            mma_bf16(dB, ad, ones_d, idZ, acc);
+                        } else {
+                            mma_bf16(dA, ad, bk, idW, acc);
+                            mma_bf16(dB, ad, bv, idW, acc);
+                        }
+                    }
+                    mma_commit(&empty[s]);
+                    if (++s == kStages) { s = 0; ph ^= 1; }
+                }
+                if (ok) mma_commit(accfull);
+            }
+        }
+    } else if (warp < 6) {
+        // ---------------- epilogue: TMEM -> workspace ----------------
+        const int q = warp & 3, row = q * 32 + lane;
+        const bool issuer = (threadIdx.x == 64);
+        int li = 0;
+        bool ok = true;     // every epilogue warp runs every named barrier, even after an abort
+        for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++li) {
+            const int frame = item >> 1;
+            ok = ok && mbar_wait(accfull, li & 1, ab, 0x604);
+            tc_fence_after();
+            const uint32_t tl = tbase + (uint32_t(q * 32) << 16);
+            if (!RELU) {
+                const float al = p.alpha[frame], bt = p.beta[frame];
+                const float sg = -al * bt * p.k_scale * p.k_scale, sw = bt * p.k_scale;
+                if (issuer) bulk_wait_read<0>();       // staging free again
+                named_bar_sync(1, 128);
+                for (int c0 = 0; c0 < kDW && ok; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tl + c0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] *= sg;
+                    store_row16(stage_img, 16384, row, c0, v);
+                }
+                for (int c0 = 0; c0 < kDW && ok; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tl + 256 + c0, v);
+                    tmem_wait_ld();
+                    uint4* bt = p.btil + ((size_t)item * 2 + (c0 >> 7)) * kBTile;
+                    const int jc = (c0 & 127) >> 3;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        bt[(jc + h) * 128 + row] = make_uint4(
+                            pack_bf16x2(v[8 * h] * sw, v[8 * h + 1] * sw),
+                            pack_bf16x2(v[8 * h + 2] * sw, v[8 * h + 3] * sw),
+                            pack_bf16x2(v[8 * h + 4] * sw, v[8 * h + 5] * sw),
+                            pack_bf16x2(v[8 * h + 6] * sw, v[8 * h + 7] * sw));
+                }
+            } else if (ok) {
+                float* bq = p.bmat + (size_t)item * kQuad;
+                for (int c0 = 0; c0 < kDW; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tl + c0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        *reinterpret_cast<float4*>(bq + quad_off(row, c0 + 4 * u)) =
+                            make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                }
+                float v[16];
+                tmem_ld16(tl + 256, v);
+                tmem_wait_ld();
+                p.dz[(size_t)item * 128 + row] = v[0];
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(accempty);
+            if (!RELU) {
+                fence_proxy_async_smem();
+                named_bar_sync(1, 128);
+                if (issuer && ok) {
+                    bulk_store(p.gimg + (size_t)item * kGImg, stage_img, kGImg);
+                    bulk_commit();
+                }
+            }
+        }
+        if (issuer) bulk_wait_all<0>();
+    } else {
+        // ---------------- ReLU transform: phi(K) in place ----------------
+        const int tl = threadIdx.x - 192;          // 0..127
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x) {
+            for (int t = 0; t < nt; ++t) {
+                if (!(ok = mbar_wait(&full[s], ph, ab, 0x605))) break;
+                uint4* kt = reinterpret_cast<uint4*>(ring + s * 2 * kGTile);
+                for (int i = tl; i < nbx * (int)kBoxG / 16; i += 128) {
+                    uint4 x = kt[i];
+                    x.x = relu_bf16x2(x.x); x.y = relu_bf16x2(x.y);
+                    x.z = relu_bf16x2(x.z); x.w = relu_bf16x2(x.w);
+                    kt[i] = x;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xform[s]);
+                if (++s == kStages) { s = 0; ph ^= 1; }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tbase, 512);
+}
+
+// ============================================================================
+// chain (GDN): one CTA per (b, h, value-column half c), state in TMEM
+// ============================================================================
+// warp 0: bulk loader of the two G''[r] row blocks of each frame;
+// warp 1: TMEM owner + MMA issuer; warps 2-9: epilogue, warp w handles key-row
+// block r = (w - 2) / 4 and TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31;
+// warp 10: publisher of the M[:, c] image of each frame.
+__global__ void __launch_bounds__(352, 1)
+wide_chain_gdn_kernel(const WideParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* stage = smem;                                 // 2 x 64 KB: G''[0], G''[1]
+    uint8_t* img = stage + 2 * kGImg;                      // M[:, c] image (64 KB)
+    uint64_t* gfull = reinterpret_cast<uint64_t*>(img + kMImg);
+    uint64_t* gempty = gfull + 2;
+    uint64_t* mdone = gempty + 2;      // both row-block MMAs of the frame finished
+    uint64_t* mready = mdone + 1;      // TMEM holds alpha M, image of M written (both groups)
+    uint64_t* idone = mready + 1;      // image of the frame written (both groups)
+    uint64_t* ipub = idone + 1;        // publisher has read the image out
+    int* bc_ok = reinterpret_cast<int*>(ipub + 1);          // [2] per row group
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bc_ok + 2);
+    uint32_t* abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.x >> 1, c = blockIdx.x & 1;
+    const int F = p.F, D = p.D;
+    if (threadIdx.x == 0) {
+        for (int r = 0; r < 2; ++r) {
+            mbar_init(&gfull[r], 1);
+            mbar_init(&gempty[r], 1);
+        }
+        mbar_init(mdone, 1);
+        mbar_init(mready, 2);
+        mbar_init(idone, 2);
+        mbar_init(ipub, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 256);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tM = *tmem_slot;
+    const Abort ab{abort_flag, p.status};
+
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int f = 0; f < F; ++f) {
+                bool ok = true;
+                for (int r = 0; r < 2 && ok; ++r) {
+                    if (!(ok = mbar_wait(&gempty[r], (f & 1) ^ 1, ab, 0x701))) break;
+                    mbar_expect_tx(&gfull[r], kGImg);
+                    bulk_load(stage + r * kGImg, p.gimg + ((size_t)bh * F + f) * 2 * kGImg + r * kGImg,
+                              kGImg, &gfull[r]);
+                }
+                if (!ok) break;
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idC = idesc_bf16(128, 128, false, true);
+            const uint32_t ib = smem_u32(img);
+            for (int f = 0; f < F; ++f) {
+                if (!mbar_wait(mready, f & 1, ab, 0x702)) break;
+                bool ok = true;
+                for (int r = 0; r < 2 && ok; ++r) {
+                    if (!(ok = mbar_wait(&gfull[r], f & 1, ab, 0x703))) break;
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(stage + r * kGImg);
+                    for (int kk = 0; kk < kDW / 16; ++kk) {
+                        const uint64_t ad = sdesc_sw128(sa + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
+                        const uint64_t bd = sdesc_sw128(ib + kk * 2048, 32768, 1024);
+                        mma_bf16(tM + r * 128, ad, bd, idC, 1u);
+                    }
+                    mma_commit(&gempty[r]);
+                }
+                if (!ok) break;
+                mma_commit(mdone);
+            }
+        }
+    } else if (warp < 10) {
+        // ---------------- epilogue ----------------
+        const int r = (warp - 2) >> 2, q = warp & 3, row = q * 32 + lane;
+        const int i = 128 * r + row;                      // key row of the state
+        const bool live = i < D;
+        const bool leader = ((threadIdx.x - 64) & 127) == 0;
+        const int bar_id = 1 + r;
+        const uint32_t tl = tM + (uint32_t(q * 32) << 16) + r * 128;
+        const float* ap = p.alpha + (size_t)bh * F;
+        // initial state: image of M_0 and alpha_0 M_0 in TMEM
+        {
+            const float a0 = __ldg(ap);
+            for (int j0 = 0; j0 < 128; j0 += 16) {
+                float v[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int col = 128 * c + j0 + e;
+                    v[e] = (p.state_in && live && col < D) ? p.state_in[((size_t)bh * D + i) * D + col]
+                                                           : 0.f;
+                }
+                store_row16(img, 32768, i, j0, v);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) v[e] *= a0;
+                tmem_st16(tl + j0, v);
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(bar_id, 128);
+            if (leader) mbar_arrive(mready);
+        }
+        // B~ row of the coming frame: 128 bf16 columns in 16 registers of 16 bytes,
+        // fetched one frame ahead so the loads never wait on the critical path.
+        uint4 bb[16];
+        auto fetch_b = [&](int f) {
+            const uint4* bt = p.btil + ((((size_t)bh * F + f) * 2 + r) * 2 + c) * kBTile;
+#pragma unroll
+            for (int jc = 0; jc < 16; ++jc) bb[jc] = __ldg(bt + jc * 128 + row);
+        };
+        fetch_b(0);
+        bool ok = true;
+        for (int f = 0; f < F; ++f) {
+            const bool more = f + 1 < F;
+            const float an = more ? __ldg(ap + f + 1) : 1.f;
+            if (leader) {
+                ok = ok && mbar_wait(mdone, f & 1, ab, 0x704);
+                if (f >= 1) ok = ok && mbar_wait(ipub, (f - 1) & 1, ab, 0x705);
+                bc_ok[r] = ok;
+            }
+            named_bar_sync(bar_id, 128);
+            const bool go = bc_ok[r];
+            tc_fence_after();
+            if (go) {
+#pragma unroll
+                for (int j0 = 0; j0 < 128; j0 += 16) {
+                    float v[16];
+                    tmem_ld16(tl + j0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint4 w = bb[j0 / 8 + h];
+                        v[8 * h + 0] += bf16_lo(w.x); v[8 * h + 1] += bf16_hi(w.x);
+                        v[8 * h + 2] += bf16_lo(w.y); v[8 * h + 3] += bf16_hi(w.y);
+                        v[8 * h + 4] += bf16_lo(w.z); v[8 * h + 5] += bf16_hi(w.z);
+                        v[8 * h + 6] += bf16_lo(w.w); v[8 * h + 7] += bf16_hi(w.w);
+                    }
+                    store_row16(img, 32768, i, j0, v);
+                    if (!more) {
+                        if (p.state_out && live) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) {
+                                const int col = 128 * c + j0 + e;
+                                if (col < D) p.state_out[((size_t)bh * D + i) * D + col] = v[e];
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] *= an;
+                        tmem_st16(tl + j0, v);
+                    }
+                }
+                if (more) fetch_b(f + 1);
+            }
+            tmem_wait_st();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(bar_id, 128);
+            if (leader) {
+                mbar_arrive(mready);
+                mbar_arrive(idone);
+            }
+        }
+    } else {
+        // ---------------- publisher ----------------
+        if (lane == 0) {
+            for (int f = 0; f < F; ++f) {
+                if (!mbar_wait(idone, f & 1, ab, 0x706)) break;
+                if (p.want_output) {
+                    bulk_store(p.mimg + (((size_t)bh * F + f) * 2 + c) * kMImg, img, kMImg);
+                    bulk_commit();
+                    bulk_wait_read<0>();
+                }
+                mbar_arrive(ipub);
+            }
+            bulk_wait_all<0>();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tM, 256);
+}
+
+// ============================================================================
+// chain (ReLU): prefix sums of dM and dz, one CTA per (b, h, 32 state columns)
+// ============================================================================
+// Thread i owns key row i and 32 columns of the state in registers; the
+// next frame's increments are fetched while the current frame is written.
+__global__ void __launch_bounds__(256)
+wide_chain_relu_kernel(const WideParams p) {
+    const int bh = blockIdx.x >> 3, cc = blockIdx.x & 7;
+    const int i = threadIdx.x, r = i >> 7, row = i & 127;
+    const int F = p.F, D = p.D;
+    const int c = cc >> 2, jl0 = (cc & 3) * 32;        // column half and first local column
+    const int j0 = 32 * cc;                           // first global column
+    const bool live = i < D;
+    float s[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+        s[e] = (p.state_in && live && j0 + e < D) ? p.state_in[((size_t)bh * D + i) * D + j0 + e] : 0.f;
+    float z = (cc == 0 && p.z_in && live) ? p.z_in[(size_t)bh * D + i] : 0.f;
+
+    float4 nx[8];
+    float dzn = 0.f;
+    auto fetch = [&](int f) {
+        const float* bq = p.bmat + (((size_t)bh * F + f) * 2 + r) * kQuad;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) nx[u] = __ldg(reinterpret_cast<const float4*>(bq + quad_off(row, j0 + 4 * u)));
+        if (cc == 0) dzn = __ldg(p.dz + (((size_t)bh * F + f) * 2 + r) * 128 + row);
+    };
+    if (F > 0) fetch(0);
+    for (int f = 0; f < F; ++f) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            s[4 * u] += nx[u].x; s[4 * u + 1] += nx[u].y;
+            s[4 * u + 2] += nx[u].z; s[4 * u + 3] += nx[u].w;
+        }
+        z += dzn;
+        if (f + 1 < F) fetch(f + 1);
+        if (p.want_output) {
+            uint8_t* im = p.mimg + (((size_t)bh * F + f) * 2 + c) * kMImg;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const int jl = jl0 + 8 * w;
+                const uint4 x = make_uint4(pack_bf16x2(s[8 * w], s[8 * w + 1]),
+                                           pack_bf16x2(s[8 * w + 2], s[8 * w + 3]),
+                                           pack_bf16x2(s[8 * w + 4], s[8 * w + 5]),
+                                           pack_bf16x2(s[8 * w + 6], s[8 * w + 7]));
+                *reinterpret_cast<uint4*>(im + (jl >> 6) * 32768 + sw128_off(i, (jl & 63) >> 3)) = x;
+            }
+            if (cc == 0) p.zf[((size_t)bh * F + f) * 256 + i] = z;
+        }
+    }
+    if (p.state_out && live) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+            if (j0 + e < D) p.state_out[((size_t)bh * D + i) * D + j0 + e] = s[e];
+    }
+    if (cc == 0 && p.z_out && live) p.z_out[(size_t)bh * D + i] = z;
+}
+
+// ============================================================================
+// output: O_f[:, c] = Q~_f bf16(M_f)[:, c]   (ReLU: / (phi(Q_f) z_f + eps))
+// ============================================================================
+// warp 0: producer (M image and z by bulk copy, Q tiles by TMA); warp 1: TMEM
+// owner + MMA issuer; warps 2-5: epilogue (TMEM -> bf16 -> TMA store, one
+// 64-column box at a time); warps 6-9 (ReLU): phi(Q) in place and the
+// per-token denominators.
+template <bool RELU>
+__global__ void __launch_bounds__(RELU ? 320 : 192, 1)
+wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
+                   const __grid_constant__ CUtensorMap mapO) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* qring = smem;                                 // 2 x 64 KB Q tiles
+    uint8_t* mbuf = qring + 2 * kOTile;                    // M[:, c] image (64 KB)
+    uint8_t* ostage = mbuf + kMImg;                        // one 64-column output box (16 KB)
+    float* zbuf = reinterpret_cast<float*>(ostage + kBoxO);           // 256
+    float* denbuf = zbuf + 256;                                       // kOAcc x 128
+    uint64_t* qfull = reinterpret_cast<uint64_t*>(denbuf + kOAcc * 128);
+    uint64_t* qempty = qfull + 2;
+    uint64_t* xform = qempty + 2;
+    uint64_t* mfull = xform + 2;
+    uint64_t* mempty = mfull + 1;
+    uint64_t* accfull = mempty + 1;
+    uint64_t* accempty = accfull + kOAcc;
+    uint64_t* denready = accempty + kOAcc;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(denready + kOAcc);
+    uint32_t* abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int D = p.D;
+    const int nbx = (D + 63) / 64;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&qfull[s], 1);
+            mbar_init(&qempty[s], 1);
+            mbar_init(&xform[s], 4);
+        }
+        mbar_init(mfull, 1);
+        mbar_init(mempty, RELU ? 5 : 1);
+        for (int a = 0; a < kOAcc; ++a) {
+            mbar_init(&accfull[a], 1);
+            mbar_init(&accempty[a], 4);
+            mbar_init(&denready[a], 4);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    for (int s = 0; s < 2; ++s)
+        for (int b = nbx; b < 4; ++b) {
+            uint4* z = reinterpret_cast<uint4*>(qring + s * kOTile + b * kBoxO);
+            for (int i = threadIdx.x; i < (int)(kBoxO / 16); i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
+        }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    const Abort ab{abort_flag, p.status};
+    const int nitems = p.BH * p.F * 2;
+    const int nt = (p.S + kTokO - 1) / kTokO;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&mapQ);
+            tma_prefetch_desc(&mapO);
+            const uint64_t pol = policy_evict_first();
+            int s = 0, li = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
+                const int frame = item >> 1;
+                if (!(ok = mbar_wait(mempty, (li & 1) ^ 1, ab, 0x801))) break;
+                mbar_expect_tx(mfull, kMImg + (RELU ? 1024 : 0));
+                bulk_load(mbuf, p.mimg + (size_t)item * kMImg, kMImg, mfull);
+                if (RELU) bulk_load(zbuf, p.zf + (size_t)frame * 256, 1024, mfull);
+                for (int t = 0; t < nt; ++t) {
+                    if (!(ok = mbar_wait(&qempty[s], ph ^ 1, ab, 0x802))) break;
+                    uint8_t* st = qring + s * kOTile;
+                    mbar_expect_tx(&qfull[s], nbx * kBoxO);
+                    for (int b = 0; b < nbx; ++b)
+                        tma_load_3d(st + b * kBoxO, &mapQ, &qfull[s], 64 * b, t * kTokO, frame, pol);
+                    if (++s == 2) { s = 0; ph ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idO = idesc_bf16(128, 128, false, true);
+            const uint32_t mb = smem_u32(mbuf);
+            int s = 0, li = 0, gt = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
+                if (!(ok = mbar_wait(mfull, li & 1, ab, 0x803))) break;
+                for (int t = 0; t < nt; ++t, ++gt) {
+                    const int a = gt % kOAcc;
+                    if (!(ok = mbar_wait(&accempty[a], ((gt / kOAcc) & 1) ^ 1, ab, 0x804))) break;
+                    if (!(ok = mbar_wait(RELU ? &xform[s] : &qfull[s], ph, ab, 0x805))) break;
+                    tc_fence_after();
+                    const uint32_t qa = smem_u32(qring + s * kOTile);
+                    for (int kk = 0; kk < 4 * nbx; ++kk) {
+                        const uint64_t ad = sdesc_sw128(qa + (kk >> 2) * kBoxO + (kk & 3) * 32, 16, 1024);
+                        const uint64_t bd = sdesc_sw128(mb + kk * 2048, 32768, 1024);
+                        mma_bf16(tbase + a * 128, ad, bd, idO, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&qempty[s]);
+                    mma_commit(&accfull[a]);
+                    if (++s == 2) { s = 0; ph ^= 1; }
+                }
+                if (ok) mma_commit(mempty);
+            }
+        }
+    } else if (warp < 6) {
+        // ---------------- epilogue ----------------
+        const int q = warp & 3, row = q * 32 + lane;
+        const bool issuer = (threadIdx.x == 64);
+        int gt = 0;
+        bool ok = true;     // every epilogue warp runs every named barrier, even after an abort
+        for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+            const int frame = item >> 1, c = item & 1;
+            for (int t = 0; t < nt; ++t, ++gt) {
+                const int a = gt % kOAcc;
+                ok = ok && mbar_wait(&accfull[a], (gt / kOAcc) & 1, ab, 0x806);
+                if (RELU) ok = ok && mbar_wait(&denready[a], (gt / kOAcc) & 1, ab, 0x807);
+                tc_fence_after();
+                const float inv = (RELU && ok) ? 1.f / denbuf[a * 128 + row] : 1.f;
+                const uint32_t tl = tbase + (uint32_t(q * 32) << 16) + a * 128;
+                for (int b = 0; b < 2; ++b) {
+                    const int x0 = 128 * c + 64 * b;
+                    if (x0 >= D) break;                       // uniform over the block
+                    if (issuer) bulk_wait_read<0>();          // staging no longer read
+                    named_bar_sync(1, 128);
+                    for (int c0 = 0; c0 < 64 && ok; c0 += 16) {
+                        float v[16];
+                        tmem_ld16(tl + 64 * b + c0, v);
+                        tmem_wait_ld();
+                        if (RELU) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) v[e] *= inv;
+                        }
+                        store_row16(ostage, 16384, row, c0, v);
+                    }
+                    fence_proxy_async_smem();
+                    named_bar_sync(1, 128);
+                    if (issuer && ok) {
+                        tma_store_3d(&mapO, ostage, x0, t * kTokO, frame);
+                        bulk_commit();
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&accempty[a]);
+            }
+        }
+        if (issuer) bulk_wait_all<0>();
+    } else {
+        // ---------------- ReLU: phi(Q) in place, denominators ----------------
+        const int row = threadIdx.x - 192;                // token row in the tile
+        int s = 0, li = 0, gt = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
+            if (!(ok = mbar_wait(mfull, li & 1, ab, 0x808))) break;
+            for (int t = 0; t < nt; ++t, ++gt) {
+                const int a = gt % kOAcc;
+                if (!(ok = mbar_wait(&qfull[s], ph, ab, 0x809))) break;
+                if (!(ok = mbar_wait(&accempty[a], ((gt / kOAcc) & 1) ^ 1, ab, 0x80a))) break;
+                uint8_t* st = qring + s * kOTile;
+                float den = 0.f;
+                for (int b = 0; b < nbx; ++b) {
+                    for (int ch = 0; ch < 8; ++ch) {
+                        uint4* pch = reinterpret_cast<uint4*>(st + b * kBoxO + sw128_off(row, ch));
+                        uint4 x = *pch;
+                        x.x = relu_bf16x2(x.x); x.y = relu_bf16x2(x.y);
+                        x.z = relu_bf16x2(x.z); x.w = relu_bf16x2(x.w);
+                        *pch = x;
+                        const float* zz = zbuf + b * 64 + ch * 8;
+                        den = fmaf(bf16_lo(x.x), zz[0], den);
+                        den = fmaf(bf16_hi(x.x), zz[1], den);
+                        den = fmaf(bf16_lo(x.y), zz[2], den);
+                        den = fmaf(bf16_hi(x.y), zz[3], den);
+                        den = fmaf(bf16_lo(x.z), zz[4], den);
+                        den = fmaf(bf16_hi(x.z), zz[5], den);
+                        den = fmaf(bf16_lo(x.w), zz[6], den);
+                        den = fmaf(bf16_hi(x.w), zz[7], den);
+                    }
+                }
+                denbuf[a * 128 + row] = den + p.eps;
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&xform[s]);
+                    mbar_arrive(&denready[a]);
+                }
+                if (++s == 2) { s = 0; ph ^= 1; }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(mempty);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) tmem_dealloc(tbase, 512);
+}
+
+// ----------------------------------------------------------------------------
+// Host side
+// ----------------------------------------------------------------------------
+struct WideLayout {
+    size_t gimg, btil, bmat, dz, mimg, zf, total;
+};
+
+WideLayout wide_layout(const ScanArgs& a) {
+    const size_t bhf = (size_t)a.B * a.H * a.F;
+    WideLayout L;
+    size_t off = kWsHeaderBytes;
+    L.gimg = off;
+    if (a.mode == LA_MODE_GDN) off += bhf * 2 * kGImg;
+    L.btil = off;
+    if (a.mode == LA_MODE_GDN) off += bhf * 4 * kBTile * 16;
+    L.bmat = off;
+    if (a.mode == LA_MODE_RELU) off += bhf * 2 * kQuad * 4;
+    L.dz = off;
+    if (a.mode == LA_MODE_RELU) off += bhf * 2 * 512;
+    L.mimg = off;
+    off += bhf * 2 * kMImg;
+    L.zf = off;
+    if (a.mode == LA_MODE_RELU) off += bhf * 1024;
+    L.total = align_up(off, 256);
+    return L;
+}
+
+template <bool RELU>
+constexpr size_t smem_wide_gram() {
+    return 1024 + (RELU ? 3 : 2) * 2 * kGTile + (RELU ? 0 : kGImg) + 2048 + 256;
+}
+constexpr size_t kSmemWideChain = 1024 + 2 * kGImg + kMImg + 256;
+constexpr size_t kSmemWideOut = 1024 + 2 * kOTile + kMImg + kBoxO + 1024 + kOAcc * 512 + 256;
+static_assert(smem_wide_gram<false>() <= 232448 && smem_wide_gram<true>() <= 232448, "gram smem");
+static_assert(kSmemWideChain <= 232448, "chain smem");
+static_assert(kSmemWideOut <= 232448, "output smem");
+
+int sm_count_wide() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+template <bool RELU>
+cudaError_t launch_wide_mode(const ScanArgs& a, cudaStream_t st) {
+    const WideLayout L = wide_layout(a);
+    uint8_t* ws = reinterpret_cast<uint8_t*>(a.ws);
+    WideParams p;
+    p.alpha = a.alpha;
+    p.beta = a.beta;
+    p.state_in = a.state_in;
+    p.z_in = a.z_in;
+    p.state_out = a.state_out;
+    p.z_out = a.z_out;
+    p.status = reinterpret_cast<unsigned int*>(ws);
+    p.gimg = ws + L.gimg;
+    p.btil = reinterpret_cast<uint4*>(ws + L.btil);
+    p.bmat = reinterpret_cast<float*>(ws + L.bmat);
+    p.dz = reinterpret_cast<float*>(ws + L.dz);
+    p.mimg = ws + L.mimg;
+    p.zf = reinterpret_cast<float*>(ws + L.zf);
+    p.k_scale = a.k_scale;
+    p.eps = a.eps;
+    p.BH = a.B * a.H;
+    p.F = a.F;
+    p.S = a.S;
+    p.D = a.D;
+    p.want_output = a.o != nullptr;
+    if ((uint64_t)p.BH * p.F * 2 >= (1ull << 31)) return cudaErrorInvalidValue;
+
+    const uint64_t bhf = (uint64_t)p.BH * p.F;
+    CUtensorMap mK, mV, mQ, mO;
+    if (!make_tmap_bf16_3d(&mK, a.k, a.D, a.S, bhf, 64, kTokG) ||
+        !make_tmap_bf16_3d(&mV, a.v, a.D, a.S, bhf, 64, kTokG))
+        return cudaErrorInvalidValue;
+    if (p.want_output && (!make_tmap_bf16_3d(&mQ, a.q, a.D, a.S, bhf, 64, kTokO) ||
+                          !make_tmap_bf16_3d(&mO, a.o, a.D, a.S, bhf, 64, kTokO)))
+        return cudaErrorInvalidValue;
+
+    static bool attr_done = false;
+    if (!attr_done) {
+        cudaFuncSetAttribute(wide_gram_kernel<RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem_wide_gram<RELU>());
+        cudaFuncSetAttribute(wide_chain_gdn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemWideChain);
+        cudaFuncSetAttribute(wide_output_kernel<RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemWideOut);
+        attr_done = true;
+    }
+    const int nsm = sm_count_wide();
+    const int items = (int)(bhf * 2);
+    const int grid = std::min(items, nsm);
+    const int thr = RELU ? 320 : 192;
+    wide_gram_kernel<RELU><<<grid, thr, smem_wide_gram<RELU>(), st>>>(p, mK, mV);
+    if (RELU)
+        wide_chain_relu_kernel<<<p.BH * 8, 256, 0, st>>>(p);
+    else
+        wide_chain_gdn_kernel<<<p.BH * 2, 352, kSmemWideChain, st>>>(p);
+    if (p.want_output) wide_output_kernel<RELU><<<grid, thr, kSmemWideOut, st>>>(p, mQ, mO);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool wide_eligible(const ScanArgs& a) {
+    return a.bf16 && a.D > 128 && a.D <= 256 && a.F > 0;
+}
+
+size_t wide_workspace_bytes(const ScanArgs& a) { return wide_layout(a).total; }
+
+int wide_kernel_count(const ScanArgs& a) { return a.o ? 3 : 2; }
+
+cudaError_t launch_wide(const ScanArgs& a, cudaStream_t st) {
+    return a.mode == LA_MODE_RELU ? launch_wide_mode<true>(a, st) : launch_wide_mode<false>(a, st);
+}
+
+}  // namespace la

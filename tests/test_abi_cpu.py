@@ -32,7 +32,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_plan_reports_a_path_and_kernel_count():
     name, n = la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 20, 181, 880, 128)
-    assert name in ("tcgen05_fused", "tcgen05", "simt_f32") and n >= 1
+    assert name in ("tcgen05_fused", "tcgen05", "tcgen05_wide", "simt_f32") and n >= 1
     name, n = la.la_plan(la.LA_MODE_RELU, la.LA_F32, 1, 2, 8, 64, 32)
     assert name == "simt_f32" and n == 1
     assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 1, 1, 1, 24) == (None, 0)

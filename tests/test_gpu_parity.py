@@ -146,7 +146,7 @@ def test_streaming_chunks_equal_single_scan():
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("D,S,F", [(16, 1, 3), (48, 17, 2), (64, 130, 3), (80, 64, 2),
                                    (96, 300, 2), (112, 200, 2), (128, 129, 3), (128, 1, 4),
-                                   (256, 70, 2)])
+                                   (144, 100, 3), (192, 257, 2), (240, 1, 2), (256, 70, 2)])
 def test_small_shapes(mode, dtype, D, S, F):
     spec = synth.small(B=2, H=2, F=F, S=S, D=D, dtype=dtype, seed=D + S)
     _compare(spec, mode, with_state=True)
@@ -170,8 +170,9 @@ def test_zero_frames_copies_state(mode):
 
 
 @pytest.mark.parametrize("mode", ["relu", "gdn"])
-def test_in_place_state(mode):
-    spec = synth.small(B=1, H=2, F=3, S=40, D=64, dtype="bf16", seed=9)
+@pytest.mark.parametrize("D", [64, 192])
+def test_in_place_state(mode, D):
+    spec = synth.small(B=1, H=2, F=3, S=40, D=D, dtype="bf16", seed=9)
     inp = device_inputs(spec)
     m0n, z0n = synth.random_state(spec, 0.1)
     m, z = torch.from_numpy(m0n).cuda(), torch.from_numpy(z0n).cuda()
@@ -189,8 +190,9 @@ def test_in_place_state(mode):
 
 
 @pytest.mark.parametrize("mode", ["relu", "gdn"])
-def test_state_step_matches_oracle(mode):
-    spec = synth.small(B=2, H=2, F=4, S=100, D=128, dtype="bf16", seed=21, keys_l2=True)
+@pytest.mark.parametrize("D", [128, 256])
+def test_state_step_matches_oracle(mode, D):
+    spec = synth.small(B=2, H=2, F=4, S=100, D=D, dtype="bf16", seed=21, keys_l2=True)
     inp = device_inputs(spec)
     m0n, z0n = synth.random_state(spec, 0.05)
     m0, z0 = torch.from_numpy(m0n).cuda(), torch.from_numpy(z0n).cuda()
@@ -211,8 +213,9 @@ def test_state_step_matches_oracle(mode):
             assert rel_err(to_np(so[b, h]), rm[0, 0]) <= TOL_BF16
 
 
-def test_outputs_do_not_write_outside_their_buffers():
-    spec = synth.small(B=1, H=2, F=2, S=77, D=48, dtype="bf16", seed=5)
+@pytest.mark.parametrize("D", [48, 144])
+def test_outputs_do_not_write_outside_their_buffers(D):
+    spec = synth.small(B=1, H=2, F=2, S=77, D=D, dtype="bf16", seed=5)
     inp = device_inputs(spec)
     n = spec.B * spec.H * spec.F * spec.S * spec.D
     guard = 4096
@@ -279,12 +282,29 @@ def test_tensor_core_path_matches_simt_path(mode, monkeypatch):
     assert rel_err(to_np(m_tc), to_np(m_simt)) <= TOL_BF16
 
 
+@pytest.mark.parametrize("mode", ["relu", "gdn"])
+@pytest.mark.parametrize("D", [192, 256])
+def test_wide_tensor_core_path_matches_simt_path(mode, D, monkeypatch):
+    spec = synth.small(B=1, H=3, F=6, S=300, D=D, dtype="bf16", seed=41, keys_l2=True)
+    m = la.LA_MODE_GDN if mode == "gdn" else la.LA_MODE_RELU
+    assert la.la_plan(m, la.LA_BF16, 1, 3, 6, 300, D)[0] == "tcgen05_wide"
+    inp = device_inputs(spec)
+    o_tc, m_tc, _ = _run(spec, mode, inp)
+    monkeypatch.setenv("LA_SCAN_FORCE_SIMT", "1")
+    o_simt, m_simt, _ = _run(spec, mode, inp)
+    torch.cuda.synchronize()
+    assert rel_err(to_np(o_tc), to_np(o_simt)) <= TOL_BF16
+    assert rel_err(to_np(m_tc), to_np(m_simt)) <= TOL_BF16
+
+
 def test_plan_of_the_workloads():
     assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05_fused", 1)
     assert la.la_plan(la.LA_MODE_RELU, la.LA_BF16, 1, 20, 21, 1560, 112) == ("tcgen05_fused", 1)
     assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 4, 20, 8, 880, 128) == ("tcgen05", 3)
     assert la.la_plan(la.LA_MODE_GDN, la.LA_F32, 1, 2, 8, 64, 32)[0] == "simt_f32"
-    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 16, 512, 1024, 256)[0] == "simt_f32"
+    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 16, 512, 1024, 256) == ("tcgen05_wide", 3)
+    assert la.la_plan(la.LA_MODE_RELU, la.LA_BF16, 1, 16, 512, 1024, 256) == ("tcgen05_wide", 3)
+    assert la.la_plan(la.LA_MODE_GDN, la.LA_F32, 1, 16, 512, 1024, 256)[0] == "simt_f32"
 
 
 @pytest.mark.parametrize("mode", ["relu", "gdn"])
