@@ -36,6 +36,8 @@
 // contiguous bytes.  B~ is kept in bf16 like the state image; the state
 // itself and all accumulation stay fp32.
 #include <algorithm>
+#include <cstdlib>
+#include <mutex>
 
 #include "tc_common.cuh"
 #include "tmap.cuh"
@@ -74,9 +76,17 @@ struct WideParams {
     float* zf;              // [BHF] x 256                      (ReLU)
     float k_scale;
     float eps;
-    int BH, F, S, D;
+    int BH, F, S, D;        // F: frames of the clip (global frame index = bh F + f)
+    int f0, Fc;             // this launch covers frames [f0, f0 + Fc) of every head
     int want_output;
 };
+
+// Global frame index (into q, k, v, o, alpha, beta) of chunk-local frame
+// `loc` = bh * Fc + fl; per-frame workspace buffers are indexed by `loc`.
+__device__ __forceinline__ int global_frame(const WideParams& p, int loc) {
+    const int bh = loc / p.Fc;
+    return bh * p.F + p.f0 + (loc - bh * p.Fc);
+}
 
 // Write 16 consecutive columns [c0, c0 + 16) of row `row` of a swizzled bf16
 // image whose 64-column blocks are `blk_bytes` apart.
@@ -105,12 +115,11 @@ template <bool RELU>
 __global__ void __launch_bounds__(RELU ? 320 : 192, 1)
 wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
                  const __grid_constant__ CUtensorMap mapV) {
-    constexpr int kStages = RELU ? 3 : 2;
+    constexpr int kStages = 3;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* ring = smem;                                  // kStages x (K 32 KB | V 32 KB)
-    uint8_t* stage_img = ring + kStages * 2 * kGTile;      // G''[r] image staging (GDN)
-    uint8_t* ones = stage_img + (RELU ? 0 : kGImg);        // 2 KB of bf16 1.0 (ReLU)
+    uint8_t* ones = ring + kStages * 2 * kGTile;           // 2 KB of bf16 1.0 (ReLU)
     uint64_t* full = reinterpret_cast<uint64_t*>(ones + 2048);
     uint64_t* empty = full + kStages;
     uint64_t* xform = empty + kStages;
@@ -154,7 +163,7 @@ wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
     const Abort ab{abort_flag, p.status};
-    const int nitems = p.BH * p.F * 2;
+    const int nitems = p.BH * p.Fc * 2;
     const int nt = (p.S + kTokG - 1) / kTokG;
 
     if (warp == 0) {
@@ -166,7 +175,7 @@ wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
             uint32_t ph = 0;
             bool ok = true;
             for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x) {
-                const int frame = item >> 1;
+                const int frame = global_frame(p, item >> 1);
                 for (int t = 0; t < nt; ++t) {
                     if (!(ok = mbar_wait(&empty[s], ph ^ 1, ab, 0x601))) break;
                     uint8_t* st = ring + s * 2 * kGTile;
@@ -222,28 +231,27 @@ wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
     } else if (warp < 6) {
         // ---------------- epilogue: TMEM -> workspace ----------------
         const int q = warp & 3, row = q * 32 + lane;
-        const bool issuer = (threadIdx.x == 64);
         int li = 0;
-        bool ok = true;     // every epilogue warp runs every named barrier, even after an abort
-        for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++li) {
-            const int frame = item >> 1;
-            ok = ok && mbar_wait(accfull, li & 1, ab, 0x604);
+        bool ok = true;
+        for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
+            const int frame = global_frame(p, item >> 1);
+            if (!(ok = mbar_wait(accfull, li & 1, ab, 0x604))) break;
             tc_fence_after();
             const uint32_t tl = tbase + (uint32_t(q * 32) << 16);
             if (!RELU) {
                 const float al = p.alpha[frame], bt = p.beta[frame];
                 const float sg = -al * bt * p.k_scale * p.k_scale, sw = bt * p.k_scale;
-                if (issuer) bulk_wait_read<0>();       // staging free again
-                named_bar_sync(1, 128);
-                for (int c0 = 0; c0 < kDW && ok; c0 += 16) {
+                // the G''[r] image goes straight from registers to its workspace slot
+                uint8_t* gi = p.gimg + (size_t)item * kGImg;
+                for (int c0 = 0; c0 < kDW; c0 += 16) {
                     float v[16];
                     tmem_ld16(tl + c0, v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 16; ++e) v[e] *= sg;
-                    store_row16(stage_img, 16384, row, c0, v);
+                    store_row16(gi, 16384, row, c0, v);
                 }
-                for (int c0 = 0; c0 < kDW && ok; c0 += 16) {
+                for (int c0 = 0; c0 < kDW; c0 += 16) {
                     float v[16];
                     tmem_ld16(tl + 256 + c0, v);
                     tmem_wait_ld();
@@ -257,7 +265,7 @@ wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
                             pack_bf16x2(v[8 * h + 4] * sw, v[8 * h + 5] * sw),
                             pack_bf16x2(v[8 * h + 6] * sw, v[8 * h + 7] * sw));
                 }
-            } else if (ok) {
+            } else {
                 float* bq = p.bmat + (size_t)item * kQuad;
                 for (int c0 = 0; c0 < kDW; c0 += 16) {
                     float v[16];
@@ -276,16 +284,7 @@ wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(accempty);
-            if (!RELU) {
-                fence_proxy_async_smem();
-                named_bar_sync(1, 128);
-                if (issuer && ok) {
-                    bulk_store(p.gimg + (size_t)item * kGImg, stage_img, kGImg);
-                    bulk_commit();
-                }
-            }
         }
-        if (issuer) bulk_wait_all<0>();
     } else {
         // ---------------- ReLU transform: phi(K) in place ----------------
         const int tl = threadIdx.x - 192;          // 0..127
@@ -339,7 +338,7 @@ wide_chain_gdn_kernel(const WideParams p) {
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.x >> 1, c = blockIdx.x & 1;
-    const int F = p.F, D = p.D;
+    const int F = p.Fc, D = p.D;          // frames of this launch; buffers are chunk-local
     if (threadIdx.x == 0) {
         for (int r = 0; r < 2; ++r) {
             mbar_init(&gfull[r], 1);
@@ -405,7 +404,7 @@ wide_chain_gdn_kernel(const WideParams p) {
         const bool leader = ((threadIdx.x - 64) & 127) == 0;
         const int bar_id = 1 + r;
         const uint32_t tl = tM + (uint32_t(q * 32) << 16) + r * 128;
-        const float* ap = p.alpha + (size_t)bh * F;
+        const float* ap = p.alpha + (size_t)bh * p.F + p.f0;
         // initial state: image of M_0 and alpha_0 M_0 in TMEM
         {
             const float a0 = __ldg(ap);
@@ -518,7 +517,7 @@ __global__ void __launch_bounds__(256)
 wide_chain_relu_kernel(const WideParams p) {
     const int bh = blockIdx.x >> 3, cc = blockIdx.x & 7;
     const int i = threadIdx.x, r = i >> 7, row = i & 127;
-    const int F = p.F, D = p.D;
+    const int F = p.Fc, D = p.D;          // frames of this launch; buffers are chunk-local
     const int c = cc >> 2, jl0 = (cc & 3) * 32;        // column half and first local column
     const int j0 = 32 * cc;                           // first global column
     const bool live = i < D;
@@ -571,21 +570,22 @@ wide_chain_relu_kernel(const WideParams p) {
 // output: O_f[:, c] = Q~_f bf16(M_f)[:, c]   (ReLU: / (phi(Q_f) z_f + eps))
 // ============================================================================
 // warp 0: producer (M image and z by bulk copy, Q tiles by TMA); warp 1: TMEM
-// owner + MMA issuer; warps 2-5: epilogue (TMEM -> bf16 -> TMA store, one
-// 64-column box at a time); warps 6-9 (ReLU): phi(Q) in place and the
-// per-token denominators.
+// owner + MMA issuer; warps 2-5: epilogue (TMEM -> bf16 staging -> TMA store,
+// one 64-column box at a time, kOStg staging buffers); warps 6-9 (ReLU):
+// phi(Q) in place and the per-token denominators.
 template <bool RELU>
 __global__ void __launch_bounds__(RELU ? 320 : 192, 1)
 wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
                    const __grid_constant__ CUtensorMap mapO) {
+    constexpr int kOStg = RELU ? 1 : 2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* qring = smem;                                 // 2 x 64 KB Q tiles
     uint8_t* mbuf = qring + 2 * kOTile;                    // M[:, c] image (64 KB)
-    uint8_t* ostage = mbuf + kMImg;                        // one 64-column output box (16 KB)
-    float* zbuf = reinterpret_cast<float*>(ostage + kBoxO);           // 256
-    float* denbuf = zbuf + 256;                                       // kOAcc x 128
-    uint64_t* qfull = reinterpret_cast<uint64_t*>(denbuf + kOAcc * 128);
+    uint8_t* ostage = mbuf + kMImg;                        // kOStg x 16 KB output boxes
+    float* zbuf = reinterpret_cast<float*>(ostage + kOStg * kBoxO);   // 256 (ReLU)
+    float* denbuf = zbuf + (RELU ? 256 : 0);                          // kOAcc x 128 (ReLU)
+    uint64_t* qfull = reinterpret_cast<uint64_t*>(denbuf + (RELU ? kOAcc * 128 : 0));
     uint64_t* qempty = qfull + 2;
     uint64_t* xform = qempty + 2;
     uint64_t* mfull = xform + 2;
@@ -630,7 +630,7 @@ wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
     const Abort ab{abort_flag, p.status};
-    const int nitems = p.BH * p.F * 2;
+    const int nitems = p.BH * p.Fc * 2;
     const int nt = (p.S + kTokO - 1) / kTokO;
 
     if (warp == 0) {
@@ -642,11 +642,11 @@ wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
             uint32_t ph = 0;
             bool ok = true;
             for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
-                const int frame = item >> 1;
+                const int frame = global_frame(p, item >> 1);
                 if (!(ok = mbar_wait(mempty, (li & 1) ^ 1, ab, 0x801))) break;
                 mbar_expect_tx(mfull, kMImg + (RELU ? 1024 : 0));
                 bulk_load(mbuf, p.mimg + (size_t)item * kMImg, kMImg, mfull);
-                if (RELU) bulk_load(zbuf, p.zf + (size_t)frame * 256, 1024, mfull);
+                if (RELU) bulk_load(zbuf, p.zf + (size_t)(item >> 1) * 256, 1024, mfull);
                 for (int t = 0; t < nt; ++t) {
                     if (!(ok = mbar_wait(&qempty[s], ph ^ 1, ab, 0x802))) break;
                     uint8_t* st = qring + s * kOTile;
@@ -685,13 +685,13 @@ wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
             }
         }
     } else if (warp < 6) {
-        // ---------------- epilogue ----------------
+        // ---------------- epilogue: TMEM -> bf16 -> TMA store ----------------
         const int q = warp & 3, row = q * 32 + lane;
         const bool issuer = (threadIdx.x == 64);
-        int gt = 0;
+        int gt = 0, gb = 0;
         bool ok = true;     // every epilogue warp runs every named barrier, even after an abort
         for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
-            const int frame = item >> 1, c = item & 1;
+            const int frame = global_frame(p, item >> 1), c = item & 1;
             for (int t = 0; t < nt; ++t, ++gt) {
                 const int a = gt % kOAcc;
                 ok = ok && mbar_wait(&accfull[a], (gt / kOAcc) & 1, ab, 0x806);
@@ -699,10 +699,11 @@ wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
                 tc_fence_after();
                 const float inv = (RELU && ok) ? 1.f / denbuf[a * 128 + row] : 1.f;
                 const uint32_t tl = tbase + (uint32_t(q * 32) << 16) + a * 128;
-                for (int b = 0; b < 2; ++b) {
+                for (int b = 0; b < 2; ++b, ++gb) {
                     const int x0 = 128 * c + 64 * b;
                     if (x0 >= D) break;                       // uniform over the block
-                    if (issuer) bulk_wait_read<0>();          // staging no longer read
+                    uint8_t* os = ostage + (gb % kOStg) * kBoxO;
+                    if (issuer) bulk_wait_read<kOStg - 1>();  // this staging buffer is free
                     named_bar_sync(1, 128);
                     for (int c0 = 0; c0 < 64 && ok; c0 += 16) {
                         float v[16];
@@ -712,12 +713,12 @@ wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
 #pragma unroll
                             for (int e = 0; e < 16; ++e) v[e] *= inv;
                         }
-                        store_row16(ostage, 16384, row, c0, v);
+                        store_row16(os, 16384, row, c0, v);
                     }
                     fence_proxy_async_smem();
                     named_bar_sync(1, 128);
                     if (issuer && ok) {
-                        tma_store_3d(&mapO, ostage, x0, t * kTokO, frame);
+                        tma_store_3d(&mapO, os, x0, t * kTokO, frame);
                         bulk_commit();
                     }
                 }
@@ -780,39 +781,76 @@ wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
 // ----------------------------------------------------------------------------
 // Host side
 // ----------------------------------------------------------------------------
+// Frames per pipeline chunk: about 8 chunks, at least 4 frames (LA_WIDE_CHUNK
+// in the environment overrides it, for tuning).
+int wide_chunk(int F) {
+    const char* e = std::getenv("LA_WIDE_CHUNK");
+    int c = e ? std::atoi(e) : 0;
+    if (c <= 0) c = std::max(4, (F + 7) / 8);
+    return std::max(1, std::min(c, F));
+}
+
+// Workspace: header | state, z carried between chunks | two chunk buffer sets
+// of the gram outputs | two chunk buffer sets of the chain outputs.
 struct WideLayout {
-    size_t gimg, btil, bmat, dz, mimg, zf, total;
+    size_t state, z;
+    size_t gimg[2], btil[2], bmat[2], dz[2], mimg[2], zf[2];
+    size_t total;
+    int Fc;
 };
 
 WideLayout wide_layout(const ScanArgs& a) {
-    const size_t bhf = (size_t)a.B * a.H * a.F;
     WideLayout L;
+    const size_t bh = (size_t)a.B * a.H;
+    L.Fc = wide_chunk(a.F);
+    const size_t bhf = bh * L.Fc;
+    const bool gdn = a.mode == LA_MODE_GDN;
+    const int nsets = a.F > L.Fc ? 2 : 1;        // a second buffer set only if chunks overlap
     size_t off = kWsHeaderBytes;
-    L.gimg = off;
-    if (a.mode == LA_MODE_GDN) off += bhf * 2 * kGImg;
-    L.btil = off;
-    if (a.mode == LA_MODE_GDN) off += bhf * 4 * kBTile * 16;
-    L.bmat = off;
-    if (a.mode == LA_MODE_RELU) off += bhf * 2 * kQuad * 4;
-    L.dz = off;
-    if (a.mode == LA_MODE_RELU) off += bhf * 2 * 512;
-    L.mimg = off;
-    off += bhf * 2 * kMImg;
-    L.zf = off;
-    if (a.mode == LA_MODE_RELU) off += bhf * 1024;
-    L.total = align_up(off, 256);
+    L.state = off;
+    off = align_up(off + bh * a.D * a.D * 4, 256);
+    L.z = off;
+    off = align_up(off + bh * a.D * 4, 256);
+    for (int b = 0; b < 2; ++b) {
+        if (b == nsets) {                        // a single chunk: both names, one set
+            L.gimg[1] = L.gimg[0]; L.btil[1] = L.btil[0]; L.bmat[1] = L.bmat[0]; L.dz[1] = L.dz[0];
+            break;
+        }
+        L.gimg[b] = off;
+        if (gdn) off += bhf * 2 * kGImg;
+        L.btil[b] = off;
+        if (gdn) off += bhf * 4 * kBTile * 16;
+        L.bmat[b] = off;
+        if (!gdn) off += bhf * 2 * kQuad * 4;
+        L.dz[b] = off;
+        if (!gdn) off += bhf * 2 * 512;
+        off = align_up(off, 256);
+    }
+    for (int b = 0; b < 2; ++b) {
+        if (b == nsets) {
+            L.mimg[1] = L.mimg[0]; L.zf[1] = L.zf[0];
+            break;
+        }
+        L.mimg[b] = off;
+        off += bhf * 2 * kMImg;
+        L.zf[b] = off;
+        if (!gdn) off += bhf * 1024;
+        off = align_up(off, 256);
+    }
+    L.total = off;
     return L;
 }
 
-template <bool RELU>
-constexpr size_t smem_wide_gram() {
-    return 1024 + (RELU ? 3 : 2) * 2 * kGTile + (RELU ? 0 : kGImg) + 2048 + 256;
-}
+constexpr size_t kSmemWideGram = 1024 + 3 * 2 * kGTile + 2048 + 256;
 constexpr size_t kSmemWideChain = 1024 + 2 * kGImg + kMImg + 256;
-constexpr size_t kSmemWideOut = 1024 + 2 * kOTile + kMImg + kBoxO + 1024 + kOAcc * 512 + 256;
-static_assert(smem_wide_gram<false>() <= 232448 && smem_wide_gram<true>() <= 232448, "gram smem");
+template <bool RELU>
+constexpr size_t smem_wide_out() {
+    return 1024 + 2 * kOTile + kMImg + (RELU ? 1 : 2) * kBoxO + (RELU ? 1024 + kOAcc * 512 : 0) +
+           256;
+}
+static_assert(kSmemWideGram <= 232448, "gram smem");
 static_assert(kSmemWideChain <= 232448, "chain smem");
-static_assert(kSmemWideOut <= 232448, "output smem");
+static_assert(smem_wide_out<false>() <= 232448 && smem_wide_out<true>() <= 232448, "output smem");
 
 int sm_count_wide() {
     static int n = 0;
@@ -825,6 +863,32 @@ int sm_count_wide() {
     return n;
 }
 
+// Streams and events of one device for the chunk pipeline: the gram kernels
+// run on the caller's stream, the chain and output kernels on two streams of
+// the library's own, forked from and joined back to the caller's stream.
+constexpr int kMaxDevices = 64;
+struct WideCtx {
+    bool ready = false;
+    cudaStream_t s_chain = nullptr, s_out = nullptr;
+    cudaEvent_t start = nullptr, gram[2] = {}, chain[2] = {}, out[2] = {};
+};
+std::mutex g_wide_mu[kMaxDevices];
+WideCtx g_wide_ctx[kMaxDevices];
+
+cudaError_t wide_ctx_init(WideCtx& c) {
+    if (c.ready) return cudaSuccess;
+    cudaError_t e = cudaStreamCreateWithFlags(&c.s_chain, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c.s_out, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c.start, cudaEventDisableTiming);
+    for (int b = 0; b < 2 && e == cudaSuccess; ++b) {
+        e = cudaEventCreateWithFlags(&c.gram[b], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c.chain[b], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c.out[b], cudaEventDisableTiming);
+    }
+    if (e == cudaSuccess) c.ready = true;
+    return e;
+}
+
 template <bool RELU>
 cudaError_t launch_wide_mode(const ScanArgs& a, cudaStream_t st) {
     const WideLayout L = wide_layout(a);
@@ -832,17 +896,7 @@ cudaError_t launch_wide_mode(const ScanArgs& a, cudaStream_t st) {
     WideParams p;
     p.alpha = a.alpha;
     p.beta = a.beta;
-    p.state_in = a.state_in;
-    p.z_in = a.z_in;
-    p.state_out = a.state_out;
-    p.z_out = a.z_out;
     p.status = reinterpret_cast<unsigned int*>(ws);
-    p.gimg = ws + L.gimg;
-    p.btil = reinterpret_cast<uint4*>(ws + L.btil);
-    p.bmat = reinterpret_cast<float*>(ws + L.bmat);
-    p.dz = reinterpret_cast<float*>(ws + L.dz);
-    p.mimg = ws + L.mimg;
-    p.zf = reinterpret_cast<float*>(ws + L.zf);
     p.k_scale = a.k_scale;
     p.eps = a.eps;
     p.BH = a.B * a.H;
@@ -864,24 +918,87 @@ cudaError_t launch_wide_mode(const ScanArgs& a, cudaStream_t st) {
     static bool attr_done = false;
     if (!attr_done) {
         cudaFuncSetAttribute(wide_gram_kernel<RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem_wide_gram<RELU>());
+                             (int)kSmemWideGram);
         cudaFuncSetAttribute(wide_chain_gdn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)kSmemWideChain);
         cudaFuncSetAttribute(wide_output_kernel<RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemWideOut);
+                             (int)smem_wide_out<RELU>());
         attr_done = true;
     }
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_wide_mu[dev]);
+    WideCtx& cx = g_wide_ctx[dev];
+    cudaError_t e = wide_ctx_init(cx);
+    if (e != cudaSuccess) return e;
+
     const int nsm = sm_count_wide();
-    const int items = (int)(bhf * 2);
-    const int grid = std::min(items, nsm);
+    const int nchunks = (p.F + L.Fc - 1) / L.Fc;
+    // GDN: with more than one chunk, chain(c) (about 3.5 us per frame on its
+    // own SMs) runs beside gram(c + 1) and output(c - 1), which share the
+    // other SMs.  ReLU: the chain is a short prefix sum, so the three kernels
+    // of a chunk simply run in order on the caller's stream (measured faster
+    // than overlapping them).
+    const int chain_sms = RELU ? 0 : std::min(2 * p.BH, nsm / 2);
+    const int share = nchunks > 1 ? nsm - chain_sms : nsm;
+    cudaStream_t s_chain = RELU ? st : cx.s_chain, s_out = RELU ? st : cx.s_out;
     const int thr = RELU ? 320 : 192;
-    wide_gram_kernel<RELU><<<grid, thr, smem_wide_gram<RELU>(), st>>>(p, mK, mV);
-    if (RELU)
-        wide_chain_relu_kernel<<<p.BH * 8, 256, 0, st>>>(p);
-    else
-        wide_chain_gdn_kernel<<<p.BH * 2, 352, kSmemWideChain, st>>>(p);
-    if (p.want_output) wide_output_kernel<RELU><<<grid, thr, kSmemWideOut, st>>>(p, mQ, mO);
-    return cudaGetLastError();
+    float* st_ws = reinterpret_cast<float*>(ws + L.state);
+    float* z_ws = reinterpret_cast<float*>(ws + L.z);
+
+    auto ok = [&](cudaError_t x) {
+        if (x != cudaSuccess && e == cudaSuccess) e = x;
+        return e == cudaSuccess;
+    };
+    ok(cudaEventRecord(cx.start, st));
+    ok(cudaStreamWaitEvent(s_chain, cx.start, 0));
+    ok(cudaStreamWaitEvent(s_out, cx.start, 0));
+    int last_b = 0;
+    for (int ci = 0; ci < nchunks && e == cudaSuccess; ++ci) {
+        const int b = ci & 1;
+        const bool first = ci == 0, last = ci == nchunks - 1;
+        p.f0 = ci * L.Fc;
+        p.Fc = std::min(L.Fc, p.F - p.f0);
+        p.gimg = ws + L.gimg[b];
+        p.btil = reinterpret_cast<uint4*>(ws + L.btil[b]);
+        p.bmat = reinterpret_cast<float*>(ws + L.bmat[b]);
+        p.dz = reinterpret_cast<float*>(ws + L.dz[b]);
+        p.mimg = ws + L.mimg[b];
+        p.zf = reinterpret_cast<float*>(ws + L.zf[b]);
+        p.state_in = first ? a.state_in : st_ws;
+        p.z_in = first ? a.z_in : z_ws;
+        p.state_out = last ? a.state_out : st_ws;
+        p.z_out = last ? a.z_out : z_ws;
+        const int items = p.BH * p.Fc * 2;
+        const int grid = std::min(items, share);
+        // gram(c) overwrites the buffers chain(c - 2) read
+        if (ci >= 2) ok(cudaStreamWaitEvent(st, cx.chain[b], 0));
+        wide_gram_kernel<RELU><<<grid, thr, kSmemWideGram, st>>>(p, mK, mV);
+        ok(cudaGetLastError());
+        ok(cudaEventRecord(cx.gram[b], st));
+        // chain(c) needs gram(c), and overwrites the images output(c - 2) read
+        ok(cudaStreamWaitEvent(s_chain, cx.gram[b], 0));
+        if (ci >= 2 && p.want_output) ok(cudaStreamWaitEvent(s_chain, cx.out[b], 0));
+        if (RELU)
+            wide_chain_relu_kernel<<<p.BH * 8, 256, 0, s_chain>>>(p);
+        else
+            wide_chain_gdn_kernel<<<p.BH * 2, 352, kSmemWideChain, s_chain>>>(p);
+        ok(cudaGetLastError());
+        ok(cudaEventRecord(cx.chain[b], s_chain));
+        if (p.want_output) {
+            ok(cudaStreamWaitEvent(s_out, cx.chain[b], 0));
+            wide_output_kernel<RELU><<<grid, thr, smem_wide_out<RELU>(), s_out>>>(p, mQ, mO);
+            ok(cudaGetLastError());
+            ok(cudaEventRecord(cx.out[b], s_out));
+        }
+        last_b = b;
+    }
+    // join: the caller's stream continues after the last chain and output
+    cudaError_t j = cudaStreamWaitEvent(st, cx.chain[last_b], 0);
+    if (j == cudaSuccess && p.want_output) j = cudaStreamWaitEvent(st, cx.out[last_b], 0);
+    if (e == cudaSuccess) e = j;
+    return e;
 }
 
 }  // namespace
@@ -892,7 +1009,10 @@ bool wide_eligible(const ScanArgs& a) {
 
 size_t wide_workspace_bytes(const ScanArgs& a) { return wide_layout(a).total; }
 
-int wide_kernel_count(const ScanArgs& a) { return a.o ? 3 : 2; }
+int wide_kernel_count(const ScanArgs& a) {
+    const int n = (a.F + wide_chunk(a.F) - 1) / wide_chunk(a.F);
+    return (a.o ? 3 : 2) * n;
+}
 
 cudaError_t launch_wide(const ScanArgs& a, cudaStream_t st) {
     return a.mode == LA_MODE_RELU ? launch_wide_mode<true>(a, st) : launch_wide_mode<false>(a, st);

@@ -297,13 +297,37 @@ def test_wide_tensor_core_path_matches_simt_path(mode, D, monkeypatch):
     assert rel_err(to_np(m_tc), to_np(m_simt)) <= TOL_BF16
 
 
+@pytest.mark.parametrize("mode", ["relu", "gdn"])
+def test_wide_path_chunking_is_exact(mode, monkeypatch):
+    """The wide path pipelines frame chunks and carries the fp32 state between
+    them, so the chunk length changes nothing: every chunking gives the same
+    bits, and matches the oracle (ragged last chunk, initial state)."""
+    spec = synth.small(B=1, H=2, F=21, S=64, D=256, dtype="bf16", seed=43, keys_l2=True)
+    inp = device_inputs(spec)
+    m0n, z0n = synth.random_state(spec, 0.05)
+    m0, z0 = torch.from_numpy(m0n).cuda(), torch.from_numpy(z0n).cuda()
+    runs = []
+    for chunk in ("1", "5", "21"):
+        monkeypatch.setenv("LA_WIDE_CHUNK", chunk)
+        runs.append(_run(spec, mode, inp, m0, z0 if mode == "relu" else None))
+    torch.cuda.synchronize()
+    for o, so, zo in runs[1:]:
+        assert torch.equal(o.view(torch.int16), runs[0][0].view(torch.int16))
+        assert torch.equal(so, runs[0][1])
+        if mode == "relu":
+            assert torch.equal(zo, runs[0][2])
+    monkeypatch.delenv("LA_WIDE_CHUNK")
+    _compare(spec, mode, with_state=True)
+
+
 def test_plan_of_the_workloads():
     assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05_fused", 1)
     assert la.la_plan(la.LA_MODE_RELU, la.LA_BF16, 1, 20, 21, 1560, 112) == ("tcgen05_fused", 1)
     assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 4, 20, 8, 880, 128) == ("tcgen05", 3)
     assert la.la_plan(la.LA_MODE_GDN, la.LA_F32, 1, 2, 8, 64, 32)[0] == "simt_f32"
-    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 16, 512, 1024, 256) == ("tcgen05_wide", 3)
-    assert la.la_plan(la.LA_MODE_RELU, la.LA_BF16, 1, 16, 512, 1024, 256) == ("tcgen05_wide", 3)
+    # 8 pipeline chunks of 64 frames, three kernels each
+    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 16, 512, 1024, 256) == ("tcgen05_wide", 24)
+    assert la.la_plan(la.LA_MODE_RELU, la.LA_BF16, 1, 16, 512, 1024, 256) == ("tcgen05_wide", 24)
     assert la.la_plan(la.LA_MODE_GDN, la.LA_F32, 1, 16, 512, 1024, 256)[0] == "simt_f32"
 
 
