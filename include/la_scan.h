@@ -39,6 +39,13 @@
  *              LA_ERR_CUDA.  Device-side waits are bounded: a wait that
  *              gives up records LA_ERR_TIMEOUT in the workspace, which
  *              la_query_device_status reports.
+ * Streams.     Wide heads (bf16, D > 128) pipeline frame chunks over two
+ *              streams of the library's own, forked from `stream` (after the
+ *              work already queued on it) and joined back to it, so the call
+ *              is still ordered on `stream` as a whole.  The first such call
+ *              on a device creates those streams and a few events and keeps
+ *              them until the process exits; calls on one device serialise
+ *              their enqueueing on a lock.
  * Aliasing.    state_in == state_out (and z_in == z_out) is allowed (in
  *              place).  o must not overlap q, k or v.
  * NULL state.  state_in == NULL (z_in == NULL) means a zero initial state;
@@ -155,7 +162,9 @@ LA_API la_status la_state_step(la_mode mode, const void* k, const void* v, la_dt
  *   whose la_workspace_size(LA_MODE_GDN, B, H, F, S, D) exceeds it returns
  *   LA_ERR_UNSUPPORTED before enqueuing anything (for bf16 inputs with
  *   64 <= D <= 128 the scan needs about 1 MiB per (b, h) pair, so up to
- *   B*H = 63; D > 128 and float32 inputs need only a few bytes).
+ *   B*H = 63; float32 inputs and D < 64 need only a few bytes; bf16 inputs
+ *   with D > 128 need per-frame buffers of about 0.4 MiB per (b, h, frame)
+ *   of a pipeline chunk, so only short clips of few heads fit).
  * Sharing.  All calls on a device share the one array, and it keeps the
  *   last call's contents; the library clears what must start at zero at the
  *   start of every call.  Calls whose GPU work overlaps (on different
@@ -241,7 +250,10 @@ LA_API la_status la_query_device_status(void* workspace, cudaStream_t stream);
 
 /* How a call of this mode, dtype and shape runs: stores the number of
  * kernels one call launches in *kernels (if not NULL) and returns the name
- * of the kernel path ("tcgen05" or "simt_f32"); NULL for an unsupported
+ * of the kernel path: "tcgen05_fused" (bf16, 64 <= D <= 128, few heads: one
+ * persistent kernel), "tcgen05" (bf16, 64 <= D <= 128, many heads: three
+ * kernels), "tcgen05_wide" (bf16, 128 < D <= 256: three kernels per frame
+ * chunk) or "simt_f32" (float32 inputs, D < 64); NULL for an unsupported
  * shape.  No counterpart in the pages: it lets a caller check which
  * kernels its calls use. */
 LA_API const char* la_plan(la_mode mode, la_dtype dt, int B, int H, int F, int S, int D,
