@@ -40,6 +40,17 @@ so a frame interval has a transition composite and an input composite, and
 an exclusive prefix over intervals recovers each interval's exact initial
 state.
 
+Reversed GDN scan -- SANA-WM paper summary, section 3, "Chunk-causal
+deployment": a reversed GDN scan that is reset at every chunk boundary gives
+each frame the later frames of its own chunk as context without leaking
+across chunks.  Reading (the pages give no formula): frames are split into
+chunks [c C, min((c + 1) C, F)); inside a chunk the GDN recurrence above
+runs from the chunk's last frame back to its first, from a zero state, and
+frame f reads the state after its own update:
+    M_{e+1} = 0 (e = last frame of the chunk)
+    M_f = alpha_f (I - beta_f Kh_f^T Kh_f) M_{f+1} + beta_f Kh_f^T V_f
+    O_f = Q_f M_f
+
 Array layout: q, k, v, o are [B, H, F, S, D]; alpha, beta are [B, H, F];
 state is [B, H, D, D] (key-major); z is [B, H, D].  Every input is widened
 to float64 first (bf16 and fp32 widen exactly).
@@ -52,7 +63,7 @@ import numpy as np
 
 __all__ = [
     "relu_scan", "gdn_scan", "relu_state_step", "gdn_state_step",
-    "gdn_interval_composite", "compose_exclusive_prefix",
+    "gdn_interval_composite", "compose_exclusive_prefix", "gdn_scan_reverse_chunked",
 ]
 
 
@@ -151,6 +162,39 @@ def gdn_scan(q, k, v, alpha, beta, k_scale: float, state_in=None,
                     o[b, h, f] = q[b, h, f] @ M       # reads the updated state
             m_out[b, h] = M
     return o, m_out
+
+
+def gdn_scan_reverse_chunked(q, k, v, alpha, beta, k_scale: float, chunk_frames: int):
+    """Reversed frame-wise GDN, reset at every chunk boundary.
+
+    SANA-WM paper summary, section 3, "Chunk-causal deployment".  For each
+    chunk of chunk_frames frames (the last one may be shorter) the state
+    starts at zero after the chunk's last frame and the frames are taken
+    from last to first, each in the direct order of gdn_scan:
+        P = Kh M;  M <- alpha (M - beta Kh^T P) + beta Kh^T V;  O = Q M.
+    No state enters or leaves.  Returns o, [B, H, F, S, D].
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    alpha, beta = _f64(alpha), _f64(beta)
+    B, H, F, S, D = _shape(k)
+    C = int(chunk_frames)
+    if C < 1:
+        raise ValueError("chunk_frames must be >= 1")
+    o = np.zeros((B, H, F, S, D))
+    kappa = float(k_scale)
+    for b in range(B):
+        for h in range(H):
+            for start in range(0, F, C):
+                end = min(start + C, F)               # frames start .. end-1
+                M = np.zeros((D, D))                  # reset at the chunk boundary
+                for f in range(end - 1, start - 1, -1):
+                    a = alpha[b, h, f]
+                    bt = beta[b, h, f]
+                    kh = kappa * k[b, h, f]
+                    P = kh @ M
+                    M = a * (M - bt * (kh.T @ P)) + bt * (kh.T @ v[b, h, f])
+                    o[b, h, f] = q[b, h, f] @ M
+    return o
 
 
 def gdn_state_step(k, v, alpha, beta, k_scale: float, state_in=None):

@@ -434,3 +434,111 @@ def _gdn_pins_pass(scan):
 def test_pins_reject_planted_mistakes(kind):
     assert _gdn_pins_pass(lambda *a: oracle.gdn_scan(*a)[0])
     assert not _gdn_pins_pass(_gdn_mutant(kind))
+
+
+# ----------------------------------------------------------------------------
+# Reversed GDN scan, reset at chunk boundaries
+# ----------------------------------------------------------------------------
+def _gdn_reverse_unrolled(q, k, v, alpha, beta, kappa, C):
+    """O_f = Q_f sum_{j = f .. e} A_f A_{f+1} .. A_{j-1} B_j within each chunk
+    (e = the chunk's last frame), assembled as an explicit block
+    upper-triangular (F*S) x (F*S) matrix per head."""
+    B, H, F, S, D = k.shape
+    out = np.zeros_like(q)
+    I = np.eye(D)
+    for b in range(B):
+        for h in range(H):
+            A = [alpha[b, h, f] * (I - beta[b, h, f] * (kappa * k[b, h, f]).T @ (kappa * k[b, h, f]))
+                 for f in range(F)]
+            L = np.zeros((F * S, F * S))
+            for f in range(F):
+                e = min((f // C + 1) * C, F) - 1
+                phi = I.copy()                    # A_f ... A_{j-1}
+                for j in range(f, e + 1):
+                    L[f * S:(f + 1) * S, j * S:(j + 1) * S] = \
+                        q[b, h, f] @ phi @ (beta[b, h, j] * (kappa * k[b, h, j]).T)
+                    phi = phi @ A[j]
+            out[b, h] = (L @ v[b, h].reshape(F * S, D)).reshape(F, S, D)
+    return out
+
+
+def _rev_inputs():
+    spec = synth.small(B=1, H=2, F=7, S=6, D=5, dtype="f32", seed=17)
+    return spec, _inputs(spec)
+
+
+@pytest.mark.parametrize("C", [1, 2, 3, 7, 10])
+def test_reverse_matches_unrolled_product(C):
+    spec, (q, k, v, a, bt) = _rev_inputs()
+    o = oracle.gdn_scan_reverse_chunked(q, k, v, a, bt, 0.35, C)
+    assert _rel(o, _gdn_reverse_unrolled(q, k, v, a, bt, 0.35, C)) < 1e-12
+
+
+def test_reverse_one_frame_chunks_are_single_writes():
+    spec, (q, k, v, a, bt) = _rev_inputs()
+    o = oracle.gdn_scan_reverse_chunked(q, k, v, a, bt, 0.35, 1)
+    for f in range(spec.F):
+        kh = 0.35 * k[0, 1, f]
+        np.testing.assert_allclose(o[0, 1, f], q[0, 1, f] @ (bt[0, 1, f] * kh.T @ v[0, 1, f]),
+                                   rtol=1e-12, atol=1e-12)
+
+
+def test_reverse_does_not_leak_across_chunks():
+    spec, (q, k, v, a, bt) = _rev_inputs()
+    C = 3                                  # chunks {0,1,2} {3,4,5} {6}
+    o = oracle.gdn_scan_reverse_chunked(q, k, v, a, bt, 0.35, C)
+    for f_pert, inside in ((1, range(0, 3)), (4, range(3, 6)), (6, range(6, 7))):
+        k2, v2, q2 = k.copy(), v.copy(), q.copy()
+        k2[:, :, f_pert] += 0.7
+        v2[:, :, f_pert] -= 1.3
+        q2[:, :, f_pert] *= 2.0
+        o2 = oracle.gdn_scan_reverse_chunked(q2, k2, v2, a, bt, 0.35, C)
+        outside = [f for f in range(spec.F) if f not in inside]
+        np.testing.assert_array_equal(o[:, :, outside], o2[:, :, outside])
+        # within the chunk: frames up to the perturbed one see it, later ones do not
+        later = [f for f in inside if f > f_pert]
+        np.testing.assert_array_equal(o[:, :, later], o2[:, :, later])
+        for f in inside:
+            if f <= f_pert:
+                assert np.max(np.abs(o[:, :, f] - o2[:, :, f])) > 1e-6
+
+
+def test_reverse_of_whole_clip_is_forward_scan_of_reversed_frames():
+    spec, (q, k, v, a, bt) = _rev_inputs()
+    o = oracle.gdn_scan_reverse_chunked(q, k, v, a, bt, 0.35, spec.F)
+    rev = lambda x: x[:, :, ::-1].copy()
+    of, _ = oracle.gdn_scan(rev(q), rev(k), rev(v), rev(a), rev(bt), 0.35)
+    assert _rel(o, rev(of)) < 1e-12
+
+
+def _reverse_mutant(kind):
+    def scan(q, k, v, alpha, beta, kappa, C):
+        B, H, F, S, D = k.shape
+        o = np.zeros_like(q, dtype=float)
+        for b in range(B):
+            for h in range(H):
+                M = np.zeros((D, D))
+                for start in range(0, F, C):
+                    end = min(start + C, F)
+                    if kind != "no_reset":
+                        M = np.zeros((D, D))
+                    frames = range(start, end) if kind == "forward_in_chunk" else \
+                        range(end - 1, start - 1, -1)
+                    for f in frames:
+                        a, bt = alpha[b, h, f], beta[b, h, f]
+                        kh = kappa * k[b, h, f]
+                        if kind == "exclusive":
+                            o[b, h, f] = q[b, h, f] @ M
+                        M = a * (M - bt * kh.T @ (kh @ M)) + bt * kh.T @ v[b, h, f]
+                        if kind != "exclusive":
+                            o[b, h, f] = q[b, h, f] @ M
+        return o
+    return scan
+
+
+@pytest.mark.parametrize("kind", ["no_reset", "forward_in_chunk", "exclusive"])
+def test_reverse_pins_reject_planted_mistakes(kind):
+    spec, (q, k, v, a, bt) = _rev_inputs()
+    ref = _gdn_reverse_unrolled(q, k, v, a, bt, 0.35, 3)
+    assert _rel(oracle.gdn_scan_reverse_chunked(q, k, v, a, bt, 0.35, 3), ref) < 1e-12
+    assert _rel(_reverse_mutant(kind)(q, k, v, a, bt, 0.35, 3), ref) > 1e-3
