@@ -48,6 +48,8 @@ WORKLOADS = {
     "stream_gdn": (3, "gdn"),
     "stress_gdn": (4, "gdn"),
     "stress_relu": (4, "relu"),
+    # reversed GDN scan reset every 8 frames, on the 720p 60 s clip
+    "gdn_720p_60s_reverse8": (2, "gdn_reverse"),
     "tiny_gdn": (0, "gdn"),
     "tiny_relu": (0, "relu"),
 }
@@ -59,9 +61,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # ----------------------------------------------------------------------------
 # Algorithmic counts (fixed formulas, whatever the kernels do)
 # ----------------------------------------------------------------------------
+REVERSE_CHUNK = 8      # frames per chunk of the reversed-scan workload
+
+
 def frame_flops(mode: str, S: int, D: int) -> int:
     """ReLU: phi(K)^T V and phi(Q) M (2SD^2 each), z and phi(Q) z (2SD each).
-    GDN: Kh^T Kh, Kh^T V, Q M (2SD^2 each) and G M (2D^3)."""
+    GDN (either direction): Kh^T Kh, Kh^T V, Q M (2SD^2 each) and G M (2D^3)."""
     if mode == "relu":
         return 4 * S * D * D + 4 * S * D
     return 6 * S * D * D + 2 * D ** 3
@@ -70,9 +75,10 @@ def frame_flops(mode: str, S: int, D: int) -> int:
 def call_bytes(mode: str, B: int, H: int, F: int, S: int, D: int, elem: int,
                state_in: bool) -> int:
     """q, k, v read once and o written once; alpha, beta read once (GDN);
-    the state (and z) written once per (b, h) and read once if given."""
-    per_frame = 4 * S * D * elem + (8 if mode == "gdn" else 0)
-    per_bh = D * D * 4 * (2 if state_in else 1)
+    the state (and z) written once per (b, h) and read once if given (the
+    reversed scan has no state in or out)."""
+    per_frame = 4 * S * D * elem + (8 if mode != "relu" else 0)
+    per_bh = D * D * 4 * (2 if state_in else 1) if mode != "gdn_reverse" else 0
     if mode == "relu":
         per_bh += D * 4 * (2 if state_in else 1)
     return B * H * (F * per_frame + per_bh)
@@ -233,6 +239,8 @@ def time_oracle_sample(spec, mode, budget_s: float, max_heads=None):
         t0 = time.perf_counter()
         if mode == "relu":
             oracle.relu_scan(q, k, v, spec.eps)
+        elif mode == "gdn_reverse":
+            oracle.gdn_scan_reverse_chunked(q, k, v, a, bt, spec.k_scale, REVERSE_CHUNK)
         else:
             oracle.gdn_scan(q, k, v, a, bt, spec.k_scale)
         t_total += time.perf_counter() - t0
@@ -327,7 +335,9 @@ def run_ours(args):
     state = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
     z = torch.empty((B, H, D), dtype=torch.float32, device=dev)
     plan = step_plan(spec, mode)
-    ws = la.workspace_for(la.LA_MODE_GDN if mode == "gdn" else la.LA_MODE_RELU,
+    mode_c = {"gdn": la.LA_MODE_GDN, "relu": la.LA_MODE_RELU,
+              "gdn_reverse": la.LA_MODE_GDN_REVERSE}[mode]
+    ws = la.workspace_for(mode_c,
                           B, H, max(n for _, n, _ in plan), S, D, dev)
     views = []
     for f0, n, si in plan:
@@ -343,7 +353,10 @@ def run_ours(args):
 
     def one_step():
         for (q, k, v, al, be, oo, si) in views:
-            if mode == "gdn":
+            if mode == "gdn_reverse":
+                la.la_scan_gdn_reverse(q, k, v, al, be, spec.k_scale, REVERSE_CHUNK, o=oo,
+                                       workspace=ws, stream=stream)
+            elif mode == "gdn":
                 la.la_scan_gdn(q, k, v, al, be, spec.k_scale, o=oo,
                                state_in=state if si else None, state_out=state,
                                workspace=ws, stream=stream)
@@ -352,7 +365,7 @@ def run_ours(args):
                                 z_in=z if si else None, state_out=state, z_out=z,
                                 eps=spec.eps, workspace=ws, stream=stream)
 
-    path, kernels_per_call = la.la_plan(la.LA_MODE_GDN if mode == "gdn" else la.LA_MODE_RELU,
+    path, kernels_per_call = la.la_plan(mode_c,
                                         dtc, B, H, plan[0][1], S, D)
 
     def barrier():
@@ -396,23 +409,40 @@ def run_ours(args):
     # scan and D2H of the output and final state all inside the timed region,
     # pipelined chunk by chunk over the library's copy streams ----
     Ke = max(3, min(K, 10))
-    mode_c = la.LA_MODE_GDN if mode == "gdn" else la.LA_MODE_RELU
     chunk = spec.chunk_frames or 0
     o_host = torch.empty_like(host["q"], pin_memory=True)
     so_host = torch.empty((B, H, D, D), dtype=torch.float32, pin_memory=True)
     zo_host = torch.empty((B, H, D), dtype=torch.float32, pin_memory=True) \
         if mode == "relu" else None
-    ins = ("q", "k", "v", "alpha", "beta") if mode == "gdn" else ("q", "k", "v")
+    ins = ("q", "k", "v") if mode == "relu" else ("q", "k", "v", "alpha", "beta")
+    if mode == "gdn_reverse":
+        so_host = None          # the reversed scan has no state out
     h2d = sum(host[x].numel() * host[x].element_size() for x in ins)
     d2h = sum(t.numel() * t.element_size() for t in (o_host, so_host, zo_host) if t is not None)
-    hws = None if args.no_e2e else la.host_workspace_for(mode_c, dtc, B, H, F, S, D, chunk, dev)
+    e2e_call = "la_scan_host"
+    if mode == "gdn_reverse":
+        # no host-buffer form of the reversed scan: H2D, the call and D2H in
+        # order on one stream
+        e2e_call = "H2D + la_scan_gdn_reverse + D2H"
+        hws = None
 
-    def e2e_step():
-        la.la_scan_host(mode_c, host["q"], host["k"], host["v"], o=o_host,
-                        alpha=host["alpha"] if mode == "gdn" else None,
-                        beta=host["beta"] if mode == "gdn" else None,
-                        k_scale=spec.k_scale, eps=spec.eps, state_out=so_host, z_out=zo_host,
-                        chunk_frames=chunk, workspace=hws, stream=stream)
+        def e2e_step():
+            for x in ins:
+                dev_in[x].copy_(host[x], non_blocking=True)
+            la.la_scan_gdn_reverse(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"],
+                                   dev_in["beta"], spec.k_scale, REVERSE_CHUNK, o=o,
+                                   workspace=ws, stream=stream)
+            o_host.copy_(o, non_blocking=True)
+    else:
+        hws = None if args.no_e2e else la.host_workspace_for(mode_c, dtc, B, H, F, S, D, chunk,
+                                                             dev)
+
+        def e2e_step():
+            la.la_scan_host(mode_c, host["q"], host["k"], host["v"], o=o_host,
+                            alpha=host["alpha"] if mode == "gdn" else None,
+                            beta=host["beta"] if mode == "gdn" else None,
+                            k_scale=spec.k_scale, eps=spec.eps, state_out=so_host, z_out=zo_host,
+                            chunk_frames=chunk, workspace=hws, stream=stream)
 
     e2e_value = None
     if not args.no_e2e:
@@ -462,7 +492,9 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if spec.dtype == "bf16" else "f32",
         "data": "synthetic (seeded numpy PCG64, bf16 round-to-nearest-even)",
-        "config": {"workload": base.name, "mode": mode, "B": B, "H": H, "F": F, "S": S, "D": D,
+        "config": {"workload": base.name + (f"_reverse{REVERSE_CHUNK}" if mode == "gdn_reverse"
+                                            else ""),
+                   "mode": mode, "B": B, "H": H, "F": F, "S": S, "D": D,
                    "calls_per_step": len(plan), "global_batch": B * world,
                    "l2": "inputs larger than L2 (no flush)",
                    "parallelism": f"replicas x{world} (no data-path collective)"},
@@ -472,8 +504,9 @@ def run_ours(args):
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "latent frames/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": Ke, "call": "la_scan_host",
-                "chunk_frames": la.la_host_chunk_frames(F, chunk),
+                "d2h_bytes_per_step": d2h, "steps": Ke, "call": e2e_call,
+                "chunk_frames": (la.la_host_chunk_frames(F, chunk) if mode != "gdn_reverse"
+                                 else None),
                 "host_memory": "pinned"},
         "clocks": clocks.summary(),
         "device_status": la.la_status_string(status),

@@ -83,7 +83,11 @@ typedef enum la_status {
 } la_status;
 
 typedef enum la_dtype { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
-typedef enum la_mode { LA_MODE_RELU = 0, LA_MODE_GDN = 1 } la_mode;
+typedef enum la_mode {
+    LA_MODE_RELU = 0,
+    LA_MODE_GDN = 1,
+    LA_MODE_GDN_REVERSE = 2      /* la_scan_gdn_reverse (for la_workspace_size, la_plan) */
+} la_mode;
 
 /*
  * Block-causal ReLU linear attention with normaliser over latent frames.
@@ -123,6 +127,32 @@ LA_API la_status la_scan_gdn(const void* q, const void* k, const void* v, void* 
                       const float* state_in, float* state_out,
                       int B, int H, int F, int S, int D,
                       void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Reversed frame-wise GDN, reset at every chunk boundary.
+ * Source: SANA-WM paper summary (paperlayer), section 3, "Chunk-causal
+ * deployment" -- a reversed GDN scan that restarts at each chunk boundary
+ * gives every frame the later frames of its own chunk as context without
+ * leaking information across chunks.  Reading (the page gives no formula):
+ * frames are split into chunks [c C, min((c+1) C, F)), C = chunk_frames;
+ * inside a chunk the recurrence of la_scan_gdn runs from the chunk's last
+ * frame back to its first, from a zero state:
+ *   M_{e+1} = 0 (e = last frame of the chunk)
+ *   M_f = alpha_f (I - beta_f Kh_f^T Kh_f) M_{f+1} + beta_f Kh_f^T V_f
+ *   O_f = Q_f M_f
+ *
+ * Arguments and layouts are those of la_scan_gdn, without state in or out;
+ * chunk_frames >= 1 (chunk_frames >= F reverses the whole clip).  The
+ * workspace is la_workspace_size(LA_MODE_GDN_REVERSE, B, H, F, S, D) bytes.
+ * bf16 inputs with 64 <= D <= 128 run on the tensor-core path; other
+ * shapes on the float32 SIMT kernel.
+ */
+LA_API la_status la_scan_gdn_reverse(const void* q, const void* k, const void* v, void* o,
+                                     la_dtype dt, const float* alpha, const float* beta,
+                                     float k_scale, int chunk_frames,
+                                     int B, int H, int F, int S, int D,
+                                     void* workspace, size_t workspace_bytes,
+                                     cudaStream_t stream);
 
 /*
  * Advance the cached state over finished frames without producing outputs:

@@ -20,7 +20,8 @@ import torch
 
 __all__ = [
     "LA_OK", "LA_ERR_INVALID_ARG", "LA_ERR_UNSUPPORTED", "LA_ERR_CUDA", "LA_ERR_TIMEOUT",
-    "LA_F32", "LA_BF16", "LA_MODE_RELU", "LA_MODE_GDN", "LaScanError", "lib", "LIB_PATH",
+    "LA_F32", "LA_BF16", "LA_MODE_RELU", "LA_MODE_GDN", "LA_MODE_GDN_REVERSE", "LaScanError",
+    "lib", "LIB_PATH", "la_scan_gdn_reverse",
     "la_scan_relu", "la_scan_gdn", "la_state_step", "la_workspace_size",
     "la_query_device_status", "la_status_string", "la_plan", "workspace_for",
     "la_scan_gdn_noalloc", "LA_NOALLOC_SCRATCH_BYTES", "la_scan_host",
@@ -29,7 +30,7 @@ __all__ = [
 
 LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CUDA, LA_ERR_TIMEOUT = 0, 1, 2, 3, 4
 LA_F32, LA_BF16 = 0, 1
-LA_MODE_RELU, LA_MODE_GDN = 0, 1
+LA_MODE_RELU, LA_MODE_GDN, LA_MODE_GDN_REVERSE = 0, 1, 2
 LA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblavf.so")
@@ -58,6 +59,8 @@ def _load() -> ctypes.CDLL:
     L.la_workspace_size.restype = Z
     L.la_query_device_status.argtypes = [P, P]
     L.la_query_device_status.restype = I
+    L.la_scan_gdn_reverse.argtypes = [P, P, P, P, I, P, P, F, I, I, I, I, I, I, P, Z, P]
+    L.la_scan_gdn_reverse.restype = I
     L.la_scan_gdn_noalloc.argtypes = [P, P, P, P, I, P, P, F, P, P, I, I, I, I, I, P]
     L.la_scan_gdn_noalloc.restype = I
     L.la_plan.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(ctypes.c_int)]
@@ -173,6 +176,26 @@ def la_scan_gdn(q, k, v, alpha, beta, k_scale: float, o=None, state_in=None, sta
                          _ptr(beta), float(k_scale), _ptr(state_in), _ptr(state_out),
                          B, H, F, S, D, _ptr(workspace), workspace.numel(), _stream(stream))
     _raise(st, "la_scan_gdn")
+    return o
+
+
+def la_scan_gdn_reverse(q, k, v, alpha, beta, k_scale: float, chunk_frames: int, o=None,
+                        workspace=None, stream=None):
+    """Reversed frame-wise GDN, reset every chunk_frames frames (no state in
+    or out; see include/la_scan.h)."""
+    B, H, F, S, D = k.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _check(t, n, (B, H, F, S, D), k.dtype)
+    for t, n in ((alpha, "alpha"), (beta, "beta")):
+        _check(t, n, (B, H, F), torch.float32)
+    if o is None:
+        o = torch.empty_like(q)
+    if workspace is None:
+        workspace = workspace_for(LA_MODE_GDN_REVERSE, B, H, F, S, D, q.device)
+    st = lib.la_scan_gdn_reverse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _dtype_code(k), _ptr(alpha),
+                                 _ptr(beta), float(k_scale), int(chunk_frames), B, H, F, S, D,
+                                 _ptr(workspace), workspace.numel(), _stream(stream))
+    _raise(st, "la_scan_gdn_reverse")
     return o
 
 

@@ -41,9 +41,22 @@ struct ScanArgs {
     int B, H, F, S, D;
     int mode;                // LA_MODE_RELU / LA_MODE_GDN
     int bf16;                // 1 if q,k,v,o are bf16
+    int rev_chunk;           // > 0: reversed GDN scan reset every rev_chunk frames
     void* ws;
     size_t ws_bytes;
 };
+
+// Frame processed at step s of a scan over F frames: s itself for the
+// forward scan (C == 0); for the reversed scan reset at chunk boundaries
+// (C > 0), chunk [c C, min((c + 1) C, F)) is taken from its last frame back
+// to its first.  A step starts a new chunk (zero state) when s % C == 0.
+__host__ __device__ inline int step_frame(int s, int F, int C) {
+    if (C <= 0) return s;
+    const int c0 = (s / C) * C;
+    const int end = c0 + C < F ? c0 + C : F;
+    return end - 1 - (s - c0);
+}
+__host__ __device__ inline bool step_resets(int s, int C) { return C > 0 && s % C == 0; }
 
 // Element access for the two storage types.
 __device__ __forceinline__ float load_elem(const void* p, size_t i, int bf16) {

@@ -12,7 +12,9 @@
 //     M_f = alpha M_{f-1} + beta Kh^T (V - alpha Kh M_{f-1})
 // which needs only the block's own columns of M, V and O.
 // ReLU mode accumulates the additive block state and normaliser of the
-// SANA-Video block KV cache (talk, block KV cache segment).
+// SANA-Video block KV cache (talk, block KV cache segment).  With
+// rev_chunk > 0 the GDN frames are taken in the reversed, chunk-reset order
+// of the SANA-WM paper summary (section 3, "Chunk-causal deployment").
 #include "common.cuh"
 
 namespace la {
@@ -71,7 +73,13 @@ simt_scan_kernel(ScanArgs a) {
     __syncthreads();
 
     const int nacc = D / kRowsPerPass;      // <= 32 accumulators (D <= 256)
-    for (int f = 0; f < F; ++f) {
+    for (int st = 0; st < F; ++st) {
+        const int f = step_frame(st, F, a.rev_chunk);
+        if (step_resets(st, a.rev_chunk)) {            // a new chunk of the reversed scan
+            __syncthreads();
+            for (int i = tid; i < D * kDJ; i += kThreads) sM[i] = 0.f;
+            __syncthreads();
+        }
         const size_t frame = (bh * F + f) * (size_t)S;   // first token row of the frame
         float al = 1.f, bt = 1.f;
         if (!relu) { al = a.alpha[bh * F + f]; bt = a.beta[bh * F + f]; }

@@ -57,6 +57,9 @@ using namespace tc;
 #ifndef LA_FUSED_WSTAGES
 #define LA_FUSED_WSTAGES 4
 #endif
+#ifndef LA_FUSED_WSTG
+#define LA_FUSED_WSTG 2
+#endif
 #ifndef LA_FUSED_EARLY_Q
 #define LA_FUSED_EARLY_Q 1
 #endif
@@ -83,6 +86,7 @@ using namespace tc;
 constexpr int kRG = 16;                 // per-head ring slots: gram -> chain
 constexpr int kRM = 16;                 // per-head ring slots: chain -> output
 constexpr int kWStages = LA_FUSED_WSTAGES;   // worker TMA ring (32 KB stages)
+constexpr int kWStg = LA_FUSED_WSTG;         // worker epilogue staging buffers (16 KB)
 constexpr int kCStages = 2;             // chain operand ring depth
 constexpr int kIQ = 4;                  // worker item queue depth
 constexpr int kThreads = 384;           // 12 warps
@@ -175,8 +179,8 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                                             const CUtensorMap* mQ, const CUtensorMap* mO) {
     uint8_t* ring = smem;                                  // kWStages x 32 KB
     uint8_t* mbuf = ring + kWStages * 32768;               // M image of the current output item
-    uint8_t* stg = mbuf + kImg;                            // 2 x 16 KB epilogue staging
-    uint8_t* ones = stg + 2 * 16384;                       // 2 KB bf16 1.0 (ReLU)
+    uint8_t* stg = mbuf + kImg;                            // kWStg x 16 KB epilogue staging
+    uint8_t* ones = stg + kWStg * 16384;                   // 2 KB bf16 1.0 (ReLU)
     float* zbuf = reinterpret_cast<float*>(ones + 2048);   // 128 (ReLU)
     float* denbuf = zbuf + 128;                            // 4 x 128 (ReLU)
     float* dzst = denbuf + 4 * 128;                        // 128: dz_f staging (ReLU)
@@ -438,9 +442,9 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                     const float sc = im == 0 ? sg : sw;
                     uint8_t* dst = (im == 0 ? p.gimg : p.bimg) + sidx * kImg;
                     for (int blk = 0; blk < nblk; ++blk) {
-                        if (leader) bulk_wait_read<1>();
+                        if (leader) bulk_wait_read<kWStg - 1>();
                         named_bar_sync(1, 128);
-                        uint8_t* sb = stg + (sctr & 1) * 16384;
+                        uint8_t* sb = stg + (sctr % kWStg) * 16384;
                         ++sctr;
                         if (go)
                             for (int c0 = blk * 64; c0 < min(D, blk * 64 + 64); c0 += 16) {
@@ -502,9 +506,9 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                     const float inv = (RELU && go) ? 1.f / denbuf[qa * 128 + row] : 1.f;
                     // one 64-column block (16 KB) at a time through staging
                     for (int blk = 0; blk < nblk; ++blk) {
-                        if (leader) bulk_wait_read<1>();
+                        if (leader) bulk_wait_read<kWStg - 1>();
                         named_bar_sync(1, 128);
-                        uint8_t* sb = stg + (sctr & 1) * 16384;
+                        uint8_t* sb = stg + (sctr % kWStg) * 16384;
                         ++sctr;
                         if (go)
                             for (int c0 = blk * 64; c0 < min(D, blk * 64 + 64); c0 += 16) {
@@ -997,7 +1001,7 @@ FusedLayout fused_layout(const ScanArgs& a) {
     return L;
 }
 
-constexpr size_t kWorkerSmem = kWStages * 32768 + kImg + 2 * 16384 + 2048 + 512 + 2048 + 512 +
+constexpr size_t kWorkerSmem = kWStages * 32768 + kImg + kWStg * 16384 + 2048 + 512 + 2048 + 512 +
                                (kIQ + 2) * sizeof(Item) + 16 +
                                (3 * kWStages + 2 + 12 + 2 * kIQ) * 8 + 8;
 constexpr size_t kChainSmem = kCStages * 2 * kImg + 2 * kImg + 1024 + 8 + 12 * 8 + 8 + 8;

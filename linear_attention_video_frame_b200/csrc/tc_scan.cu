@@ -68,6 +68,7 @@ struct TcParams {
     float eps;
     int BH, F, S, D;
     int want_output;
+    int rev_chunk;          // > 0: reversed GDN scan reset every rev_chunk frames
 };
 
 // ============================================================================
@@ -322,7 +323,7 @@ tc_chain_kernel(const TcParams p) {
             uint32_t ph = 0;
             for (int f = 0; f < F; ++f) {
                 if (!mbar_wait(&empty[s], ph ^ 1, ab, 0x201)) break;
-                const size_t frame = (size_t)bh * F + f;
+                const size_t frame = (size_t)bh * F + step_frame(f, F, p.rev_chunk);
                 uint8_t* st = ring + s * kStage;
                 mbar_expect_tx(&full[s], kStage);
                 if (!RELU) {
@@ -382,7 +383,10 @@ tc_chain_kernel(const TcParams p) {
         uint32_t ph = 0;
         bool ok = true;     // every epilogue warp runs every named barrier, even after an abort
         for (int f = 0; f < F; ++f) {
-            const size_t frame = (size_t)bh * F + f;
+            const size_t frame = (size_t)bh * F + step_frame(f, F, p.rev_chunk);
+            // first frame of a chunk of the reversed scan: the state restarts
+            // from zero, so whatever the MMA left in TMEM is not used
+            const bool reset = step_resets(f, p.rev_chunk);
             ok = ok && mbar_wait(&full[s], ph, ab, 0x204);
             if (!RELU) ok = ok && mbar_wait(mdone, f & 1, ab, 0x205);
             tc_fence_after();
@@ -399,10 +403,11 @@ tc_chain_kernel(const TcParams p) {
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     const float4 b = *reinterpret_cast<const float4*>(bq + ((c0 / 4 + u) * 128 + row) * 4);
-                    v[4 * u] = fmaf(al, v[4 * u], b.x);
-                    v[4 * u + 1] = fmaf(al, v[4 * u + 1], b.y);
-                    v[4 * u + 2] = fmaf(al, v[4 * u + 2], b.z);
-                    v[4 * u + 3] = fmaf(al, v[4 * u + 3], b.w);
+                    const float ae = reset ? 0.f : al;
+                    v[4 * u] = reset ? b.x : fmaf(ae, v[4 * u], b.x);
+                    v[4 * u + 1] = reset ? b.y : fmaf(ae, v[4 * u + 1], b.y);
+                    v[4 * u + 2] = reset ? b.z : fmaf(ae, v[4 * u + 2], b.z);
+                    v[4 * u + 3] = reset ? b.w : fmaf(ae, v[4 * u + 3], b.w);
                 }
                 tmem_st16(tl + c0, v);
                 store_row16_bf16(mimg, row, c0, v);
@@ -713,6 +718,7 @@ cudaError_t launch_tc_mode(const ScanArgs& a, cudaStream_t st) {
     p.S = a.S;
     p.D = a.D;
     p.want_output = a.o != nullptr;
+    p.rev_chunk = a.rev_chunk;
 
     const uint64_t bhf = (uint64_t)p.BH * p.F;
     CUtensorMap mK, mV, mQ, mO;

@@ -21,7 +21,8 @@ def test_header_declares_the_abi():
     assert declared_symbols() == sorted([
         "la_scan_relu", "la_scan_gdn", "la_state_step", "la_workspace_size",
         "la_query_device_status", "la_status_string", "la_plan", "la_scan_gdn_noalloc",
-        "la_scan_host", "la_host_workspace_size", "la_host_chunk_frames"])
+        "la_scan_host", "la_host_workspace_size", "la_host_chunk_frames",
+        "la_scan_gdn_reverse"])
 
 
 def test_library_exports_every_declared_symbol():
@@ -97,6 +98,26 @@ def test_argument_errors_return_before_any_cuda_call():
                           1, 1, 2, 8, 32, 1e-6, P(), ws, None) == la.LA_ERR_INVALID_ARG
     assert L.la_state_step(5, P(), P(), la.LA_BF16, None, None, 1.0, None, None, None, None,
                            1, 1, 2, 8, 32, P(), ws, None) == la.LA_ERR_INVALID_ARG
+
+
+def test_reverse_scan_argument_errors_and_sizes():
+    L = la.lib
+    P = _fake
+    ws = la.la_workspace_size(la.LA_MODE_GDN_REVERSE, 1, 1, 4, 16, 64)
+    assert ws >= 256 and ws % 256 == 0
+    # the reversed scan never takes the fused path, so it needs per-frame buffers
+    assert la.la_workspace_size(la.LA_MODE_GDN_REVERSE, 1, 20, 181, 880, 128) > \
+        la.la_workspace_size(la.LA_MODE_GDN, 1, 20, 181, 880, 128)
+    assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05", 3)
+    assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 1, 16, 512, 1024, 256)[0] == "simt_f32"
+    args = lambda C, D=64, w=ws: (P(), P(), P(), P(), la.LA_BF16, P(), P(), 0.1, C,
+                                  1, 1, 4, 16, D, P(), w, None)
+    assert L.la_scan_gdn_reverse(*args(0)) == la.LA_ERR_INVALID_ARG
+    assert L.la_scan_gdn_reverse(*args(-3)) == la.LA_ERR_INVALID_ARG
+    assert L.la_scan_gdn_reverse(*args(2, D=24)) == la.LA_ERR_UNSUPPORTED
+    assert L.la_scan_gdn_reverse(*args(2, w=16)) == la.LA_ERR_INVALID_ARG
+    assert L.la_state_step(la.LA_MODE_GDN_REVERSE, P(), P(), la.LA_BF16, P(), P(), 0.1, None,
+                           None, None, None, 1, 1, 4, 16, 64, P(), ws, None) == la.LA_ERR_INVALID_ARG
 
 
 def test_host_chunking_rule():
