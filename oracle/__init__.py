@@ -51,6 +51,14 @@ frame f reads the state after its own update:
     M_f = alpha_f (I - beta_f Kh_f^T Kh_f) M_{f+1} + beta_f Kh_f^T V_f
     O_f = Q_f M_f
 
+Per-token update gate -- SANA-WM paper summary, section 3, "Hybrid
+GDN/Softmax Attention": a decay and a per-token update gate control old
+content.  Reading: the update gate of frame f is a vector beta_f in R^S (one
+value per spatial token) that weighs each token's erase and write, i.e.
+beta_f Kh^T Kh and beta_f Kh^T V become Kh^T diag(beta_f) Kh and
+Kh^T diag(beta_f) V:
+    M_f = alpha_f (M_{f-1} - Kh_f^T diag(beta_f) Kh_f M_{f-1}) + Kh_f^T diag(beta_f) V_f
+
 Array layout: q, k, v, o are [B, H, F, S, D]; alpha, beta are [B, H, F];
 state is [B, H, D, D] (key-major); z is [B, H, D].  Every input is widened
 to float64 first (bf16 and fp32 widen exactly).
@@ -64,6 +72,7 @@ import numpy as np
 __all__ = [
     "relu_scan", "gdn_scan", "relu_state_step", "gdn_state_step",
     "gdn_interval_composite", "compose_exclusive_prefix", "gdn_scan_reverse_chunked",
+    "gdn_scan_token_beta",
 ]
 
 
@@ -195,6 +204,37 @@ def gdn_scan_reverse_chunked(q, k, v, alpha, beta, k_scale: float, chunk_frames:
                     M = a * (M - bt * (kh.T @ P)) + bt * (kh.T @ v[b, h, f])
                     o[b, h, f] = q[b, h, f] @ M
     return o
+
+
+def gdn_scan_token_beta(q, k, v, alpha, beta_token, k_scale: float, state_in=None):
+    """Frame-wise GDN with a per-token update gate.
+
+    SANA-WM paper summary, section 3 ("Hybrid GDN/Softmax Attention"): decay
+    gate per frame, update gate per token.  beta_token: [B, H, F, S].  Each
+    frame in the direct order
+        P = Kh M;  M <- alpha (M - Kh^T (beta * P)) + Kh^T (beta * V);  O = Q M,
+    where beta * X scales row t (token t) of X by beta_t.
+    Returns (o, M_F).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    alpha, bt = _f64(alpha), _f64(beta_token)
+    B, H, F, S, D = _shape(k)
+    o = np.zeros((B, H, F, S, D))
+    m_out = np.zeros((B, H, D, D))
+    m0 = _f64(state_in)
+    kappa = float(k_scale)
+    for b in range(B):
+        for h in range(H):
+            M = np.zeros((D, D)) if m0 is None else m0[b, h].copy()
+            for f in range(F):
+                a = alpha[b, h, f]
+                w = bt[b, h, f][:, None]              # [S, 1] token weights
+                kh = kappa * k[b, h, f]
+                P = kh @ M
+                M = a * (M - kh.T @ (w * P)) + kh.T @ (w * v[b, h, f])
+                o[b, h, f] = q[b, h, f] @ M
+            m_out[b, h] = M
+    return o, m_out
 
 
 def gdn_state_step(k, v, alpha, beta, k_scale: float, state_in=None):

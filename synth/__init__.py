@@ -30,8 +30,8 @@ from typing import Optional, Tuple
 
 import numpy as np
 
-TENSOR_IDS = {"q": 0, "k": 1, "v": 2, "alpha": 10, "beta": 11, "outlier": 20,
-              "state": 30, "z": 31}
+TENSOR_IDS = {"q": 0, "k": 1, "v": 2, "alpha": 10, "beta": 11, "beta_token": 12,
+              "outlier": 20, "state": 30, "z": 31}
 
 
 # ----------------------------------------------------------------------------
@@ -215,6 +215,13 @@ def gates(spec: Spec) -> Tuple[np.ndarray, np.ndarray]:
     a = _draw_gate(spec.alpha, _rng(spec.seed, TENSOR_IDS["alpha"]), shape)
     bt = _draw_gate(spec.beta, _rng(spec.seed, TENSOR_IDS["beta"]), shape)
     return a, bt
+
+
+def token_gates(spec: Spec) -> np.ndarray:
+    """Per-token update gate beta, float32 [B, H, F, S], drawn from the
+    workload's beta distribution (one value per token instead of per frame)."""
+    shape = (spec.B, spec.H, spec.F, spec.S)
+    return _draw_gate(spec.beta, _rng(spec.seed, TENSOR_IDS["beta_token"]), shape)
 
 
 def random_state(spec: Spec, scale: float = 1.0) -> Tuple[np.ndarray, np.ndarray]:

@@ -542,3 +542,81 @@ def test_reverse_pins_reject_planted_mistakes(kind):
     ref = _gdn_reverse_unrolled(q, k, v, a, bt, 0.35, 3)
     assert _rel(oracle.gdn_scan_reverse_chunked(q, k, v, a, bt, 0.35, 3), ref) < 1e-12
     assert _rel(_reverse_mutant(kind)(q, k, v, a, bt, 0.35, 3), ref) > 1e-3
+
+
+# ----------------------------------------------------------------------------
+# Per-token update gate
+# ----------------------------------------------------------------------------
+def _tok_inputs():
+    spec = synth.small(B=1, H=2, F=4, S=6, D=5, dtype="f32", seed=19)
+    q, k, v, a, _ = _inputs(spec)
+    bt = synth.token_gates(spec).astype(np.float64)
+    return spec, q, k, v, a, bt
+
+
+def _gdn_token_unrolled(q, k, v, alpha, bt, kappa, m0):
+    """O_f = Q_f (A_f..A_1 M0 + sum_j A_f..A_{j+1} B_j) with the explicit
+    A_f = alpha_f (I - Kh^T diag(beta_f) Kh) and B_j = Kh^T diag(beta_j) V_j."""
+    B, H, F, S, D = k.shape
+    out = np.zeros_like(q)
+    I = np.eye(D)
+    for b in range(B):
+        for h in range(H):
+            kh = [kappa * k[b, h, f] for f in range(F)]
+            A = [alpha[b, h, f] * (I - kh[f].T @ np.diag(bt[b, h, f]) @ kh[f]) for f in range(F)]
+            Bm = [kh[f].T @ np.diag(bt[b, h, f]) @ v[b, h, f] for f in range(F)]
+            for f in range(F):
+                M = m0[b, h].copy()
+                for j in range(f + 1):
+                    M = A[j] @ M + Bm[j]
+                out[b, h, f] = q[b, h, f] @ M
+    return out
+
+
+def test_token_gate_matches_unrolled_product():
+    spec, q, k, v, a, bt = _tok_inputs()
+    m0, _ = synth.random_state(spec)
+    o, _ = oracle.gdn_scan_token_beta(q, k, v, a, bt, 0.3, m0)
+    assert _rel(o, _gdn_token_unrolled(q, k, v, a, bt, 0.3, m0.astype(float))) < 1e-12
+
+
+def test_token_gate_constant_over_tokens_is_the_frame_gate():
+    spec, q, k, v, a, bt = _tok_inputs()
+    _, _, _, _, bf = _inputs(spec)
+    btok = np.repeat(bf[..., None], spec.S, axis=-1)
+    o, m = oracle.gdn_scan_token_beta(q, k, v, a, btok, 0.3)
+    of, mf = oracle.gdn_scan(q, k, v, a, bf, 0.3)
+    assert _rel(o, of) < 1e-12 and _rel(m, mf) < 1e-12
+
+
+def test_token_gate_zero_removes_the_token():
+    """A token with beta = 0 neither erases nor writes: the scan equals the
+    per-frame-gate scan of the frame without that token."""
+    spec, q, k, v, a, _ = _tok_inputs()
+    btok = np.full((spec.B, spec.H, spec.F, spec.S), 0.6)
+    btok[..., 2] = 0.0
+    o, m = oracle.gdn_scan_token_beta(q, k, v, a, btok, 0.3)
+    keep = [t for t in range(spec.S) if t != 2]
+    _, mf = oracle.gdn_scan(q[..., keep, :], k[..., keep, :], v[..., keep, :], a,
+                            np.full((spec.B, spec.H, spec.F), 0.6), 0.3)
+    assert _rel(m, mf) < 1e-12
+
+
+@pytest.mark.parametrize("kind", ["write_only", "squared", "erase_only"])
+def test_token_gate_pins_reject_planted_mistakes(kind):
+    spec, q, k, v, a, bt = _tok_inputs()
+    m0, _ = synth.random_state(spec)
+    ref = _gdn_token_unrolled(q, k, v, a, bt, 0.3, m0.astype(float))
+    B, H, F, S, D = k.shape
+    o = np.zeros_like(q)
+    for b in range(B):
+        for h in range(H):
+            M = m0[b, h].astype(float)
+            for f in range(F):
+                w = bt[b, h, f][:, None]
+                kh = 0.3 * k[b, h, f]
+                ew = {"write_only": 1.0, "squared": w * w, "erase_only": w}[kind]
+                ww = {"write_only": w, "squared": w * w, "erase_only": 1.0}[kind]
+                M = a[b, h, f] * (M - kh.T @ (ew * (kh @ M))) + kh.T @ (ww * v[b, h, f])
+                o[b, h, f] = q[b, h, f] @ M
+    assert _rel(o, ref) > 1e-3
