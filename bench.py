@@ -50,6 +50,8 @@ WORKLOADS = {
     "stress_relu": (4, "relu"),
     # reversed GDN scan reset every 8 frames, on the 720p 60 s clip
     "gdn_720p_60s_reverse8": (2, "gdn_reverse"),
+    # per-token update gate on the 720p 60 s clip
+    "gdn_720p_60s_token_beta": (2, "gdn_token_beta"),
     "tiny_gdn": (0, "gdn"),
     "tiny_relu": (0, "relu"),
 }
@@ -77,7 +79,8 @@ def call_bytes(mode: str, B: int, H: int, F: int, S: int, D: int, elem: int,
     """q, k, v read once and o written once; alpha, beta read once (GDN);
     the state (and z) written once per (b, h) and read once if given (the
     reversed scan has no state in or out)."""
-    per_frame = 4 * S * D * elem + (8 if mode != "relu" else 0)
+    per_frame = 4 * S * D * elem + (8 if mode != "relu" else 0) + \
+        (4 * (S - 1) if mode == "gdn_token_beta" else 0)
     per_bh = D * D * 4 * (2 if state_in else 1) if mode != "gdn_reverse" else 0
     if mode == "relu":
         per_bh += D * 4 * (2 if state_in else 1)
@@ -230,6 +233,7 @@ def time_oracle_sample(spec, mode, budget_s: float, max_heads=None):
     budget_s of CPU time has passed; return (equivalent frames/s, sample text)."""
     import oracle
     a_all, b_all = synth.gates(spec)
+    btok_all = synth.token_gates(spec) if mode == "gdn_token_beta" else None
     pairs = [(b, h) for b in range(spec.B) for h in range(spec.H)]
     done, t_total = 0, 0.0
     for b, h in pairs:
@@ -241,6 +245,8 @@ def time_oracle_sample(spec, mode, budget_s: float, max_heads=None):
             oracle.relu_scan(q, k, v, spec.eps)
         elif mode == "gdn_reverse":
             oracle.gdn_scan_reverse_chunked(q, k, v, a, bt, spec.k_scale, REVERSE_CHUNK)
+        elif mode == "gdn_token_beta":
+            oracle.gdn_scan_token_beta(q, k, v, a, btok_all[b:b + 1, h:h + 1], spec.k_scale)
         else:
             oracle.gdn_scan(q, k, v, a, bt, spec.k_scale)
         t_total += time.perf_counter() - t0
@@ -336,7 +342,11 @@ def run_ours(args):
     z = torch.empty((B, H, D), dtype=torch.float32, device=dev)
     plan = step_plan(spec, mode)
     mode_c = {"gdn": la.LA_MODE_GDN, "relu": la.LA_MODE_RELU,
-              "gdn_reverse": la.LA_MODE_GDN_REVERSE}[mode]
+              "gdn_reverse": la.LA_MODE_GDN_REVERSE,
+              "gdn_token_beta": la.LA_MODE_GDN_TOKEN_BETA}[mode]
+    if mode == "gdn_token_beta":
+        host["beta"] = torch.from_numpy(synth.token_gates(spec)).pin_memory()
+        dev_in["beta"] = host["beta"].to(dev)
     ws = la.workspace_for(mode_c,
                           B, H, max(n for _, n, _ in plan), S, D, dev)
     views = []
@@ -353,7 +363,10 @@ def run_ours(args):
 
     def one_step():
         for (q, k, v, al, be, oo, si) in views:
-            if mode == "gdn_reverse":
+            if mode == "gdn_token_beta":
+                la.la_scan_gdn_token_beta(q, k, v, al, be, spec.k_scale, o=oo, state_out=state,
+                                          workspace=ws, stream=stream)
+            elif mode == "gdn_reverse":
                 la.la_scan_gdn_reverse(q, k, v, al, be, spec.k_scale, REVERSE_CHUNK, o=oo,
                                        workspace=ws, stream=stream)
             elif mode == "gdn":
@@ -417,21 +430,28 @@ def run_ours(args):
     ins = ("q", "k", "v") if mode == "relu" else ("q", "k", "v", "alpha", "beta")
     if mode == "gdn_reverse":
         so_host = None          # the reversed scan has no state out
+    special = mode in ("gdn_reverse", "gdn_token_beta")
     h2d = sum(host[x].numel() * host[x].element_size() for x in ins)
     d2h = sum(t.numel() * t.element_size() for t in (o_host, so_host, zo_host) if t is not None)
     e2e_call = "la_scan_host"
-    if mode == "gdn_reverse":
-        # no host-buffer form of the reversed scan: H2D, the call and D2H in
-        # order on one stream
-        e2e_call = "H2D + la_scan_gdn_reverse + D2H"
+    if special:
+        # no host-buffer form of these calls: H2D, the call and D2H in order
+        # on one stream
+        e2e_call = f"H2D + la_scan_{mode} + D2H"
         hws = None
 
         def e2e_step():
             for x in ins:
                 dev_in[x].copy_(host[x], non_blocking=True)
-            la.la_scan_gdn_reverse(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"],
-                                   dev_in["beta"], spec.k_scale, REVERSE_CHUNK, o=o,
-                                   workspace=ws, stream=stream)
+            if mode == "gdn_reverse":
+                la.la_scan_gdn_reverse(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"],
+                                       dev_in["beta"], spec.k_scale, REVERSE_CHUNK, o=o,
+                                       workspace=ws, stream=stream)
+            else:
+                la.la_scan_gdn_token_beta(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"],
+                                          dev_in["beta"], spec.k_scale, o=o, state_out=state,
+                                          workspace=ws, stream=stream)
+                so_host.copy_(state, non_blocking=True)
             o_host.copy_(o, non_blocking=True)
     else:
         hws = None if args.no_e2e else la.host_workspace_for(mode_c, dtc, B, H, F, S, D, chunk,
@@ -492,8 +512,8 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if spec.dtype == "bf16" else "f32",
         "data": "synthetic (seeded numpy PCG64, bf16 round-to-nearest-even)",
-        "config": {"workload": base.name + (f"_reverse{REVERSE_CHUNK}" if mode == "gdn_reverse"
-                                            else ""),
+        "config": {"workload": base.name + {"gdn_reverse": f"_reverse{REVERSE_CHUNK}",
+                                            "gdn_token_beta": "_token_beta"}.get(mode, ""),
                    "mode": mode, "B": B, "H": H, "F": F, "S": S, "D": D,
                    "calls_per_step": len(plan), "global_batch": B * world,
                    "l2": "inputs larger than L2 (no flush)",
@@ -505,8 +525,7 @@ def run_ours(args):
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "latent frames/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": Ke, "call": e2e_call,
-                "chunk_frames": (la.la_host_chunk_frames(F, chunk) if mode != "gdn_reverse"
-                                 else None),
+                "chunk_frames": (la.la_host_chunk_frames(F, chunk) if not special else None),
                 "host_memory": "pinned"},
         "clocks": clocks.summary(),
         "device_status": la.la_status_string(status),

@@ -86,7 +86,8 @@ typedef enum la_dtype { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
 typedef enum la_mode {
     LA_MODE_RELU = 0,
     LA_MODE_GDN = 1,
-    LA_MODE_GDN_REVERSE = 2      /* la_scan_gdn_reverse (for la_workspace_size, la_plan) */
+    LA_MODE_GDN_REVERSE = 2,     /* la_scan_gdn_reverse (for la_workspace_size, la_plan) */
+    LA_MODE_GDN_TOKEN_BETA = 3   /* la_scan_gdn_token_beta (for la_workspace_size, la_plan) */
 } la_mode;
 
 /*
@@ -153,6 +154,31 @@ LA_API la_status la_scan_gdn_reverse(const void* q, const void* k, const void* v
                                      int B, int H, int F, int S, int D,
                                      void* workspace, size_t workspace_bytes,
                                      cudaStream_t stream);
+
+/*
+ * Frame-wise GDN with a per-token update gate.
+ * Source: SANA-WM paper summary (paperlayer), section 3, "Hybrid GDN/Softmax
+ * Attention" -- a decay gate and a per-token update gate control how old
+ * content is kept.  Reading: the update gate of frame f is one value per
+ * spatial token, weighing that token's erase and write:
+ *   M_f = alpha_f (M_{f-1} - Kh_f^T diag(beta_f) Kh_f M_{f-1}) + Kh_f^T diag(beta_f) V_f
+ *   O_f = Q_f M_f
+ *
+ * beta_token  in : [B,H,F,S] f32, each value >= 0 (the gate of token s of
+ *                  frame f); alpha [B,H,F] as for la_scan_gdn.
+ * Everything else as for la_scan_gdn.  The workspace is
+ * la_workspace_size(LA_MODE_GDN_TOKEN_BETA, B, H, F, S, D) bytes.  bf16
+ * inputs with 64 <= D <= 128 run on the tensor-core path (each token row of
+ * K and V is scaled by sqrt(beta) in shared memory, in bf16, before the
+ * unchanged contractions); other shapes on the float32 SIMT kernel.
+ */
+LA_API la_status la_scan_gdn_token_beta(const void* q, const void* k, const void* v, void* o,
+                                        la_dtype dt, const float* alpha,
+                                        const float* beta_token, float k_scale,
+                                        const float* state_in, float* state_out,
+                                        int B, int H, int F, int S, int D,
+                                        void* workspace, size_t workspace_bytes,
+                                        cudaStream_t stream);
 
 /*
  * Advance the cached state over finished frames without producing outputs:

@@ -21,7 +21,8 @@ import torch
 __all__ = [
     "LA_OK", "LA_ERR_INVALID_ARG", "LA_ERR_UNSUPPORTED", "LA_ERR_CUDA", "LA_ERR_TIMEOUT",
     "LA_F32", "LA_BF16", "LA_MODE_RELU", "LA_MODE_GDN", "LA_MODE_GDN_REVERSE", "LaScanError",
-    "lib", "LIB_PATH", "la_scan_gdn_reverse",
+    "lib", "LIB_PATH", "la_scan_gdn_reverse", "la_scan_gdn_token_beta",
+    "LA_MODE_GDN_TOKEN_BETA",
     "la_scan_relu", "la_scan_gdn", "la_state_step", "la_workspace_size",
     "la_query_device_status", "la_status_string", "la_plan", "workspace_for",
     "la_scan_gdn_noalloc", "LA_NOALLOC_SCRATCH_BYTES", "la_scan_host",
@@ -30,7 +31,7 @@ __all__ = [
 
 LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CUDA, LA_ERR_TIMEOUT = 0, 1, 2, 3, 4
 LA_F32, LA_BF16 = 0, 1
-LA_MODE_RELU, LA_MODE_GDN, LA_MODE_GDN_REVERSE = 0, 1, 2
+LA_MODE_RELU, LA_MODE_GDN, LA_MODE_GDN_REVERSE, LA_MODE_GDN_TOKEN_BETA = 0, 1, 2, 3
 LA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblavf.so")
@@ -59,6 +60,8 @@ def _load() -> ctypes.CDLL:
     L.la_workspace_size.restype = Z
     L.la_query_device_status.argtypes = [P, P]
     L.la_query_device_status.restype = I
+    L.la_scan_gdn_token_beta.argtypes = [P, P, P, P, I, P, P, F, P, P, I, I, I, I, I, P, Z, P]
+    L.la_scan_gdn_token_beta.restype = I
     L.la_scan_gdn_reverse.argtypes = [P, P, P, P, I, P, P, F, I, I, I, I, I, I, P, Z, P]
     L.la_scan_gdn_reverse.restype = I
     L.la_scan_gdn_noalloc.argtypes = [P, P, P, P, I, P, P, F, P, P, I, I, I, I, I, P]
@@ -196,6 +199,29 @@ def la_scan_gdn_reverse(q, k, v, alpha, beta, k_scale: float, chunk_frames: int,
                                  _ptr(beta), float(k_scale), int(chunk_frames), B, H, F, S, D,
                                  _ptr(workspace), workspace.numel(), _stream(stream))
     _raise(st, "la_scan_gdn_reverse")
+    return o
+
+
+def la_scan_gdn_token_beta(q, k, v, alpha, beta_token, k_scale: float, o=None, state_in=None,
+                           state_out=None, workspace=None, stream=None):
+    """Frame-wise GDN with a per-token update gate beta_token [B, H, F, S]
+    (see include/la_scan.h)."""
+    B, H, F, S, D = k.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _check(t, n, (B, H, F, S, D), k.dtype)
+    _check(alpha, "alpha", (B, H, F), torch.float32)
+    _check(beta_token, "beta_token", (B, H, F, S), torch.float32)
+    for t, n in ((state_in, "state_in"), (state_out, "state_out")):
+        _check(t, n, (B, H, D, D), torch.float32)
+    if o is None:
+        o = torch.empty_like(q)
+    if workspace is None:
+        workspace = workspace_for(LA_MODE_GDN_TOKEN_BETA, B, H, F, S, D, q.device)
+    st = lib.la_scan_gdn_token_beta(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _dtype_code(k),
+                                    _ptr(alpha), _ptr(beta_token), float(k_scale),
+                                    _ptr(state_in), _ptr(state_out), B, H, F, S, D,
+                                    _ptr(workspace), workspace.numel(), _stream(stream))
+    _raise(st, "la_scan_gdn_token_beta")
     return o
 
 

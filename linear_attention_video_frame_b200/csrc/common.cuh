@@ -31,7 +31,8 @@ struct ScanArgs {
     const void* v;
     void* o;                 // NULL for a state step
     const float* alpha;      // GDN only
-    const float* beta;       // GDN only
+    const float* beta;       // GDN only (per frame)
+    const float* beta_tok;   // GDN with a per-token update gate [B, H, F, S], else NULL
     const float* state_in;   // may be NULL
     const float* z_in;       // ReLU only, may be NULL
     float* state_out;        // may be NULL

@@ -57,14 +57,17 @@ bool force_simt() {
 
 bool use_tc(const ScanArgs& a) { return !force_simt() && tc_eligible(a); }
 
-// The reversed scan runs on the three-kernel tensor-core path or the SIMT kernel.
-bool use_wide(const ScanArgs& a) { return !force_simt() && a.rev_chunk == 0 && wide_eligible(a); }
+// The reversed scan and the per-token gate run on the three-kernel tensor-core
+// path or the SIMT kernel.
+bool special(const ScanArgs& a) { return a.rev_chunk != 0 || a.beta_tok != nullptr; }
+
+bool use_wide(const ScanArgs& a) { return !force_simt() && !special(a) && wide_eligible(a); }
 
 // LA_SCAN_NO_FUSE=1 keeps tensor-core calls on the three-kernel path (tests
 // compare the two).
 bool use_fused(const ScanArgs& a) {
     const char* e = std::getenv("LA_SCAN_NO_FUSE");
-    return use_tc(a) && a.rev_chunk == 0 && !(e && e[0] == '1') && fused_eligible(a);
+    return use_tc(a) && !special(a) && !(e && e[0] == '1') && fused_eligible(a);
 }
 
 size_t workspace_needed(const ScanArgs& a) {
@@ -88,12 +91,13 @@ la_status validate(const ScanArgs& a, bool need_q) {
     if (a.F > 0) {
         if (!a.k || !a.v) return LA_ERR_INVALID_ARG;
         if (need_q && (!a.q || !a.o)) return LA_ERR_INVALID_ARG;
-        if (a.mode == LA_MODE_GDN && (!a.alpha || !a.beta)) return LA_ERR_INVALID_ARG;
+        if (a.mode == LA_MODE_GDN && (!a.alpha || (!a.beta && !a.beta_tok)))
+            return LA_ERR_INVALID_ARG;
     }
     int dev = 0;
     la_status s = check_device(&dev);
     if (s != LA_OK) return s;
-    const void* ptrs[] = {a.q, a.k, a.v, a.o, a.alpha, a.beta, a.state_in, a.z_in,
+    const void* ptrs[] = {a.q, a.k, a.v, a.o, a.alpha, a.beta, a.beta_tok, a.state_in, a.z_in,
                           a.state_out, a.z_out, a.ws};
     for (const void* p : ptrs)
         if ((s = check_ptr(p, dev)) != LA_OK) return s;
@@ -181,6 +185,24 @@ extern "C" la_status la_scan_gdn_reverse(const void* q, const void* k, const voi
     return run(a, stream);
 }
 
+extern "C" la_status la_scan_gdn_token_beta(const void* q, const void* k, const void* v, void* o,
+                                            la_dtype dt, const float* alpha,
+                                            const float* beta_token, float k_scale,
+                                            const float* state_in, float* state_out,
+                                            int B, int H, int F, int S, int D,
+                                            void* workspace, size_t workspace_bytes,
+                                            cudaStream_t stream) {
+    if (dt != LA_F32 && dt != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (F > 0 && !beta_token) return LA_ERR_INVALID_ARG;
+    ScanArgs a = base_args(k, v, dt, B, H, F, S, D, workspace, workspace_bytes);
+    a.q = q; a.o = o; a.mode = LA_MODE_GDN; a.k_scale = k_scale;
+    a.alpha = alpha; a.beta_tok = beta_token;
+    a.state_in = state_in; a.state_out = state_out;
+    la_status s = validate(a, true);
+    if (s != LA_OK) return s;
+    return run(a, stream);
+}
+
 extern "C" la_status la_state_step(la_mode mode, const void* k, const void* v, la_dtype dt,
                                    const float* alpha, const float* beta, float k_scale,
                                    const float* state_in, const float* z_in,
@@ -204,10 +226,11 @@ extern "C" la_status la_state_step(la_mode mode, const void* k, const void* v, l
 
 extern "C" size_t la_workspace_size(la_mode mode, int B, int H, int F, int S, int D) {
     if (B < 1 || H < 1 || F < 0 || S < 1 || !shape_supported(D)) return 0;
-    if (mode != LA_MODE_RELU && mode != LA_MODE_GDN && mode != LA_MODE_GDN_REVERSE) return 0;
+    if (mode < LA_MODE_RELU || mode > LA_MODE_GDN_TOKEN_BETA) return 0;
     ScanArgs a = base_args(nullptr, nullptr, LA_BF16, B, H, F, S, D, nullptr, 0);
     a.mode = mode == LA_MODE_RELU ? LA_MODE_RELU : LA_MODE_GDN;
     a.rev_chunk = mode == LA_MODE_GDN_REVERSE ? 1 : 0;
+    if (mode == LA_MODE_GDN_TOKEN_BETA) a.beta_tok = reinterpret_cast<const float*>(uintptr_t(16));
     size_t n = workspace_needed(a);
     a.bf16 = 0;
     size_t n32 = workspace_needed(a);
@@ -228,12 +251,12 @@ extern "C" la_status la_query_device_status(void* workspace, cudaStream_t stream
 extern "C" const char* la_plan(la_mode mode, la_dtype dt, int B, int H, int F, int S, int D,
                                int* kernels) {
     if (B < 1 || H < 1 || F < 0 || S < 1 || !shape_supported(D)) return nullptr;
-    if ((mode != LA_MODE_RELU && mode != LA_MODE_GDN && mode != LA_MODE_GDN_REVERSE) ||
-        (dt != LA_F32 && dt != LA_BF16))
+    if (mode < LA_MODE_RELU || mode > LA_MODE_GDN_TOKEN_BETA || (dt != LA_F32 && dt != LA_BF16))
         return nullptr;
     ScanArgs a = base_args(nullptr, nullptr, dt, B, H, F, S, D, nullptr, 0);
     a.mode = mode == LA_MODE_RELU ? LA_MODE_RELU : LA_MODE_GDN;
     a.rev_chunk = mode == LA_MODE_GDN_REVERSE ? 1 : 0;
+    if (mode == LA_MODE_GDN_TOKEN_BETA) a.beta_tok = reinterpret_cast<const float*>(uintptr_t(16));
     a.o = reinterpret_cast<void*>(uintptr_t(1));    // a scan (with outputs)
     if (use_fused(a)) {
         if (kernels) *kernels = 1;

@@ -82,7 +82,11 @@ simt_scan_kernel(ScanArgs a) {
         }
         const size_t frame = (bh * F + f) * (size_t)S;   // first token row of the frame
         float al = 1.f, bt = 1.f;
-        if (!relu) { al = a.alpha[bh * F + f]; bt = a.beta[bh * F + f]; }
+        if (!relu) {
+            al = a.alpha[bh * F + f];
+            bt = a.beta_tok ? 1.f : a.beta[bh * F + f];   // per-token gates weigh U below
+        }
+        const float* btok = a.beta_tok ? a.beta_tok + (bh * F + f) * (size_t)S : nullptr;
 
         float acc[32];
 #pragma unroll
@@ -110,7 +114,8 @@ simt_scan_kernel(ScanArgs a) {
                 for (int t = rr; t < kT; t += kRowsPerPass) {
                     float s = 0.f;
                     for (int d = 0; d < D; ++d) s = fmaf(sK[t * D + d], sM[d * kDJ + jj], s);
-                    sU[t * kDJ + jj] = sV[t * kDJ + jj] - al * s;
+                    const float w = (btok && t < nt) ? btok[t0 + t] : 1.f;
+                    sU[t * kDJ + jj] = w * (sV[t * kDJ + jj] - al * s);
                 }
                 __syncthreads();
                 src = sU;

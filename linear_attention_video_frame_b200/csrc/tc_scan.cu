@@ -69,15 +69,19 @@ struct TcParams {
     int BH, F, S, D;
     int want_output;
     int rev_chunk;          // > 0: reversed GDN scan reset every rev_chunk frames
+    const float* beta_tok;  // per-token update gate [BHF][S] (GDN), or NULL
 };
 
 // ============================================================================
 // gram: per-frame contractions over tokens
 // ============================================================================
 // warp 0: TMA producer; warp 1: TMEM owner + MMA issuer; warps 2-5: epilogue;
-// warps 6-9 (ReLU): apply phi to each K tile in shared memory before the MMA.
-template <bool RELU>
-__global__ void __launch_bounds__(RELU ? 320 : 192, 1)
+// warps 6-9 (ReLU): apply phi to each K tile in shared memory before the MMA;
+// (GDN with a per-token update gate, TOKB): scale every token row of the K and
+// V tiles by sqrt(beta_t), so that the unchanged MMAs produce
+// Kh^T diag(beta) Kh and Kh^T diag(beta) V.
+template <bool RELU, bool TOKB = false>
+__global__ void __launch_bounds__((RELU || TOKB) ? 320 : 192, 1)
 tc_gram_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapK,
                const __grid_constant__ CUtensorMap mapV) {
     extern __shared__ uint8_t smem_raw[];
@@ -159,7 +163,8 @@ tc_gram_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapK,
                 tc_fence_after();
                 const uint32_t dG = tbase + slot * 256, dW = dG + 128;
                 for (int t = 0; t < nt; ++t) {
-                    if (!(ok = mbar_wait(RELU ? &xform[s] : &full[s], ph, ab, 0x103))) break;
+                    if (!(ok = mbar_wait((RELU || TOKB) ? &xform[s] : &full[s], ph, ab, 0x103)))
+                        break;
                     tc_fence_after();
                     const uint32_t sk = smem_u32(ring + s * 32768), sv = sk + 16384;
 #pragma unroll
@@ -194,7 +199,7 @@ tc_gram_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapK,
             const uint32_t tl = tbase + (uint32_t(q * 32) << 16) + slot * 256;
             float* bq = p.bmat + (size_t)item * (kQuadMat / 4);
             if (!RELU) {
-                const float bt = p.beta[item];
+                const float bt = TOKB ? 1.f : p.beta[item];   // TOKB: beta is in the operands
                 const float sg = bt * p.k_scale * p.k_scale, sw = bt * p.k_scale;
                 if (issuer) bulk_wait_read<0>();       // staging free again
                 named_bar_sync(1, kEpiThreads);
@@ -245,20 +250,57 @@ tc_gram_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapK,
         }
         if (issuer) bulk_wait_all<0>();
     } else {
-        // ---------------- ReLU transform: phi(K) in place ----------------
+        // ---------------- transform: phi(K) (ReLU) or sqrt(beta_t) rows (TOKB) ----------------
         const int tl = threadIdx.x - 192;          // 0..127
         int s = 0;
         uint32_t ph = 0;
         bool ok = true;
+        // TOKB: chunk i = tl + 128 m of a stage lies in token row (tl / 8 + 16 m) % 64,
+        // so a thread needs the gates of 4 rows per tile; they are fetched one
+        // tile ahead.
+        auto gates4 = [&](int item, int t, float (&w)[4]) {
+            const float* bq = p.beta_tok + (size_t)item * p.S;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int tok = t * kTokG + (tl >> 3) + 16 * u;
+                w[u] = tok < p.S ? __ldg(bq + tok) : 0.f;
+            }
+        };
+        float wn[4] = {0.f, 0.f, 0.f, 0.f};
+        if (TOKB && blockIdx.x < nitems) gates4(blockIdx.x, 0, wn);
         for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x) {
             for (int t = 0; t < nt; ++t) {
+                float w[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) w[u] = sqrtf(wn[u]);
+                if (TOKB) {                                   // the next tile's gates
+                    if (t + 1 < nt) gates4(item, t + 1, wn);
+                    else if (item + (int)gridDim.x < nitems) gates4(item + gridDim.x, 0, wn);
+                }
                 if (!(ok = mbar_wait(&full[s], ph, ab, 0x105))) break;
                 uint4* kt = reinterpret_cast<uint4*>(ring + s * 32768);
-                for (int i = tl; i < 2 * (int)kBoxG / 16; i += 128) {
-                    uint4 x = kt[i];
-                    x.x = relu_bf16x2(x.x); x.y = relu_bf16x2(x.y);
-                    x.z = relu_bf16x2(x.z); x.w = relu_bf16x2(x.w);
-                    kt[i] = x;
+                if (TOKB) {
+                    // all 32 KB of the stage (K and V, both 64-column boxes): 64 token
+                    // rows of 128 bytes per box; a row's 16-byte chunks are permuted
+                    // by the swizzle but stay in the row, so row scaling ignores it
+#pragma unroll 4
+                    for (int m = 0; m < 16; ++m) {
+                        const int i = tl + 128 * m;
+                        const float ww = w[m & 3];
+                        uint4 x = kt[i];
+                        x.x = pack_bf16x2(bf16_lo(x.x) * ww, bf16_hi(x.x) * ww);
+                        x.y = pack_bf16x2(bf16_lo(x.y) * ww, bf16_hi(x.y) * ww);
+                        x.z = pack_bf16x2(bf16_lo(x.z) * ww, bf16_hi(x.z) * ww);
+                        x.w = pack_bf16x2(bf16_lo(x.w) * ww, bf16_hi(x.w) * ww);
+                        kt[i] = x;
+                    }
+                } else {
+                    for (int i = tl; i < 2 * (int)kBoxG / 16; i += 128) {
+                        uint4 x = kt[i];
+                        x.x = relu_bf16x2(x.x); x.y = relu_bf16x2(x.y);
+                        x.z = relu_bf16x2(x.z); x.w = relu_bf16x2(x.w);
+                        kt[i] = x;
+                    }
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -719,6 +761,7 @@ cudaError_t launch_tc_mode(const ScanArgs& a, cudaStream_t st) {
     p.D = a.D;
     p.want_output = a.o != nullptr;
     p.rev_chunk = a.rev_chunk;
+    p.beta_tok = a.beta_tok;
 
     const uint64_t bhf = (uint64_t)p.BH * p.F;
     CUtensorMap mK, mV, mQ, mO;
@@ -731,6 +774,9 @@ cudaError_t launch_tc_mode(const ScanArgs& a, cudaStream_t st) {
 
     static bool attr_done = false;
     if (!attr_done) {
+        if (!RELU)
+            cudaFuncSetAttribute(tc_gram_kernel<false, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_gram);
         cudaFuncSetAttribute(tc_gram_kernel<RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem_gram);
         cudaFuncSetAttribute(tc_chain_kernel<RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -742,7 +788,10 @@ cudaError_t launch_tc_mode(const ScanArgs& a, cudaStream_t st) {
     const int nsm = sm_count();
     const int grid_f = (int)std::min<uint64_t>(bhf, (uint64_t)nsm);
     const int thr = RELU ? 320 : 192;
-    tc_gram_kernel<RELU><<<grid_f, thr, smem_gram, st>>>(p, mK, mV);
+    if (!RELU && p.beta_tok)
+        tc_gram_kernel<false, true><<<grid_f, 320, smem_gram, st>>>(p, mK, mV);
+    else
+        tc_gram_kernel<RELU><<<grid_f, thr, smem_gram, st>>>(p, mK, mV);
     tc_chain_kernel<RELU><<<p.BH, 192, RELU ? smem_chain_relu : smem_chain_gdn, st>>>(p);
     if (p.want_output) tc_output_kernel<RELU><<<grid_f, thr, smem_out, st>>>(p, mQ, mO);
     return cudaGetLastError();

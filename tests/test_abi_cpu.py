@@ -22,7 +22,7 @@ def test_header_declares_the_abi():
         "la_scan_relu", "la_scan_gdn", "la_state_step", "la_workspace_size",
         "la_query_device_status", "la_status_string", "la_plan", "la_scan_gdn_noalloc",
         "la_scan_host", "la_host_workspace_size", "la_host_chunk_frames",
-        "la_scan_gdn_reverse"])
+        "la_scan_gdn_reverse", "la_scan_gdn_token_beta"])
 
 
 def test_library_exports_every_declared_symbol():
@@ -118,6 +118,21 @@ def test_reverse_scan_argument_errors_and_sizes():
     assert L.la_scan_gdn_reverse(*args(2, w=16)) == la.LA_ERR_INVALID_ARG
     assert L.la_state_step(la.LA_MODE_GDN_REVERSE, P(), P(), la.LA_BF16, P(), P(), 0.1, None,
                            None, None, None, 1, 1, 4, 16, 64, P(), ws, None) == la.LA_ERR_INVALID_ARG
+
+
+def test_token_gate_scan_argument_errors_and_plan():
+    L = la.lib
+    P = _fake
+    ws = la.la_workspace_size(la.LA_MODE_GDN_TOKEN_BETA, 1, 1, 4, 16, 64)
+    assert ws >= 256 and ws % 256 == 0
+    assert la.la_plan(la.LA_MODE_GDN_TOKEN_BETA, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05", 3)
+    assert la.la_plan(la.LA_MODE_GDN_TOKEN_BETA, la.LA_F32, 1, 2, 8, 64, 32)[0] == "simt_f32"
+    assert la.la_workspace_size(4, 1, 1, 4, 16, 64) == 0
+    args = lambda bt=P(), D=64, w=ws: (P(), P(), P(), P(), la.LA_BF16, P(), bt, 0.1, None, None,
+                                       1, 1, 4, 16, D, P(), w, None)
+    assert L.la_scan_gdn_token_beta(*args(bt=None)) == la.LA_ERR_INVALID_ARG
+    assert L.la_scan_gdn_token_beta(*args(D=24)) == la.LA_ERR_UNSUPPORTED
+    assert L.la_scan_gdn_token_beta(*args(w=16)) == la.LA_ERR_INVALID_ARG
 
 
 def test_host_chunking_rule():
