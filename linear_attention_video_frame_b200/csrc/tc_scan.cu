@@ -31,6 +31,10 @@
 // The fp32 per-frame matrices B_f / dM_f are stored "quad-interleaved":
 // element (i, j) at ((j / 4) * 128 + i) * 4 + j % 4, so that the 32 lanes of
 // a warp, which own 32 consecutive rows, touch 512 contiguous bytes.
+#include <algorithm>
+#include <cstdlib>
+#include <mutex>
+
 #include "tc_common.cuh"
 #include "tmap.cuh"
 
@@ -70,7 +74,15 @@ struct TcParams {
     int want_output;
     int rev_chunk;          // > 0: reversed GDN scan reset every rev_chunk frames
     const float* beta_tok;  // per-token update gate [BHF][S] (GDN), or NULL
+    int f0, Fc;             // this launch covers frames [f0, f0 + Fc) of every head
 };
+
+// Global frame index (into q, k, v, o, the gates and the per-frame workspace
+// buffers, all sized for the whole clip) of launch-local item `it` = bh Fc + fl.
+__device__ __forceinline__ int global_item(const TcParams& p, int it) {
+    const int bh = it / p.Fc;
+    return bh * p.F + p.f0 + (it - bh * p.Fc);
+}
 
 // ============================================================================
 // gram: per-frame contractions over tokens
@@ -124,7 +136,7 @@ tc_gram_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapK,
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
     const Abort ab{abort_flag, p.status};
-    const int nitems = p.BH * p.F;
+    const int nitems = p.BH * p.Fc;
     const int nt = (p.S + kTokG - 1) / kTokG;
     const int D = p.D;
 
@@ -136,7 +148,8 @@ tc_gram_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapK,
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
-            for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x) {
+            for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+            const int item = global_item(p, it);
                 for (int t = 0; t < nt; ++t) {
                     if (!(ok = mbar_wait(&empty[s], ph ^ 1, ab, 0x101))) break;
                     uint8_t* st = ring + s * 32768;
@@ -157,7 +170,8 @@ tc_gram_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapK,
             int s = 0, li = 0;
             uint32_t ph = 0;
             bool ok = true;
-            for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
+            for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++li) {
+            const int item = global_item(p, it);
                 const int slot = li & 1;
                 if (!(ok = mbar_wait(&accempty[slot], ((li >> 1) & 1) ^ 1, ab, 0x102))) break;
                 tc_fence_after();
@@ -192,7 +206,8 @@ tc_gram_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapK,
         const bool issuer = (threadIdx.x == 64);
         int li = 0;
         bool ok = true;     // every epilogue warp runs every named barrier, even after an abort
-        for (int item = blockIdx.x; item < nitems; item += gridDim.x, ++li) {
+        for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++li) {
+            const int item = global_item(p, it);
             const int slot = li & 1;
             ok = ok && mbar_wait(&accfull[slot], (li >> 1) & 1, ab, 0x104);
             tc_fence_after();
@@ -267,15 +282,17 @@ tc_gram_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapK,
             }
         };
         float wn[4] = {0.f, 0.f, 0.f, 0.f};
-        if (TOKB && blockIdx.x < nitems) gates4(blockIdx.x, 0, wn);
-        for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x) {
+        if (TOKB && (int)blockIdx.x < nitems) gates4(global_item(p, blockIdx.x), 0, wn);
+        for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+            const int item = global_item(p, it);
             for (int t = 0; t < nt; ++t) {
                 float w[4];
 #pragma unroll
                 for (int u = 0; u < 4; ++u) w[u] = sqrtf(wn[u]);
                 if (TOKB) {                                   // the next tile's gates
                     if (t + 1 < nt) gates4(item, t + 1, wn);
-                    else if (item + (int)gridDim.x < nitems) gates4(item + gridDim.x, 0, wn);
+                    else if (it + (int)gridDim.x < nitems)
+                        gates4(global_item(p, it + gridDim.x), 0, wn);
                 }
                 if (!(ok = mbar_wait(&full[s], ph, ab, 0x105))) break;
                 uint4* kt = reinterpret_cast<uint4*>(ring + s * 32768);
@@ -339,6 +356,7 @@ tc_chain_kernel(const TcParams p) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.x;
     const int F = p.F, D = p.D;
+    const int nsteps = p.Fc;                // steps of this launch: clip steps f0 .. f0 + Fc - 1
     if (threadIdx.x == 0) {
         for (int s = 0; s < kCStages; ++s) {
             mbar_init(&full[s], 1);
@@ -363,9 +381,9 @@ tc_chain_kernel(const TcParams p) {
         if (lane == 0) {
             int s = 0;
             uint32_t ph = 0;
-            for (int f = 0; f < F; ++f) {
+            for (int f = 0; f < nsteps; ++f) {
                 if (!mbar_wait(&empty[s], ph ^ 1, ab, 0x201)) break;
-                const size_t frame = (size_t)bh * F + step_frame(f, F, p.rev_chunk);
+                const size_t frame = (size_t)bh * F + step_frame(p.f0 + f, F, p.rev_chunk);
                 uint8_t* st = ring + s * kStage;
                 mbar_expect_tx(&full[s], kStage);
                 if (!RELU) {
@@ -383,7 +401,7 @@ tc_chain_kernel(const TcParams p) {
             const uint32_t idC = idesc_bf16(128, D, false, true, /*negate_a=*/true);
             int s = 0;
             uint32_t ph = 0;
-            for (int f = 0; f < F; ++f) {
+            for (int f = 0; f < nsteps; ++f) {
                 if (!mbar_wait(&full[s], ph, ab, 0x202)) break;
                 if (!mbar_wait(mready, f & 1, ab, 0x203)) break;
                 tc_fence_after();
@@ -424,11 +442,11 @@ tc_chain_kernel(const TcParams p) {
         int s = 0;
         uint32_t ph = 0;
         bool ok = true;     // every epilogue warp runs every named barrier, even after an abort
-        for (int f = 0; f < F; ++f) {
-            const size_t frame = (size_t)bh * F + step_frame(f, F, p.rev_chunk);
+        for (int f = 0; f < nsteps; ++f) {
+            const size_t frame = (size_t)bh * F + step_frame(p.f0 + f, F, p.rev_chunk);
             // first frame of a chunk of the reversed scan: the state restarts
             // from zero, so whatever the MMA left in TMEM is not used
-            const bool reset = step_resets(f, p.rev_chunk);
+            const bool reset = step_resets(p.f0 + f, p.rev_chunk);
             ok = ok && mbar_wait(&full[s], ph, ab, 0x204);
             if (!RELU) ok = ok && mbar_wait(mdone, f & 1, ab, 0x205);
             tc_fence_after();
@@ -437,7 +455,7 @@ tc_chain_kernel(const TcParams p) {
             const float* bq = reinterpret_cast<const float*>(st + (RELU ? 0 : kImg));
             if (issuer && p.want_output) bulk_wait_read<0>();   // image free for rewriting
             named_bar_sync(1, kEpiThreads);
-            const bool last = (f == F - 1);
+            const bool last = (f == nsteps - 1);
             for (int c0 = 0; c0 < D && ok; c0 += 16) {
                 float v[16];
                 tmem_ld16(tl + c0, v);
@@ -540,7 +558,7 @@ tc_output_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapQ,
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
     const Abort ab{abort_flag, p.status};
-    const int nitems = p.BH * p.F;
+    const int nitems = p.BH * p.Fc;
     const int nt = (p.S + kTokO - 1) / kTokO;
     const int D = p.D;
 
@@ -552,7 +570,8 @@ tc_output_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapQ,
             int s = 0, li = 0;
             uint32_t ph = 0;
             bool ok = true;
-            for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
+            for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++li) {
+            const int item = global_item(p, it);
                 const int mb = li & 1;
                 if (!(ok = mbar_wait(&mempty[mb], ((li >> 1) & 1) ^ 1, ab, 0x301))) break;
                 mbar_expect_tx(&mfull[mb], kImg + (RELU ? 512 : 0));
@@ -574,7 +593,8 @@ tc_output_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapQ,
             int s = 0, li = 0, gt = 0;
             uint32_t ph = 0;
             bool ok = true;
-            for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
+            for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++li) {
+            const int item = global_item(p, it);
                 const int mb = li & 1;
                 if (!(ok = mbar_wait(&mfull[mb], (li >> 1) & 1, ab, 0x303))) break;
                 const uint32_t mimg_a = smem_u32(mbuf + mb * kImg);
@@ -602,7 +622,8 @@ tc_output_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapQ,
         const bool issuer = (threadIdx.x == 64);
         int gt = 0;
         bool ok = true;     // every epilogue warp runs every named barrier, even after an abort
-        for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+        for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
+            const int item = global_item(p, it);
             for (int t = 0; t < nt; ++t, ++gt) {
                 const int a = gt % kOAcc, ob = gt & 1;
                 ok = ok && mbar_wait(&accfull[a], (gt / kOAcc) & 1, ab, 0x306);
@@ -642,7 +663,8 @@ tc_output_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapQ,
         int s = 0, li = 0, gt = 0;
         uint32_t ph = 0;
         bool ok = true;
-        for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
+        for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++li) {
+            const int item = global_item(p, it);
             const int mb = li & 1;
             if (!(ok = mbar_wait(&mfull[mb], (li >> 1) & 1, ab, 0x307))) break;
             const float* z = zbuf + mb * 128;
@@ -693,7 +715,7 @@ tc_output_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapQ,
 // Host side
 // ----------------------------------------------------------------------------
 struct WsLayout {
-    size_t gimg, bmat, mimg, dz, zf, total;
+    size_t gimg, bmat, mimg, dz, zf, state, z, total;
 };
 
 WsLayout ws_layout(const ScanArgs& a) {
@@ -713,6 +735,13 @@ WsLayout ws_layout(const ScanArgs& a) {
         L.zf = off;
         off += bhf * 512;
     }
+    // state (and z) carried between the chunk launches of the pipeline
+    const size_t bh = (size_t)a.B * a.H;
+    off = align_up(off, 256);
+    L.state = off;
+    off += bh * a.D * a.D * 4;
+    L.z = off;
+    off += bh * a.D * 4;
     L.total = align_up(off, 256);
     return L;
 }
@@ -736,6 +765,44 @@ int sm_count() {
     return n;
 }
 
+// Frames per pipeline chunk of the three-kernel path: about 8 chunks of at
+// least 16 frames, and whole chunks of the reversed scan; one chunk (no
+// pipeline) for short clips or when the per-head chain CTAs would take more
+// than half of the SMs.
+int tc_chunk(const ScanArgs& a, int nsm) {
+    int c = a.F;
+    if (a.F >= 32 && 2 * a.B * a.H <= nsm) c = std::max(16, (a.F + 7) / 8);
+    if (a.rev_chunk > 0) c = (c + a.rev_chunk - 1) / a.rev_chunk * a.rev_chunk;
+    if (const char* e = std::getenv("LA_TC_CHUNK")) {
+        const int v = std::atoi(e);
+        if (v > 0) c = a.rev_chunk > 0 ? (v + a.rev_chunk - 1) / a.rev_chunk * a.rev_chunk : v;
+    }
+    return std::max(1, std::min(c, std::max(a.F, 1)));
+}
+
+// Streams and events of one device for the chunk pipeline (gram kernels on
+// the caller's stream, chain and output kernels on two streams of the
+// library's own, forked from and joined back to the caller's stream).
+constexpr int kMaxDevicesTc = 64;
+struct TcCtx {
+    bool ready = false;
+    cudaStream_t s_chain = nullptr, s_out = nullptr;
+    cudaEvent_t start = nullptr, gram = nullptr, chain = nullptr, out = nullptr;
+};
+std::mutex g_tc_mu[kMaxDevicesTc];
+TcCtx g_tc_ctx[kMaxDevicesTc];
+
+cudaError_t tc_ctx_init(TcCtx& c) {
+    if (c.ready) return cudaSuccess;
+    cudaError_t e = cudaStreamCreateWithFlags(&c.s_chain, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&c.s_out, cudaStreamNonBlocking);
+    cudaEvent_t* evs[] = {&c.start, &c.gram, &c.chain, &c.out};
+    for (cudaEvent_t* p : evs)
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(p, cudaEventDisableTiming);
+    if (e == cudaSuccess) c.ready = true;
+    return e;
+}
+
 template <bool RELU>
 cudaError_t launch_tc_mode(const ScanArgs& a, cudaStream_t st) {
     const WsLayout L = ws_layout(a);
@@ -743,10 +810,6 @@ cudaError_t launch_tc_mode(const ScanArgs& a, cudaStream_t st) {
     TcParams p;
     p.alpha = a.alpha;
     p.beta = a.beta;
-    p.state_in = a.state_in;
-    p.z_in = a.z_in;
-    p.state_out = a.state_out;
-    p.z_out = a.z_out;
     p.status = reinterpret_cast<unsigned int*>(ws);
     p.gimg = ws + L.gimg;
     p.bmat = reinterpret_cast<float*>(ws + L.bmat);
@@ -786,15 +849,75 @@ cudaError_t launch_tc_mode(const ScanArgs& a, cudaStream_t st) {
         attr_done = true;
     }
     const int nsm = sm_count();
-    const int grid_f = (int)std::min<uint64_t>(bhf, (uint64_t)nsm);
+    const int Fc = tc_chunk(a, nsm);
+    const int nchunks = (p.F + Fc - 1) / Fc;
     const int thr = RELU ? 320 : 192;
-    if (!RELU && p.beta_tok)
-        tc_gram_kernel<false, true><<<grid_f, 320, smem_gram, st>>>(p, mK, mV);
-    else
-        tc_gram_kernel<RELU><<<grid_f, thr, smem_gram, st>>>(p, mK, mV);
-    tc_chain_kernel<RELU><<<p.BH, 192, RELU ? smem_chain_relu : smem_chain_gdn, st>>>(p);
-    if (p.want_output) tc_output_kernel<RELU><<<grid_f, thr, smem_out, st>>>(p, mQ, mO);
-    return cudaGetLastError();
+    float* st_ws = reinterpret_cast<float*>(ws + L.state);
+    float* z_ws = reinterpret_cast<float*>(ws + L.z);
+    auto set_chunk = [&](int ci) {
+        p.f0 = ci * Fc;
+        p.Fc = std::min(Fc, p.F - p.f0);
+        p.state_in = ci == 0 ? a.state_in : st_ws;
+        p.z_in = ci == 0 ? a.z_in : z_ws;
+        p.state_out = ci == nchunks - 1 ? a.state_out : st_ws;
+        p.z_out = ci == nchunks - 1 ? a.z_out : z_ws;
+    };
+    auto gram = [&](int grid, cudaStream_t s) {
+        if (!RELU && p.beta_tok)
+            tc_gram_kernel<false, true><<<grid, 320, smem_gram, s>>>(p, mK, mV);
+        else
+            tc_gram_kernel<RELU><<<grid, thr, smem_gram, s>>>(p, mK, mV);
+    };
+    if (nchunks == 1) {
+        set_chunk(0);
+        const int grid_f = (int)std::min<uint64_t>(bhf, (uint64_t)nsm);
+        gram(grid_f, st);
+        tc_chain_kernel<RELU><<<p.BH, 192, RELU ? smem_chain_relu : smem_chain_gdn, st>>>(p);
+        if (p.want_output) tc_output_kernel<RELU><<<grid_f, thr, smem_out, st>>>(p, mQ, mO);
+        return cudaGetLastError();
+    }
+    // Pipeline: chain(c) (one CTA per head, on its own SMs) runs beside
+    // gram(c + 1) and output(c - 1), which share the other SMs.  Every chunk
+    // writes its own frames of the clip-sized buffers, so only gram -> chain
+    // -> output of the same chunk (and chain -> chain through the carried
+    // state, in stream order) must be ordered.
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevicesTc)
+        return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_tc_mu[dev]);
+    TcCtx& cx = g_tc_ctx[dev];
+    cudaError_t e = tc_ctx_init(cx);
+    if (e != cudaSuccess) return e;
+    const int share = std::max(8, nsm - p.BH);
+    auto ok = [&](cudaError_t x) {
+        if (x != cudaSuccess && e == cudaSuccess) e = x;
+        return e == cudaSuccess;
+    };
+    ok(cudaEventRecord(cx.start, st));
+    ok(cudaStreamWaitEvent(cx.s_chain, cx.start, 0));
+    ok(cudaStreamWaitEvent(cx.s_out, cx.start, 0));
+    for (int ci = 0; ci < nchunks && e == cudaSuccess; ++ci) {
+        set_chunk(ci);
+        const int grid = std::min(p.BH * p.Fc, share);
+        gram(grid, st);
+        ok(cudaGetLastError());
+        ok(cudaEventRecord(cx.gram, st));
+        ok(cudaStreamWaitEvent(cx.s_chain, cx.gram, 0));
+        tc_chain_kernel<RELU><<<p.BH, 192, RELU ? smem_chain_relu : smem_chain_gdn, cx.s_chain>>>(p);
+        ok(cudaGetLastError());
+        ok(cudaEventRecord(cx.chain, cx.s_chain));
+        if (p.want_output) {
+            ok(cudaStreamWaitEvent(cx.s_out, cx.chain, 0));
+            tc_output_kernel<RELU><<<grid, thr, smem_out, cx.s_out>>>(p, mQ, mO);
+            ok(cudaGetLastError());
+        }
+    }
+    // join: the caller's stream continues after the last chain and output
+    cudaError_t j = cudaEventRecord(cx.out, cx.s_out);
+    if (j == cudaSuccess) j = cudaStreamWaitEvent(st, cx.chain, 0);
+    if (j == cudaSuccess) j = cudaStreamWaitEvent(st, cx.out, 0);
+    if (e == cudaSuccess) e = j;
+    return e;
 }
 
 }  // namespace
@@ -805,7 +928,10 @@ bool tc_eligible(const ScanArgs& a) {
 
 size_t tc_workspace_bytes(const ScanArgs& a) { return ws_layout(a).total; }
 
-int tc_kernel_count(const ScanArgs& a) { return a.o ? 3 : 2; }
+int tc_kernel_count(const ScanArgs& a) {
+    const int Fc = tc_chunk(a, sm_count());
+    return (a.o ? 3 : 2) * ((a.F + Fc - 1) / Fc);
+}
 
 cudaError_t launch_tc(const ScanArgs& a, cudaStream_t st) {
     return a.mode == LA_MODE_RELU ? launch_tc_mode<true>(a, st) : launch_tc_mode<false>(a, st);

@@ -108,7 +108,7 @@ def test_reverse_scan_argument_errors_and_sizes():
     # the reversed scan never takes the fused path, so it needs per-frame buffers
     assert la.la_workspace_size(la.LA_MODE_GDN_REVERSE, 1, 20, 181, 880, 128) > \
         la.la_workspace_size(la.LA_MODE_GDN, 1, 20, 181, 880, 128)
-    assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05", 3)
+    assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05", 24)
     assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 1, 16, 512, 1024, 256)[0] == "simt_f32"
     args = lambda C, D=64, w=ws: (P(), P(), P(), P(), la.LA_BF16, P(), P(), 0.1, C,
                                   1, 1, 4, 16, D, P(), w, None)
@@ -125,7 +125,7 @@ def test_token_gate_scan_argument_errors_and_plan():
     P = _fake
     ws = la.la_workspace_size(la.LA_MODE_GDN_TOKEN_BETA, 1, 1, 4, 16, 64)
     assert ws >= 256 and ws % 256 == 0
-    assert la.la_plan(la.LA_MODE_GDN_TOKEN_BETA, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05", 3)
+    assert la.la_plan(la.LA_MODE_GDN_TOKEN_BETA, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05", 24)
     assert la.la_plan(la.LA_MODE_GDN_TOKEN_BETA, la.LA_F32, 1, 2, 8, 64, 32)[0] == "simt_f32"
     assert la.la_workspace_size(4, 1, 1, 4, 16, 64) == 0
     args = lambda bt=P(), D=64, w=ws: (P(), P(), P(), P(), la.LA_BF16, P(), bt, 0.1, None, None,

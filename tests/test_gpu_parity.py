@@ -320,6 +320,32 @@ def test_wide_path_chunking_is_exact(mode, monkeypatch):
     _compare(spec, mode, with_state=True)
 
 
+@pytest.mark.parametrize("mode", ["relu", "gdn"])
+def test_three_kernel_chunk_pipeline_is_exact(mode, monkeypatch):
+    """Long clips on the three-kernel path run as a pipeline of frame chunks
+    (chain beside gram and output, fp32 state carried between chunk
+    launches): any chunk length gives the same bits, and the oracle's values."""
+    spec = synth.small(B=1, H=3, F=40, S=96, D=128, dtype="bf16", seed=71, keys_l2=True)
+    monkeypatch.setenv("LA_SCAN_NO_FUSE", "1")
+    m = la.LA_MODE_GDN if mode == "gdn" else la.LA_MODE_RELU
+    assert la.la_plan(m, la.LA_BF16, 1, 3, 40, 96, 128) == ("tcgen05", 9)   # 3 chunks
+    inp = device_inputs(spec)
+    m0n, z0n = synth.random_state(spec, 0.05)
+    m0, z0 = torch.from_numpy(m0n).cuda(), torch.from_numpy(z0n).cuda()
+    runs = []
+    for chunk in ("7", "16", "40"):
+        monkeypatch.setenv("LA_TC_CHUNK", chunk)
+        runs.append(_run(spec, mode, inp, m0, z0 if mode == "relu" else None))
+    torch.cuda.synchronize()
+    for o, so, zo in runs[1:]:
+        assert torch.equal(o.view(torch.int16), runs[0][0].view(torch.int16))
+        assert torch.equal(so, runs[0][1])
+        if mode == "relu":
+            assert torch.equal(zo, runs[0][2])
+    monkeypatch.delenv("LA_TC_CHUNK")
+    _compare(spec, mode, with_state=True)
+
+
 def test_plan_of_the_workloads():
     assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05_fused", 1)
     assert la.la_plan(la.LA_MODE_RELU, la.LA_BF16, 1, 20, 21, 1560, 112) == ("tcgen05_fused", 1)
