@@ -42,18 +42,18 @@ import numpy as np  # noqa: E402
 import synth  # noqa: E402
 
 WORKLOADS = {
-    # name: (config index, mode)
-    "gdn_720p_60s": (2, "gdn"),
-    "relu_480p": (1, "relu"),
-    "stream_gdn": (3, "gdn"),
-    "stress_gdn": (4, "gdn"),
-    "stress_relu": (4, "relu"),
+    # bench name: (synthetic workload, mode)
+    "gdn_720p_60s": ("gdn_720p_60s", "gdn"),
+    "relu_480p": ("relu_480p", "relu"),
+    "stream_gdn": ("gdn_stream", "gdn"),
+    "stress_gdn": ("stress_d256", "gdn"),
+    "stress_relu": ("stress_d256", "relu"),
     # reversed GDN scan reset every 8 frames, on the 720p 60 s clip
-    "gdn_720p_60s_reverse8": (2, "gdn_reverse"),
+    "gdn_720p_60s_reverse8": ("gdn_720p_60s", "gdn_reverse"),
     # per-token update gate on the 720p 60 s clip
-    "gdn_720p_60s_token_beta": (2, "gdn_token_beta"),
-    "tiny_gdn": (0, "gdn"),
-    "tiny_relu": (0, "relu"),
+    "gdn_720p_60s_token_beta": ("gdn_720p_60s", "gdn_token_beta"),
+    "tiny_gdn": ("tiny_fp32", "gdn"),
+    "tiny_relu": ("tiny_fp32", "relu"),
 }
 DEFAULT_WORKLOAD = "gdn_720p_60s"
 METRIC = "latent frames/s and TFLOP/s of block-causal GDN/ReLU scan; % of B200 roofline"
@@ -263,8 +263,8 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    idx, mode = WORKLOADS[args.workload]
-    spec = synth.config(idx)
+    wname, mode = WORKLOADS[args.workload]
+    spec = synth.workload(wname)
     byts, flops = step_counts(spec, mode)
     for _ in range(args.warmup):
         time_oracle_sample(spec, mode, 0.0, max_heads=1)
@@ -309,8 +309,8 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=dev)
 
-    idx, mode = WORKLOADS[args.workload]
-    base = synth.config(idx)
+    wname, mode = WORKLOADS[args.workload]
+    base = synth.workload(wname)
     if args.frames:
         base = base.with_(F=args.frames, name=f"{base.name}_clip{args.frames}")
     spec = rank_spec(base, rank)   # own data per rank

@@ -87,27 +87,32 @@ class Spec:
         return dataclasses.replace(self, **kw)
 
 
-CONFIGS = {
-    0: Spec("tiny_fp32_B1_H2_D32_F8_S64", B=1, H=2, F=8, S=64, D=32, dtype="f32",
+# The five workloads (seeds are the position in this table).
+WORKLOADS = {
+    "tiny_fp32": Spec("tiny_fp32_B1_H2_D32_F8_S64", B=1, H=2, F=8, S=64, D=32, dtype="f32",
             seed=0, modes=("relu", "gdn"), alpha=("uniform", 0.9, 1.0),
             beta=("uniform", 0.0, 1.0)),
-    1: Spec("relu_480p_B1_H20_D112_F21_S1560", B=1, H=20, F=21, S=1560, D=112,
+    "relu_480p": Spec("relu_480p_B1_H20_D112_F21_S1560", B=1, H=20, F=21, S=1560, D=112,
             dtype="bf16", seed=1, modes=("relu",)),
-    2: Spec("gdn_720p_60s_B1_H20_D128_F181_S880", B=1, H=20, F=181, S=880, D=128,
+    "gdn_720p_60s": Spec("gdn_720p_60s_B1_H20_D128_F181_S880", B=1, H=20, F=181, S=880, D=128,
             dtype="bf16", seed=2, modes=("gdn",), keys_l2=True,
             alpha=("sigmoid_normal", 3.0, 1.0), beta=("sigmoid_normal", 0.0, 1.0)),
-    3: Spec("gdn_stream_B4_H20_D128_8x8frames_S880", B=4, H=20, F=64, S=880, D=128,
+    "gdn_stream": Spec("gdn_stream_B4_H20_D128_8x8frames_S880", B=4, H=20, F=64, S=880, D=128,
             dtype="bf16", seed=3, modes=("gdn",), keys_l2=True,
             alpha=("sigmoid_normal", 3.0, 1.0), beta=("sigmoid_normal", 0.0, 1.0),
             chunk_frames=8),
-    4: Spec("stress_B1_H16_D256_F512_S1024", B=1, H=16, F=512, S=1024, D=256,
+    "stress_d256": Spec("stress_B1_H16_D256_F512_S1024", B=1, H=16, F=512, S=1024, D=256,
             dtype="bf16", seed=4, modes=("relu", "gdn"), outlier_frac=0.01,
             alpha=("uniform", 0.8, 1.0), beta=("uniform", 0.0, 1.0)),
 }
 
 
-def config(idx: int) -> Spec:
-    return CONFIGS[idx]
+WORKLOAD_NAMES = tuple(WORKLOADS)
+
+
+def workload(name: str) -> Spec:
+    """The seeded synthetic workload of this name (see WORKLOADS)."""
+    return WORKLOADS[name]
 
 
 def _rng(*key: int) -> np.random.Generator:

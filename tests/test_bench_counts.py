@@ -1,22 +1,23 @@
 """The benchmark's algorithmic byte and flop counts (fixed formulas, whatever
-the kernels do) reproduce the roofline table of the hot-path survey:
-C1 588.1 MB / 33.17 GF, C2 3.263 GB / 328.3 GF, C3 4.692 GB / 464.4 GF,
-C4 17.184 GB / 2.208 TF (ReLU) and 3.573 TF (GDN)."""
+the kernels do), checked against values worked out by hand from the
+workload shapes: 480p ReLU 588.1 MB / 33.17 GF, 720p 60 s GDN 3.263 GB /
+328.3 GF, streaming GDN 4.692 GB / 464.4 GF, D = 256 stress 17.184 GB /
+2.208 TF (ReLU) and 3.573 TF (GDN)."""
 import pytest
 
 import bench
 import synth
 
 
-@pytest.mark.parametrize("idx,mode,gbytes,gflop", [
-    (1, "relu", 0.5881, 33.17),
-    (2, "gdn", 3.263, 328.3),
-    (3, "gdn", 4.692, 464.4),
-    (4, "relu", 17.184, 2208.0),
-    (4, "gdn", 17.184, 3573.0),
+@pytest.mark.parametrize("name,mode,gbytes,gflop", [
+    ("relu_480p", "relu", 0.5881, 33.17),
+    ("gdn_720p_60s", "gdn", 3.263, 328.3),
+    ("gdn_stream", "gdn", 4.692, 464.4),
+    ("stress_d256", "relu", 17.184, 2208.0),
+    ("stress_d256", "gdn", 17.184, 3573.0),
 ])
-def test_step_counts_match_the_roofline_table(idx, mode, gbytes, gflop):
-    b, f = bench.step_counts(synth.config(idx), mode)
+def test_step_counts_match_hand_worked_values(name, mode, gbytes, gflop):
+    b, f = bench.step_counts(synth.workload(name), mode)
     assert abs(b / 1e9 - gbytes) / gbytes < 1e-3
     assert abs(f / 1e9 - gflop) / gflop < 1e-3
 
@@ -38,6 +39,6 @@ def test_frame_counts_by_hand():
 
 
 def test_streaming_plan_passes_the_state_between_chunks():
-    plan = bench.step_plan(synth.config(3), "gdn")
+    plan = bench.step_plan(synth.workload("gdn_stream"), "gdn")
     assert plan == [(8 * c, 8, c > 0) for c in range(8)]
-    assert bench.step_plan(synth.config(2), "gdn") == [(0, 181, False)]
+    assert bench.step_plan(synth.workload("gdn_720p_60s"), "gdn") == [(0, 181, False)]

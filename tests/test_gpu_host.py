@@ -162,7 +162,7 @@ def test_host_scan_pageable_memory():
 def test_host_scan_full_720p_gdn_sampled_heads():
     """The 720p 60 s GDN workload (B1 H20 D128 F181 S880) through the host
     path with the automatic chunking the end-to-end benchmark uses."""
-    spec = synth.config(2)
+    spec = synth.workload("gdn_720p_60s")
     inp = _host_inputs(spec)
     o, so, _ = _host_scan(spec, "gdn", inp, 0)
     assert la.la_host_chunk_frames(spec.F, 0) == 12

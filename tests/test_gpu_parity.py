@@ -93,29 +93,29 @@ def _compare(spec, mode, heads=None, with_state=False):
 # ----------------------------------------------------------------------------
 @pytest.mark.parametrize("mode", ["relu", "gdn"])
 def test_tiny_fp32_config(mode):
-    _compare(synth.config(0), mode)
+    _compare(synth.workload("tiny_fp32"), mode)
 
 
 @pytest.mark.parametrize("mode", ["relu", "gdn"])
 def test_tiny_fp32_config_with_state_in(mode):
-    _compare(synth.config(0), mode, with_state=True)
+    _compare(synth.workload("tiny_fp32"), mode, with_state=True)
 
 
 def test_relu_480p_all_heads():
-    _compare(synth.config(1), "relu")
+    _compare(synth.workload("relu_480p"), "relu")
 
 
 def test_gdn_720p_60s_all_heads():
-    _compare(synth.config(2), "gdn")
+    _compare(synth.workload("gdn_720p_60s"), "gdn")
 
 
 @pytest.mark.parametrize("mode", ["relu", "gdn"])
 def test_stress_d256_sampled_heads(mode):
-    _compare(synth.config(4), mode, heads=[(0, 0), (0, 11)])
+    _compare(synth.workload("stress_d256"), mode, heads=[(0, 0), (0, 11)])
 
 
 def test_streaming_chunks_equal_single_scan():
-    spec = synth.config(3)
+    spec = synth.workload("gdn_stream")
     inp = device_inputs(spec)
     B, H, F, D, C = spec.B, spec.H, spec.F, spec.D, spec.chunk_frames
     whole, m_whole, _ = _run(spec, "gdn", inp)

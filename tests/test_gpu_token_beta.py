@@ -71,7 +71,7 @@ def test_token_gate_scan_matches_oracle(dtype, D, S, F):
 
 def test_token_gate_scan_720p_gdn_sampled_heads():
     """The 720p 60 s GDN workload with one update gate per token."""
-    spec = synth.config(2)
+    spec = synth.workload("gdn_720p_60s")
     # eight pipeline chunks of 23 frames, three kernels each
     assert la.la_plan(la.LA_MODE_GDN_TOKEN_BETA, la.LA_BF16, 1, 20, 181, 880, 128) == \
         ("tcgen05", 24)

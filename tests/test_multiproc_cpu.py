@@ -30,7 +30,7 @@ def _worker(rank, world, port, q):
     dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
                             world_size=world, timeout=datetime.timedelta(seconds=60))
     t = bench.max_over_ranks(0.5 + rank, device="cpu")
-    spec = bench.rank_spec(synth.config(2), rank)
+    spec = bench.rank_spec(synth.workload("gdn_720p_60s"), rank)
     first = synth.slice_storage(spec.with_(F=1, H=1), "q", 0, 0).tobytes()[:64]
     q.put((rank, t, spec.seed, first))
     dist.barrier()

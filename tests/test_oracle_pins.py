@@ -85,7 +85,7 @@ def _relu_unrolled(q, k, v, eps, m0=None, z0=None):
 
 
 def test_relu_matches_unrolled_attention_tiny_config():
-    spec = synth.config(0)
+    spec = synth.workload("tiny_fp32")
     q, k, v, _, _ = _inputs(spec)
     o, _, _ = oracle.relu_scan(q, k, v, spec.eps)
     ref = _relu_unrolled(q, k, v, spec.eps)
@@ -164,7 +164,7 @@ def _gdn_unrolled(q, k, v, alpha, beta, kappa, m0=None):
 
 
 def test_gdn_matches_unrolled_product_tiny_config():
-    spec = synth.config(0)
+    spec = synth.workload("tiny_fp32")
     q, k, v, a, bt = _inputs(spec)
     o, _ = oracle.gdn_scan(q, k, v, a, bt, spec.k_scale)
     ref = _gdn_unrolled(q, k, v, a, bt, spec.k_scale)
@@ -254,7 +254,7 @@ def test_gdn_delta_rule_retrieval_with_orthonormal_keys(alpha, beta):
 # Additive limit: GDN with alpha = 1, beta = delta, V / delta -> linear-attention cumsum
 # ----------------------------------------------------------------------------
 def test_gdn_additive_limit_is_linear_attention_cumsum():
-    spec = synth.config(0)
+    spec = synth.workload("tiny_fp32")
     q, k, v, _, _ = _inputs(spec)
     q, k, v = q[:, :1], k[:, :1], v[:, :1]
     kap = spec.k_scale
@@ -283,9 +283,9 @@ def test_gdn_additive_limit_is_linear_attention_cumsum():
 @pytest.mark.parametrize("cfg", [0, "c2_like"])
 def test_key_scaling_bounds_transition_norm(cfg):
     if cfg == "c2_like":
-        spec = synth.config(2).with_(B=1, H=2, F=6)   # same shape and recipe, fewer frames
+        spec = synth.workload("gdn_720p_60s").with_(B=1, H=2, F=6)   # same shape and recipe, fewer frames
     else:
-        spec = synth.config(0)
+        spec = synth.workload("tiny_fp32")
     k = synth.full_values(spec, "k").astype(np.float64)
     _, bt = synth.gates(spec)
     kap = spec.k_scale
@@ -304,7 +304,7 @@ def test_key_scaling_bounds_transition_norm(cfg):
 
 
 def test_gdn_scan_is_a_contraction_in_the_initial_state():
-    spec = synth.config(0)
+    spec = synth.workload("tiny_fp32")
     q, k, v, a, bt = _inputs(spec)
     m0, _ = synth.random_state(spec)
     m1 = m0 + synth.random_state(spec.with_(seed=99))[0]
@@ -321,7 +321,7 @@ def test_gdn_scan_is_a_contraction_in_the_initial_state():
 # Chunked vs whole, and the composite route of context-parallel training
 # ----------------------------------------------------------------------------
 def test_chunked_equals_whole_bitwise():
-    spec = synth.config(0)
+    spec = synth.workload("tiny_fp32")
     q, k, v, a, bt = _inputs(spec)
     o, m = oracle.gdn_scan(q, k, v, a, bt, spec.k_scale)
     o1, m1 = oracle.gdn_scan(q[:, :, :3], k[:, :, :3], v[:, :, :3], a[:, :, :3], bt[:, :, :3],
@@ -339,7 +339,7 @@ def test_chunked_equals_whole_bitwise():
 
 
 def test_state_step_matches_scan_state():
-    spec = synth.config(0)
+    spec = synth.workload("tiny_fp32")
     q, k, v, a, bt = _inputs(spec)
     m0, z0 = synth.random_state(spec)
     _, m = oracle.gdn_scan(q, k, v, a, bt, spec.k_scale, m0)
@@ -351,7 +351,7 @@ def test_state_step_matches_scan_state():
 
 
 def test_composite_exclusive_prefix_recovers_interval_states():
-    spec = synth.config(0)
+    spec = synth.workload("tiny_fp32")
     q, k, v, a, bt = _inputs(spec)
     m0, _ = synth.random_state(spec)
     cuts = [0, 2, 3, 6, 8]
@@ -419,7 +419,7 @@ def _gdn_pins_pass(scan):
                  g["k_scale"])
         if np.max(np.abs(o[0, 0] - np.array(g["expected_o"]))) > 1e-12:
             return False
-        spec = synth.config(0)
+        spec = synth.workload("tiny_fp32")
         q, k, v, a, bt = _inputs(spec)
         o = scan(q, k, v, a, bt, spec.k_scale)
         if _rel(o, _gdn_unrolled(q, k, v, a, bt, spec.k_scale)) > 1e-12:

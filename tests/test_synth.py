@@ -37,7 +37,7 @@ def test_slices_are_regenerable_and_deterministic():
 
 
 def test_fp32_config_is_plain_normal():
-    spec = synth.config(0)
+    spec = synth.workload("tiny_fp32")
     q = synth.full_storage(spec, "q")
     assert q.dtype == np.float32 and q.shape == (1, 2, 8, 64, 32)
     assert abs(q.mean()) < 0.05 and abs(q.std() - 1) < 0.05
@@ -48,7 +48,7 @@ def test_fp32_config_is_plain_normal():
 
 
 def test_l2_normalised_keys_recipe():
-    spec = synth.config(2).with_(H=1, F=3)
+    spec = synth.workload("gdn_720p_60s").with_(H=1, F=3)
     k = synth.slice_values(spec, "k", 0, 0).astype(np.float64)
     n = np.linalg.norm(k, axis=-1)
     assert np.all(np.abs(n - 1) < 4e-3)          # unit norm up to bf16 rounding
@@ -58,7 +58,7 @@ def test_l2_normalised_keys_recipe():
 
 
 def test_outlier_tokens_recipe():
-    spec = synth.config(4).with_(F=4, S=256, D=32, H=2)
+    spec = synth.workload("stress_d256").with_(F=4, S=256, D=32, H=2)
     rows = synth.outlier_rows(spec, 0)
     assert rows.size == round(0.01 * 4 * 256) and len(np.unique(rows)) == rows.size
     q0 = synth.slice_values(spec, "q", 0, 0).reshape(-1, 32)
@@ -71,6 +71,6 @@ def test_outlier_tokens_recipe():
 
 
 def test_config_table_shapes():
-    assert [synth.config(i).D for i in range(5)] == [32, 112, 128, 128, 256]
-    assert synth.config(1).S == 30 * 52 and synth.config(2).S == 22 * 40
-    assert synth.config(3).chunk_frames * 8 == synth.config(3).F
+    assert [synth.workload(n).D for n in synth.WORKLOAD_NAMES] == [32, 112, 128, 128, 256]
+    assert synth.workload("relu_480p").S == 30 * 52 and synth.workload("gdn_720p_60s").S == 22 * 40
+    assert synth.workload("gdn_stream").chunk_frames * 8 == synth.workload("gdn_stream").F
