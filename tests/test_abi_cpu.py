@@ -190,3 +190,27 @@ def test_python_binding_refuses_cpu_tensors():
     a = torch.ones(1, 1, 1)
     with pytest.raises(ValueError):
         la.la_scan_gdn(x, x, x, a, a, 0.1, workspace=torch.zeros(1024, dtype=torch.uint8))
+
+
+@pytest.mark.parametrize("F,chunks", [(8, 1), (31, 1), (32, 2), (40, 3), (181, 8), (512, 8)])
+def test_three_kernel_path_chunk_count(F, chunks):
+    """Clips of 32+ frames with few heads run as a pipeline of frame chunks of
+    max(16, ceil(F / 8)) frames, three kernels per chunk (two without output)."""
+    assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 1, 4, F, 64, 128) == ("tcgen05", 3 * chunks)
+
+
+def test_three_kernel_pipeline_needs_free_sms():
+    # 80 heads would hold more than half of the SMs with chain CTAs: one chunk
+    assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 4, 20, 64, 880, 128) == ("tcgen05", 3)
+
+
+def test_reversed_scan_chunks_align_with_pipeline_chunks():
+    # F = 181 -> pipeline chunks of 23 frames, rounded up to whole 8-frame reversed
+    # chunks (24 frames): 8 launches of three kernels
+    assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05", 24)
+
+
+@pytest.mark.parametrize("F,chunks", [(2, 1), (4, 1), (6, 2), (21, 6), (64, 8), (512, 8)])
+def test_wide_path_chunk_count(F, chunks):
+    """Wide heads run in chunks of max(4, ceil(F / 8)) frames."""
+    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 2, F, 64, 256) == ("tcgen05_wide", 3 * chunks)

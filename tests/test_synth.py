@@ -74,3 +74,15 @@ def test_config_table_shapes():
     assert [synth.workload(n).D for n in synth.WORKLOAD_NAMES] == [32, 112, 128, 128, 256]
     assert synth.workload("relu_480p").S == 30 * 52 and synth.workload("gdn_720p_60s").S == 22 * 40
     assert synth.workload("gdn_stream").chunk_frames * 8 == synth.workload("gdn_stream").F
+
+
+def test_token_gates_are_seeded_per_workload_and_follow_the_beta_recipe():
+    spec = synth.small(B=1, H=2, F=3, S=50, D=32, seed=5, beta=("sigmoid_normal", 0.0, 1.0))
+    a = synth.token_gates(spec)
+    assert a.shape == (1, 2, 3, 50) and a.dtype == np.float32
+    np.testing.assert_array_equal(a, synth.token_gates(spec))            # reproducible
+    assert not np.array_equal(a, synth.token_gates(spec.with_(seed=6)))  # seed matters
+    assert (a > 0).all() and (a < 1).all()                              # sigmoid of a normal
+    # independent of the per-frame gates drawn for the same workload
+    _, bt = synth.gates(spec)
+    assert not np.allclose(a[..., 0], bt)
