@@ -259,6 +259,12 @@ def time_oracle_sample(spec, mode, budget_s: float, max_heads=None):
     return frames / t_total, t_total, sample
 
 
+def workload_label(spec_name: str, mode: str) -> str:
+    """config.workload of a JSON line: the workload's name, plus the variant."""
+    return spec_name + {"gdn_reverse": f"_reverse{REVERSE_CHUNK}",
+                        "gdn_token_beta": "_token_beta"}.get(mode, "")
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -280,7 +286,8 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * ts / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy PCG64)",
-        "config": {"workload": spec.name, "mode": mode, "B": spec.B, "H": spec.H, "F": spec.F,
+        "config": {"workload": workload_label(spec.name, mode), "mode": mode, "B": spec.B,
+                   "H": spec.H, "F": spec.F,
                    "S": spec.S, "D": spec.D},
         "cpu_baseline": {"value": value, "unit": "latent frames/s", "cores": cores,
                          "kind": "oracle", "sample": sample},
@@ -512,8 +519,7 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if spec.dtype == "bf16" else "f32",
         "data": "synthetic (seeded numpy PCG64, bf16 round-to-nearest-even)",
-        "config": {"workload": base.name + {"gdn_reverse": f"_reverse{REVERSE_CHUNK}",
-                                            "gdn_token_beta": "_token_beta"}.get(mode, ""),
+        "config": {"workload": workload_label(base.name, mode),
                    "mode": mode, "B": B, "H": H, "F": F, "S": S, "D": D,
                    "calls_per_step": len(plan), "global_batch": B * world,
                    "l2": "inputs larger than L2 (no flush)",

@@ -1,0 +1,54 @@
+"""The benchmark's command line on a machine without a GPU: the reference
+arm (the CPU oracle) prints one JSON line with the fields the benchmark
+contract asks for, labelled like the GPU arm's line of the same workload."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+import bench
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _run(*args):
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    return json.loads(out.stdout.strip().splitlines()[-1])
+
+
+@pytest.mark.parametrize("workload", ["tiny_gdn", "tiny_relu"])
+def test_reference_arm_prints_the_contract_line(workload):
+    d = _run("--impl", "reference", "--workload", workload, "--steps", "2", "--warmup", "1")
+    assert d["impl"] == "reference"
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["metric"] == bench.METRIC and d["unit"] == "latent frames/s"
+    assert d["higher_is_better"] is True and d["n_gpus"] == 1 and d["steps"] == 2
+    assert d["value"] > 0 and d["vs_baseline"] is None
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
+    assert "oracle on" in cb["sample"]
+    e = d["e2e"]
+    assert e["value"] == d["value"] and e["unit"] == d["unit"]
+    assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
+    assert d["config"]["workload"] == "tiny_fp32_B1_H2_D32_F8_S64"
+
+
+def test_workload_labels_of_the_variants():
+    assert bench.workload_label("gdn_720p_60s_B1", "gdn") == "gdn_720p_60s_B1"
+    assert bench.workload_label("gdn_720p_60s_B1", "gdn_reverse") == "gdn_720p_60s_B1_reverse8"
+    assert bench.workload_label("gdn_720p_60s_B1", "gdn_token_beta") == "gdn_720p_60s_B1_token_beta"
+
+
+def test_every_bench_workload_names_a_synthetic_workload():
+    import synth
+    for name, (wname, mode) in bench.WORKLOADS.items():
+        spec = synth.workload(wname)
+        assert mode in ("relu", "gdn", "gdn_reverse", "gdn_token_beta"), name
+        assert spec.F > 0 and spec.S > 0
