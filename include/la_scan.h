@@ -30,7 +30,8 @@
  *              are rounded to nearest even).  The state, the normaliser and
  *              all accumulation are float32.
  * Memory.      Every pointer is a device pointer of the current device (or
- *              managed memory), 16-byte aligned.  The caller owns all
+ *              managed memory), 16-byte aligned (la_scan_host takes host
+ *              pointers instead; see there).  The caller owns all
  *              buffers, including the workspace; the library never
  *              allocates, frees or synchronises (except
  *              la_query_device_status, which synchronises on purpose).
@@ -39,13 +40,15 @@
  *              LA_ERR_CUDA.  Device-side waits are bounded: a wait that
  *              gives up records LA_ERR_TIMEOUT in the workspace, which
  *              la_query_device_status reports.
- * Streams.     Wide heads (bf16, D > 128) pipeline frame chunks over two
+ * Streams.     Wide heads (bf16, D > 128) and the three-kernel path on
+ *              clips of 32 or more frames pipeline frame chunks over two
  *              streams of the library's own, forked from `stream` (after the
  *              work already queued on it) and joined back to it, so the call
- *              is still ordered on `stream` as a whole.  The first such call
- *              on a device creates those streams and a few events and keeps
- *              them until the process exits; calls on one device serialise
- *              their enqueueing on a lock.
+ *              is still ordered on `stream` as a whole (and can be captured
+ *              into a CUDA graph).  The first such call on a device creates
+ *              those streams and a few events and keeps them until the
+ *              process exits; calls on one device serialise their
+ *              enqueueing on a lock.
  * Aliasing.    state_in == state_out (and z_in == z_out) is allowed (in
  *              place).  o must not overlap q, k or v.
  * NULL state.  state_in == NULL (z_in == NULL) means a zero initial state;
