@@ -620,3 +620,25 @@ def test_token_gate_pins_reject_planted_mistakes(kind):
                 M = a[b, h, f] * (M - kh.T @ (ew * (kh @ M))) + kh.T @ (ww * v[b, h, f])
                 o[b, h, f] = q[b, h, f] @ M
     assert _rel(o, ref) > 1e-3
+
+
+# ----------------------------------------------------------------------------
+# Hand-worked fixtures of the reversed scan and the per-token gate
+# ----------------------------------------------------------------------------
+def test_golden_token_gate_hand_example():
+    g = json.load(open(os.path.join(GOLDEN, "gdn_token_gate_hand_2x2.json")))
+    arr = lambda x: np.array(x, float)[None, None]
+    o, m = oracle.gdn_scan_token_beta(arr(g["q"]), arr(g["k"]), arr(g["v"]), arr(g["alpha"]),
+                                      arr(g["beta_token"]), g["k_scale"])
+    np.testing.assert_allclose(o[0, 0], np.array(g["expected_o"], float), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(m[0, 0], np.array(g["expected_state"], float), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("chunk", [1, 2])
+def test_golden_reverse_hand_example(chunk):
+    g = json.load(open(os.path.join(GOLDEN, "gdn_reverse_hand_2x2.json")))
+    arr = lambda x: np.array(x, float)[None, None]
+    o = oracle.gdn_scan_reverse_chunked(arr(g["q"]), arr(g["k"]), arr(g["v"]), arr(g["alpha"]),
+                                        arr(g["beta"]), g["k_scale"], chunk)
+    np.testing.assert_allclose(o[0, 0], np.array(g[f"expected_o_chunk{chunk}"], float),
+                               rtol=0, atol=1e-12)
