@@ -22,6 +22,18 @@
 // exchanges (appendix C.1) -- and the block-causal ReLU linear attention of
 // the SANA-Video talk (block KV cache segment).
 //
+// Variants.  The reversed GDN scan reset at chunk boundaries (SANA-WM paper
+// summary, section 3, "Chunk-causal deployment") changes only the chain:
+// its frame order and a zero state at each chunk start.  The per-token
+// update gate (section 3, "Hybrid GDN/Softmax Attention") changes only the
+// gram: each token row of K and V is scaled by sqrt(beta_t) before the
+// contractions, which then give Kh^T diag(beta) Kh and Kh^T diag(beta) V.
+//
+// Pipeline.  Clips of 32+ frames with few enough heads run as chunks of
+// frames: chain(c) on its own SMs beside gram(c + 1) and output(c - 1), on
+// streams forked from and joined to the caller's, with the fp32 state
+// carried between the chunk launches.
+//
 // Layouts.  q, k, v, o are viewed by TMA as [B*H*F][S][D] bf16 with a 64-wide
 // (128-byte) swizzled box; out-of-range tokens and columns read as zero.
 // Operand images in the workspace are byte-exact shared-memory images
