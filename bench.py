@@ -16,9 +16,10 @@ step) are far larger than the 126 MB L2, so no L2 flush is needed between
 steps.
 
 --impl reference times the CPU oracle on the host cores instead (a bounded
-sample of the same workload each step).  N > 1 (torchrun) runs the
-workload once per rank on its own data, no collective on the data path
-(weak scaling); the reported time is the max over ranks.
+sample of the same workload each step).  N > 1 runs the workload once per
+rank on its own data, no collective on the data path (weak scaling); the
+reported time is the max over ranks.  Under torchrun the ranks come from
+the environment; `--gpus N` without torchrun launches N ranks itself.
 """
 from __future__ import annotations
 
@@ -174,8 +175,8 @@ class ClockSampler:
         0x100: "display_clock_setting",
     }
 
-    def __init__(self, index: int, period_s: float = 0.01):
-        self.samples, self.reasons, self.max_mhz = [], 0, None
+    def __init__(self, index: int, period_s: float = 0.001):
+        self.samples, self.stamps, self.reasons, self.max_mhz = [], [], 0, None
         self.period = period_s
         self._stop = threading.Event()
         self._thr = None
@@ -192,8 +193,10 @@ class ClockSampler:
     def _run(self):
         while not self._stop.is_set():
             try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
                 self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append(mhz)
+                self.stamps.append(time.perf_counter())
             except Exception:
                 pass
             time.sleep(self.period)
@@ -207,6 +210,10 @@ class ClockSampler:
         if self._thr:
             self._stop.set()
             self._thr.join()
+
+    def between(self, t0: float, t1: float):
+        """SM clock samples taken between host times t0 and t1."""
+        return [m for m, t in zip(self.samples, self.stamps) if t0 <= t <= t1]
 
     def summary(self):
         if not self.nv:
@@ -267,6 +274,7 @@ def workload_label(spec_name: str, mode: str) -> str:
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return 0
     wname, mode = WORKLOADS[args.workload]
@@ -283,7 +291,7 @@ def run_reference(args):
     cores = oracle_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "latent frames/s",
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * ts / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy PCG64)",
         "config": {"workload": workload_label(spec.name, mode), "mode": mode, "B": spec.B,
@@ -419,6 +427,31 @@ def run_ours(args):
     call_ms = [s.elapsed_time(e) / len(plan) for s, e in evs]
     t_max = max_over_ranks(t_local, dev)
 
+    # ---- optional: sustained back-to-back calls, binned by block, beside the
+    # SM clock sampled during each block (does a slowdown track the clock?) ----
+    drift = None
+    if args.drift_blocks > 0:
+        dclk = ClockSampler(local)
+        dclk.start()
+        drift = []
+        for blk in range(args.drift_blocks):
+            d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            h0 = time.perf_counter()
+            d0.record(stream)
+            for _ in range(args.drift_calls):
+                one_step()
+            d1.record(stream)
+            d1.synchronize()
+            h1 = time.perf_counter()
+            ms = d0.elapsed_time(d1) / (args.drift_calls * len(plan))
+            mhz = dclk.between(h0, h1)
+            med = statistics.median(mhz) if mhz else None
+            drift.append({"block": blk, "calls": args.drift_calls, "ms_per_call": ms,
+                          "sm_mhz_median": med, "sm_mhz_min": min(mhz) if mhz else None,
+                          "samples": len(mhz), "ms_x_ghz": ms * med / 1e3 if med else None})
+        dclk.stop()
+        barrier()
+
     byts, flops = step_counts(spec, mode)
     frames_all = B * F * K * world
     value = frames_all / t_max
@@ -536,12 +569,31 @@ def run_ours(args):
         "clocks": clocks.summary(),
         "device_status": la.la_status_string(status),
     }
+    if drift is not None:
+        line["drift"] = drift
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def free_port() -> int:
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def relaunch_ranks(n: int) -> int:
+    """Run this same command as n ranks (one process per GPU) under torchrun
+    on this node; rank 0 prints the JSON line.  Returns torchrun's status."""
+    import subprocess
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr=127.0.0.1", f"--master-port={free_port()}",
+           os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
 
 
 def main():
@@ -558,7 +610,19 @@ def main():
                     help="skip the host-buffer end-to-end leg (profiling runs)")
     ap.add_argument("--frames", type=int, default=0,
                     help="profiling only: a shorter clip (this many latent frames) of the workload")
+    ap.add_argument("--drift-blocks", type=int, default=0,
+                    help="analysis: after the timed steps, run this many blocks of back-to-back "
+                         "calls and report each block's ms per call beside the SM clock "
+                         "sampled during it")
+    ap.add_argument("--drift-calls", type=int, default=50, help="calls per drift block")
     args = ap.parse_args()
+    # N ranks, one per GPU: launched here unless torchrun already did
+    world_env = os.environ.get("WORLD_SIZE")
+    if world_env is None and args.gpus > 1:
+        return relaunch_ranks(args.gpus)
+    if int(world_env or 1) != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world_env}", file=sys.stderr)
+        return 2
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":

@@ -219,11 +219,18 @@ LA_API la_status la_state_step(la_mode mode, const void* k, const void* v, la_dt
  * Scratch.  A __device__ array of LA_NOALLOC_SCRATCH_BYTES (64 MiB) that
  *   every GPU which loads the library holds until the process exits.  A call
  *   whose la_workspace_size(LA_MODE_GDN, B, H, F, S, D) exceeds it returns
- *   LA_ERR_UNSUPPORTED before enqueuing anything (for bf16 inputs with
- *   64 <= D <= 128 the scan needs about 1 MiB per (b, h) pair, so up to
- *   B*H = 63; float32 inputs and D < 64 need only a few bytes; bf16 inputs
- *   with D > 128 need per-frame buffers of about 0.4 MiB per (b, h, frame)
- *   of a pipeline chunk, so only short clips of few heads fit).
+ *   LA_ERR_UNSUPPORTED before enqueuing anything.  What fits (la_workspace_size
+ *   is the exact test):
+ *     - bf16 inputs, 64 <= D <= 128, B*H <= 49 (on a 148-SM B200: the
+ *       single-kernel path): about 1.5 MiB per (b, h) pair whatever F is,
+ *       so B*H <= 42;
+ *     - bf16 inputs, 64 <= D <= 128, more pairs (the three-kernel path):
+ *       per-frame buffers of 128 KiB per (b, h, frame) plus the state
+ *       (64 KiB per pair at D = 128), so about B*H*F <= 480 at D = 128
+ *       (for example B*H = 63 with F <= 7);
+ *     - bf16 inputs, 128 < D <= 256: per-frame buffers of about 0.4 MiB per
+ *       (b, h, frame of a pipeline chunk), so only short clips of few heads;
+ *     - float32 inputs, or D < 64: a few hundred bytes.
  * Sharing.  All calls on a device share the one array, and it keeps the
  *   last call's contents; the library clears what must start at zero at the
  *   start of every call.  Calls whose GPU work overlaps (on different
@@ -232,15 +239,23 @@ LA_API la_status la_state_step(la_mode mode, const void* k, const void* v, la_dt
  * Set-up.  The first call on each device looks up the array's device
  *   address (cudaGetSymbolAddress) with that device current; make that first
  *   call before any stream capture begins.
- * Status.  la_query_device_status is not available for this entry point
- *   (the caller has no workspace pointer); device-side timeouts surface as
- *   invalid outputs only.
+ * Status.  A bounded device-side wait that gives up records LA_ERR_TIMEOUT in
+ *   the array, and the outputs of that call are then not valid;
+ *   la_query_noalloc_status reads it back.
  */
 #define LA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 LA_API la_status la_scan_gdn_noalloc(const void* q, const void* k, const void* v, void* o,
                                      la_dtype dt, const float* alpha, const float* beta,
                                      float k_scale, const float* state_in, float* state_out,
                                      int B, int H, int F, int S, int D, cudaStream_t stream);
+
+/* Synchronise `stream`, then report the device-side status that the most
+ * recent la_scan_gdn_noalloc call on the current device recorded in the
+ * built-in scratch array: LA_OK, or LA_ERR_TIMEOUT when a bounded wait gave
+ * up (that call's outputs are then not valid).  Returns LA_ERR_CUDA if the
+ * synchronisation fails.  Like la_query_device_status, it synchronises on
+ * purpose.  No counterpart in the pages. */
+LA_API la_status la_query_noalloc_status(cudaStream_t stream);
 
 /*
  * The scan of a clip held in HOST memory, streamed through the GPU in chunks

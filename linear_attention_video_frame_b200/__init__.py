@@ -25,7 +25,7 @@ __all__ = [
     "LA_MODE_GDN_TOKEN_BETA",
     "la_scan_relu", "la_scan_gdn", "la_state_step", "la_workspace_size",
     "la_query_device_status", "la_status_string", "la_plan", "workspace_for",
-    "la_scan_gdn_noalloc", "LA_NOALLOC_SCRATCH_BYTES", "la_scan_host",
+    "la_scan_gdn_noalloc", "la_query_noalloc_status", "LA_NOALLOC_SCRATCH_BYTES", "la_scan_host",
     "la_host_workspace_size", "la_host_chunk_frames", "host_workspace_for",
 ]
 
@@ -66,6 +66,8 @@ def _load() -> ctypes.CDLL:
     L.la_scan_gdn_reverse.restype = I
     L.la_scan_gdn_noalloc.argtypes = [P, P, P, P, I, P, P, F, P, P, I, I, I, I, I, P]
     L.la_scan_gdn_noalloc.restype = I
+    L.la_query_noalloc_status.argtypes = [P]
+    L.la_query_noalloc_status.restype = I
     L.la_plan.argtypes = [I, I, I, I, I, I, I, ctypes.POINTER(ctypes.c_int)]
     L.la_plan.restype = ctypes.c_char_p
     L.la_scan_host.argtypes = [I, P, P, P, P, I, P, P, F, F, P, P, P, P,
@@ -268,6 +270,11 @@ def la_state_step(mode: int, k, v, alpha=None, beta=None, k_scale: float = 1.0,
 
 def la_query_device_status(workspace, stream=None) -> int:
     return int(lib.la_query_device_status(_ptr(workspace), _stream(stream)))
+
+
+def la_query_noalloc_status(stream=None) -> int:
+    """Status the last la_scan_gdn_noalloc call on the current device recorded."""
+    return int(lib.la_query_noalloc_status(_stream(stream)))
 
 
 def la_host_workspace_size(mode: int, dt: int, B: int, H: int, F: int, S: int, D: int,

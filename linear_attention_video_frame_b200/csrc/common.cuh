@@ -69,6 +69,15 @@ __device__ __forceinline__ void store_elem(void* p, size_t i, float x, int bf16)
     else reinterpret_cast<float*>(p)[i] = x;
 }
 
+// Per-device facts (devinfo.cu).  A process may drive several GPUs, so
+// everything that belongs to a device is cached per device.
+constexpr int kDefaultSmCount = 148;   // B200; used only when no device is visible
+int current_device();                   // current device, or -1
+int device_sm_count();                  // SMs of the current device (cached per device)
+// Opt `kernel` in to `bytes` of dynamic shared memory on the current device
+// (once per device and kernel); returns the CUDA error of the first failure.
+cudaError_t ensure_dyn_smem(const void* kernel, int bytes);
+
 // Launchers (host side), each returns cudaGetLastError() of its launches.
 cudaError_t launch_simt(const ScanArgs& a, cudaStream_t st);
 size_t simt_workspace_bytes(const ScanArgs& a);

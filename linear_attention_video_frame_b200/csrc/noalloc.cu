@@ -65,3 +65,13 @@ extern "C" la_status la_scan_gdn_noalloc(const void* q, const void* k, const voi
     return la_scan_gdn(q, k, v, o, dt, alpha, beta, k_scale, state_in, state_out, B, H, F, S, D,
                        scratch, (size_t)LA_NOALLOC_SCRATCH_BYTES, stream);
 }
+
+// The status word lives in the first bytes of the scratch array, exactly as
+// it does in a caller's workspace, so the workspace query reads it once the
+// array's device address is known.
+extern "C" la_status la_query_noalloc_status(cudaStream_t stream) {
+    void* scratch = nullptr;
+    const la_status s = scratch_of_current_device(&scratch);
+    if (s != LA_OK) return s;
+    return la_query_device_status(scratch, stream);
+}

@@ -1008,17 +1008,6 @@ constexpr size_t kChainSmem = kCStages * 2 * kImg + 2 * kImg + 1024 + 8 + 12 * 8
 constexpr size_t kFusedSmem = 1024 + (kWorkerSmem > kChainSmem ? kWorkerSmem : kChainSmem);
 static_assert(kFusedSmem <= 232448, "fused kernel shared memory");
 
-int sm_count_fused() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
-}
-
 template <bool RELU>
 cudaError_t launch_fused_mode(const ScanArgs& a, cudaStream_t st) {
     const FusedLayout L = fused_layout(a);
@@ -1050,7 +1039,7 @@ cudaError_t launch_fused_mode(const ScanArgs& a, cudaStream_t st) {
     if (const char* e = std::getenv("LA_SCAN_LAG")) p.lag = std::max(1, std::min(std::atoi(e), kRG + kRM - 1));
     p.skip_publish = -1;
     if (const char* e = std::getenv("LA_SCAN_TEST_SKIP_PUBLISH")) p.skip_publish = std::atoi(e);
-    const int nsm = sm_count_fused();
+    const int nsm = device_sm_count();
     p.n_chain = p.BH;                 // one chain block per (b, h)
     p.heads_per_chain = 1;
     if (p.n_chain >= nsm || 2ull * p.BH * p.F >= (1ull << 31)) return cudaErrorInvalidValue;
@@ -1072,13 +1061,8 @@ cudaError_t launch_fused_mode(const ScanArgs& a, cudaStream_t st) {
     cudaError_t e = cudaMemsetAsync(a.ws, 0, L.flags_end, st);
     if (e != cudaSuccess) return e;
 
-    static bool attr_done = false;
-    if (!attr_done) {
-        e = cudaFuncSetAttribute(tc_fused_kernel<RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)kFusedSmem);
-        if (e != cudaSuccess) return e;
-        attr_done = true;
-    }
+    e = ensure_dyn_smem(reinterpret_cast<const void*>(tc_fused_kernel<RELU>), (int)kFusedSmem);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(nsm);
     cfg.blockDim = dim3(kThreads);
@@ -1107,7 +1091,7 @@ extern "C" __attribute__((visibility("default"))) int la_trace_install(void* buf
 // least two thirds of them stream.
 bool fused_eligible(const ScanArgs& a) {
     if (!tc_eligible(a)) return false;
-    const int nsm = sm_count_fused();
+    const int nsm = device_sm_count();
     return (long)a.B * a.H <= (long)(nsm / 3);
 }
 

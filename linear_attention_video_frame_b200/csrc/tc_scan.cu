@@ -766,17 +766,6 @@ constexpr size_t smem_out = 1024 + kOStages * 32768 + 2 * kImg + 2 * 32768 +
 static_assert(smem_chain_gdn <= 232448, "chain smem");
 static_assert(smem_out <= 232448, "output smem");
 
-int sm_count() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
-}
-
 // Frames per pipeline chunk of the three-kernel path: about 8 chunks of at
 // least 16 frames, and whole chunks of the reversed scan; one chunk (no
 // pipeline) for short clips or when the per-head chain CTAs would take more
@@ -847,20 +836,19 @@ cudaError_t launch_tc_mode(const ScanArgs& a, cudaStream_t st) {
                           !make_tmap_bf16_3d(&mO, a.o, a.D, a.S, bhf, 64, kTokO)))
         return cudaErrorInvalidValue;
 
-    static bool attr_done = false;
-    if (!attr_done) {
-        if (!RELU)
-            cudaFuncSetAttribute(tc_gram_kernel<false, true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_gram);
-        cudaFuncSetAttribute(tc_gram_kernel<RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem_gram);
-        cudaFuncSetAttribute(tc_chain_kernel<RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)(RELU ? smem_chain_relu : smem_chain_gdn));
-        cudaFuncSetAttribute(tc_output_kernel<RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem_out);
-        attr_done = true;
+    {
+        const void* kernels[] = {reinterpret_cast<const void*>(tc_gram_kernel<RELU>),
+                                 reinterpret_cast<const void*>(tc_chain_kernel<RELU>),
+                                 reinterpret_cast<const void*>(tc_output_kernel<RELU>),
+                                 reinterpret_cast<const void*>(tc_gram_kernel<false, true>)};
+        const int bytes[] = {(int)smem_gram, (int)(RELU ? smem_chain_relu : smem_chain_gdn),
+                             (int)smem_out, (int)smem_gram};
+        for (int i = 0; i < (RELU ? 3 : 4); ++i) {
+            const cudaError_t e = ensure_dyn_smem(kernels[i], bytes[i]);
+            if (e != cudaSuccess) return e;
+        }
     }
-    const int nsm = sm_count();
+    const int nsm = device_sm_count();
     const int Fc = tc_chunk(a, nsm);
     const int nchunks = (p.F + Fc - 1) / Fc;
     const int thr = RELU ? 320 : 192;
@@ -941,7 +929,7 @@ bool tc_eligible(const ScanArgs& a) {
 size_t tc_workspace_bytes(const ScanArgs& a) { return ws_layout(a).total; }
 
 int tc_kernel_count(const ScanArgs& a) {
-    const int Fc = tc_chunk(a, sm_count());
+    const int Fc = tc_chunk(a, device_sm_count());
     return (a.o ? 3 : 2) * ((a.F + Fc - 1) / Fc);
 }
 

@@ -852,17 +852,6 @@ static_assert(kSmemWideGram <= 232448, "gram smem");
 static_assert(kSmemWideChain <= 232448, "chain smem");
 static_assert(smem_wide_out<false>() <= 232448 && smem_wide_out<true>() <= 232448, "output smem");
 
-int sm_count_wide() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
-}
-
 // Streams and events of one device for the chunk pipeline: the gram kernels
 // run on the caller's stream, the chain and output kernels on two streams of
 // the library's own, forked from and joined back to the caller's stream.
@@ -915,15 +904,15 @@ cudaError_t launch_wide_mode(const ScanArgs& a, cudaStream_t st) {
                           !make_tmap_bf16_3d(&mO, a.o, a.D, a.S, bhf, 64, kTokO)))
         return cudaErrorInvalidValue;
 
-    static bool attr_done = false;
-    if (!attr_done) {
-        cudaFuncSetAttribute(wide_gram_kernel<RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemWideGram);
-        cudaFuncSetAttribute(wide_chain_gdn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)kSmemWideChain);
-        cudaFuncSetAttribute(wide_output_kernel<RELU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem_wide_out<RELU>());
-        attr_done = true;
+    {
+        const void* kernels[] = {reinterpret_cast<const void*>(wide_gram_kernel<RELU>),
+                                 reinterpret_cast<const void*>(wide_chain_gdn_kernel),
+                                 reinterpret_cast<const void*>(wide_output_kernel<RELU>)};
+        const int bytes[] = {(int)kSmemWideGram, (int)kSmemWideChain, (int)smem_wide_out<RELU>()};
+        for (int i = 0; i < 3; ++i) {
+            const cudaError_t e = ensure_dyn_smem(kernels[i], bytes[i]);
+            if (e != cudaSuccess) return e;
+        }
     }
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
@@ -933,7 +922,7 @@ cudaError_t launch_wide_mode(const ScanArgs& a, cudaStream_t st) {
     cudaError_t e = wide_ctx_init(cx);
     if (e != cudaSuccess) return e;
 
-    const int nsm = sm_count_wide();
+    const int nsm = device_sm_count();
     const int nchunks = (p.F + L.Fc - 1) / L.Fc;
     // GDN: with more than one chunk, chain(c) (about 3.5 us per frame on its
     // own SMs) runs beside gram(c + 1) and output(c - 1), which share the

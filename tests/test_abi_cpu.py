@@ -22,7 +22,7 @@ def test_header_declares_the_abi():
         "la_scan_relu", "la_scan_gdn", "la_state_step", "la_workspace_size",
         "la_query_device_status", "la_status_string", "la_plan", "la_scan_gdn_noalloc",
         "la_scan_host", "la_host_workspace_size", "la_host_chunk_frames",
-        "la_scan_gdn_reverse", "la_scan_gdn_token_beta"])
+        "la_scan_gdn_reverse", "la_scan_gdn_token_beta", "la_query_noalloc_status"])
 
 
 def test_library_exports_every_declared_symbol():
@@ -214,3 +214,19 @@ def test_reversed_scan_chunks_align_with_pipeline_chunks():
 def test_wide_path_chunk_count(F, chunks):
     """Wide heads run in chunks of max(4, ceil(F / 8)) frames."""
     assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 2, F, 64, 256) == ("tcgen05_wide", 3 * chunks)
+
+
+def test_noalloc_scratch_limit_matches_its_documentation():
+    """The built-in 64 MiB scratch holds the single-kernel path's per-head
+    buffers (about 1.5 MiB per (b, h) pair whatever F is) for up to 42 pairs
+    of 128 x 128 state; 43 pairs need more and are refused."""
+    lim = la.LA_NOALLOC_SCRATCH_BYTES
+    for F in (1, 181, 961):
+        assert la.la_workspace_size(la.LA_MODE_GDN, 1, 42, F, 880, 128) <= lim
+        assert la.la_workspace_size(la.LA_MODE_GDN, 1, 43, F, 880, 128) > lim
+    # three-kernel path (more than 49 pairs): per-frame buffers, so F matters
+    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 63, 7, 880, 128)[0] == "tcgen05"
+    assert la.la_workspace_size(la.LA_MODE_GDN, 1, 63, 7, 880, 128) <= lim
+    assert la.la_workspace_size(la.LA_MODE_GDN, 1, 63, 8, 880, 128) > lim
+    # float32 inputs and D < 64 need only the header
+    assert la.la_workspace_size(la.LA_MODE_GDN, 4, 20, 181, 880, 32) < 4096

@@ -52,3 +52,25 @@ def test_every_bench_workload_names_a_synthetic_workload():
         spec = synth.workload(wname)
         assert mode in ("relu", "gdn", "gdn_reverse", "gdn_token_beta"), name
         assert spec.F > 0 and spec.S > 0
+
+
+def test_gpus_n_launches_n_ranks_and_reports_them():
+    """`bench.py --gpus 2` starts two ranks itself (torchrun on this node);
+    rank 0 prints the one line, with n_gpus equal to the ranks that ran."""
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny_gdn", "--gpus", "2", "--steps", "1",
+                          "--warmup", "1"],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out.stdout
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2
+
+
+def test_world_size_that_disagrees_with_gpus_is_an_error():
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--workload", "tiny_gdn", "--gpus", "4", "--steps", "1"],
+                         capture_output=True, text=True, timeout=300, cwd=ROOT, env=env)
+    assert out.returncode != 0 and "WORLD_SIZE" in out.stderr

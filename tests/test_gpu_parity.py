@@ -3,8 +3,7 @@
 Bars (max|gpu - ref| / max|ref| over the compared tensor): 1e-4 for float32
 inputs, 2e-2 for bfloat16 inputs with a float32 state.  Small cases are
 compared element by element in full; the full-size workloads in the launch
-configuration the benchmark times are compared on every head where the
-oracle is quick (480p ReLU, 720p GDN) and on sampled heads otherwise.
+configuration the benchmark times are compared on every head.
 """
 import ctypes
 
@@ -59,8 +58,27 @@ def _oracle(spec, mode, b, h, m0=None, z0=None):
     return o[0, 0], m[0, 0], None
 
 
-def _compare(spec, mode, heads=None, with_state=False):
-    inp = device_inputs(spec)
+class _MaxRel:
+    """max|got - ref| / max|ref| over several slices, accumulated slice by slice
+    (a full-size head is about 1 GB in float64, so heads are not stacked)."""
+
+    def __init__(self):
+        self.num = 0.0
+        self.den = 0.0
+
+    def add(self, got, ref):
+        got = np.asarray(got, dtype=np.float64)
+        ref = np.asarray(ref, dtype=np.float64)
+        self.num = max(self.num, float(np.max(np.abs(got - ref))))
+        self.den = max(self.den, float(np.max(np.abs(ref))))
+
+    @property
+    def value(self) -> float:
+        return self.num / self.den if self.den > 0 else self.num
+
+
+def _compare(spec, mode, heads=None, with_state=False, inp=None, tol=None):
+    inp = device_inputs(spec) if inp is None else inp
     m0 = z0 = None
     if with_state:
         m0n, z0n = synth.random_state(spec, scale=0.05)
@@ -68,24 +86,23 @@ def _compare(spec, mode, heads=None, with_state=False):
     o, so, zo = _run(spec, mode, inp, m0, z0 if mode == "relu" else None)
     torch.cuda.synchronize()
     assert torch.isfinite(o.float()).all()
-    tol = tol_for(spec)
+    tol = tol_for(spec) if tol is None else tol
     pairs = heads if heads is not None else [(b, h) for b in range(spec.B) for h in range(spec.H)]
-    worst = 0.0
-    ref_o, got_o, ref_m, got_m = [], [], [], []
+    e_o, e_m = _MaxRel(), _MaxRel()
     for b, h in pairs:
         rm0 = None if m0 is None else m0n[b:b + 1, h:h + 1]
         rz0 = None if z0 is None else z0n[b:b + 1, h:h + 1]
         ro, rm, rz = _oracle(spec, mode, b, h, rm0, rz0)
-        ref_o.append(ro); got_o.append(to_np(o[b, h]))
-        ref_m.append(rm); got_m.append(to_np(so[b, h]))
+        e_o.add(to_np(o[b, h]), ro)
+        e_m.add(to_np(so[b, h]), rm)
         if rz is not None:
             assert rel_err(to_np(zo[b, h]), rz) < 1e-5
-    e_o = rel_err(np.stack(got_o), np.stack(ref_o))
-    e_m = rel_err(np.stack(got_m), np.stack(ref_m))
-    print(f"\n[parity] {spec.name} {mode}: output {e_o:.3e} state {e_m:.3e} (bar {tol})")
-    assert e_o <= tol, f"output error {e_o:.3e} > {tol}"
-    assert e_m <= tol, f"state error {e_m:.3e} > {tol}"
-    return e_o, e_m
+        del ro, rm
+    print(f"\n[parity] {spec.name} {mode} ({len(pairs)} heads): output {e_o.value:.3e} "
+          f"state {e_m.value:.3e} (bar {tol})")
+    assert e_o.value <= tol, f"output error {e_o.value:.3e} > {tol}"
+    assert e_m.value <= tol, f"state error {e_m.value:.3e} > {tol}"
+    return e_o.value, e_m.value
 
 
 # ----------------------------------------------------------------------------
@@ -110,8 +127,29 @@ def test_gdn_720p_60s_all_heads():
 
 
 @pytest.mark.parametrize("mode", ["relu", "gdn"])
-def test_stress_d256_sampled_heads(mode):
-    _compare(synth.workload("stress_d256"), mode, heads=[(0, 0), (0, 11)])
+def test_stress_d256_all_heads(mode):
+    # all 16 heads, element by element: the outlier tokens are shared by every head
+    _compare(synth.workload("stress_d256"), mode)
+
+
+def test_fused_relu_on_a_60s_clip():
+    """The single-kernel path adds each frame's increment phi(K)^T V to the
+    fp32 state as a bf16 operand; ReLU has no decay, so over 181 frames the
+    rounding of the increments would compound if it were biased."""
+    spec = synth.workload("gdn_720p_60s").with_(name="relu_720p_60s_B1_H20_D128_F181_S880",
+                                                keys_l2=False, modes=("relu",))
+    assert la.la_plan(la.LA_MODE_RELU, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05_fused", 1)
+    _compare(spec, "relu")
+
+
+def test_fused_gdn_near_additive_on_a_60s_clip():
+    """alpha = 1 and small beta: the GDN state is nearly a plain sum of the
+    bf16-rounded increments beta kappa K^T V over all 181 frames."""
+    spec = synth.workload("gdn_720p_60s").with_(name="gdn_720p_60s_alpha1_beta0.05",
+                                                alpha=("const", 1.0),
+                                                beta=("uniform", 0.0, 0.05))
+    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05_fused", 1)
+    _compare(spec, "gdn")
 
 
 def test_streaming_chunks_equal_single_scan():
@@ -132,11 +170,16 @@ def test_streaming_chunks_equal_single_scan():
     # chunked == single scan up to float32 summation order
     assert rel_err(to_np(chunked), to_np(whole)) < 1e-2
     assert rel_err(to_np(state), to_np(m_whole)) < 1e-3
-    # and both match the oracle's single 64-frame scan on sampled batch items
-    for b, h in [(0, 0), (3, 19)]:
-        ro, rm, _ = _oracle(spec, "gdn", b, h)
-        assert rel_err(to_np(chunked[b, h]), ro) <= TOL_BF16
-        assert rel_err(to_np(state[b, h]), rm) <= TOL_BF16
+    # and both match the oracle's single 64-frame scan on every (b, h)
+    e_o, e_m = _MaxRel(), _MaxRel()
+    for b in range(B):
+        for h in range(H):
+            ro, rm, _ = _oracle(spec, "gdn", b, h)
+            e_o.add(to_np(chunked[b, h]), ro)
+            e_m.add(to_np(state[b, h]), rm)
+    print(f"\n[parity] {spec.name} chunked, {B * H} heads: output {e_o.value:.3e} "
+          f"state {e_m.value:.3e}")
+    assert e_o.value <= TOL_BF16 and e_m.value <= TOL_BF16
 
 
 # ----------------------------------------------------------------------------

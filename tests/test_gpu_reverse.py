@@ -62,11 +62,11 @@ def test_reverse_scan_matches_oracle(dtype, D, S, F, C):
     _compare(spec, C)
 
 
-def test_reverse_scan_720p_gdn_sampled_heads():
+def test_reverse_scan_720p_gdn_all_heads():
     """The 720p 60 s GDN workload (B1 H20 D128 F181 S880) in chunks of 8 frames."""
     spec = synth.workload("gdn_720p_60s")
     assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05", 24)
-    _compare(spec, 8, heads=[(0, 0), (0, 7), (0, 19)])
+    _compare(spec, 8)
 
 
 def test_reverse_tensor_core_path_matches_simt_path(monkeypatch):

@@ -62,6 +62,7 @@ def test_single_process_max_is_identity():
 def test_reference_arm_other_ranks_exit_quietly():
     env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
-                        "--steps", "1", "--warmup", "0"], env=env, capture_output=True,
+                        "--gpus", "2", "--steps", "1", "--warmup", "0"], env=env,
+                       capture_output=True,
                        text=True, timeout=300)
     assert r.returncode == 0 and r.stdout.strip() == ""
