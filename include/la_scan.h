@@ -90,7 +90,8 @@ typedef enum la_mode {
     LA_MODE_RELU = 0,
     LA_MODE_GDN = 1,
     LA_MODE_GDN_REVERSE = 2,     /* la_scan_gdn_reverse (for la_workspace_size, la_plan) */
-    LA_MODE_GDN_TOKEN_BETA = 3   /* la_scan_gdn_token_beta (for la_workspace_size, la_plan) */
+    LA_MODE_GDN_TOKEN_BETA = 3,  /* la_scan_gdn_token_beta (for la_workspace_size, la_plan) */
+    LA_MODE_GDN_COMPOSITE = 4    /* la_gdn_interval_composite (for la_workspace_size, la_plan) */
 } la_mode;
 
 /*
@@ -200,6 +201,69 @@ LA_API la_status la_state_step(la_mode mode, const void* k, const void* v, la_dt
                         float* state_out, float* z_out,
                         int B, int H, int F, int S, int D,
                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Transition and input composites of a frame interval (GDN).
+ * Source: SANA-WM paper summary (paperlayer), appendix C.1, "Context-parallel
+ * training" -- the 961-frame latent sequence is sharded over P GPUs along
+ * time; each rank summarises its frame interval by a compact GDN transition
+ * composite and input composite, the gathered summaries are combined by an
+ * exclusive prefix, and every rank recovers its exact initial state.
+ * Every frame is affine in the state, M_f = A_f M_{f-1} + B_f with
+ * A_f = alpha_f (I - beta_f Kh_f^T Kh_f) and B_f = beta_f Kh_f^T V_f, so for
+ * the F frames given here:
+ *   transition_out = A_F ... A_1            [B,H,D,D] f32 (key x key)
+ *   input_out      = sum_j A_F ... A_{j+1} B_j
+ *                  = the state after the F frames from a zero state
+ *                                           [B,H,D,D] f32, key-major
+ * and the state after the interval from any start M is
+ * transition_out . M + input_out.
+ *
+ * k, v, alpha, beta, k_scale as for la_scan_gdn (no q, no outputs); both
+ * output pointers are required and must not overlap.  F == 0 gives the
+ * identity and zeros.  Workspace: la_workspace_size(LA_MODE_GDN_COMPOSITE,
+ * B, H, F, S, D) bytes.  bf16 inputs with 64 <= D <= 128 run on the
+ * tensor-core path (the gram once, then 2 B H chain blocks: the input
+ * composite from zero and the transition from the identity); other shapes
+ * on the float32 SIMT kernel.
+ */
+LA_API la_status la_gdn_interval_composite(const void* k, const void* v, la_dtype dt,
+                                           const float* alpha, const float* beta,
+                                           float k_scale, float* transition_out,
+                                           float* input_out, int B, int H, int F, int S, int D,
+                                           void* workspace, size_t workspace_bytes,
+                                           cudaStream_t stream);
+
+/*
+ * Exclusive prefix over interval composites: the initial state of every
+ * interval.  Source: SANA-WM paper summary (paperlayer), appendix C.1 --
+ * the all-gathered composite summaries are composed as an exclusive prefix,
+ * which restores each rank's mathematically exact initial GDN state.
+ *
+ *   starts_out[0]   = state_in (zeros if NULL)
+ *   starts_out[r+1] = T_r . starts_out[r] + U_r
+ *
+ * transitions, inputs in : the composites of n consecutive intervals in frame
+ *                          order, each a [B, H, D, D] f32 block as
+ *                          la_gdn_interval_composite writes it; T_r starts
+ *                          at transitions + r * interval_stride and U_r at
+ *                          inputs + r * interval_stride (in floats, at least
+ *                          B*H*D*D).  Packed arrays use B*H*D*D; the
+ *                          all-gathered [n][2][B, H, D, D] buffer of a
+ *                          context-parallel exchange is read in place with
+ *                          inputs = transitions + B*H*D*D and 2*B*H*D*D.
+ * state_in            in : [B, H, D, D] f32 or NULL.
+ * starts_out         out : [n, B, H, D, D] f32, the start state of each interval.
+ * state_out          out : [B, H, D, D] f32 or NULL: the state after all n
+ *                          intervals.
+ * n >= 1; D a multiple of 16 in [16, 256].  No workspace: starts_out holds
+ * the running state.  The outputs must not overlap the inputs.  float32
+ * SIMT kernel, one launch.
+ */
+LA_API la_status la_gdn_compose_prefix(const float* transitions, const float* inputs,
+                                       size_t interval_stride, const float* state_in,
+                                       float* starts_out, float* state_out, int n, int B, int H,
+                                       int D, cudaStream_t stream);
 
 /*
  * Frame-wise GDN scan for callers that cannot allocate device memory.

@@ -27,11 +27,13 @@ __all__ = [
     "la_query_device_status", "la_status_string", "la_plan", "workspace_for",
     "la_scan_gdn_noalloc", "la_query_noalloc_status", "LA_NOALLOC_SCRATCH_BYTES", "la_scan_host",
     "la_host_workspace_size", "la_host_chunk_frames", "host_workspace_for",
+    "LA_MODE_GDN_COMPOSITE", "la_gdn_interval_composite", "la_gdn_compose_prefix",
 ]
 
 LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CUDA, LA_ERR_TIMEOUT = 0, 1, 2, 3, 4
 LA_F32, LA_BF16 = 0, 1
 LA_MODE_RELU, LA_MODE_GDN, LA_MODE_GDN_REVERSE, LA_MODE_GDN_TOKEN_BETA = 0, 1, 2, 3
+LA_MODE_GDN_COMPOSITE = 4
 LA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblavf.so")
@@ -77,6 +79,10 @@ def _load() -> ctypes.CDLL:
     L.la_host_workspace_size.restype = Z
     L.la_host_chunk_frames.argtypes = [I, I]
     L.la_host_chunk_frames.restype = I
+    L.la_gdn_interval_composite.argtypes = [P, P, I, P, P, F, P, P, I, I, I, I, I, P, Z, P]
+    L.la_gdn_interval_composite.restype = I
+    L.la_gdn_compose_prefix.argtypes = [P, P, Z, P, P, P, I, I, I, I, P]
+    L.la_gdn_compose_prefix.restype = I
     L.la_status_string.argtypes = [I]
     L.la_status_string.restype = ctypes.c_char_p
     return L
@@ -245,6 +251,51 @@ def la_scan_gdn_noalloc(q, k, v, alpha, beta, k_scale: float, o=None, state_in=N
                                  B, H, F, S, D, _stream(stream))
     _raise(st, "la_scan_gdn_noalloc")
     return o
+
+
+def la_gdn_interval_composite(k, v, alpha, beta, k_scale: float, out=None, workspace=None,
+                              stream=None):
+    """Transition and input composites of this frame interval, written to
+    out[0] (A_F ... A_1) and out[1] (the state from zero): out is
+    [2, B, H, D, D] float32 and is returned."""
+    B, H, F, S, D = k.shape
+    _check(k, "k", (B, H, F, S, D))
+    _check(v, "v", (B, H, F, S, D), k.dtype)
+    for t, n in ((alpha, "alpha"), (beta, "beta")):
+        _check(t, n, (B, H, F), torch.float32)
+    if out is None:
+        out = torch.empty((2, B, H, D, D), dtype=torch.float32, device=k.device)
+    _check(out, "out", (2, B, H, D, D), torch.float32)
+    if workspace is None:
+        workspace = workspace_for(LA_MODE_GDN_COMPOSITE, B, H, F, S, D, k.device)
+    st = lib.la_gdn_interval_composite(_ptr(k), _ptr(v), _dtype_code(k), _ptr(alpha), _ptr(beta),
+                                       float(k_scale), _ptr(out[0]), _ptr(out[1]), B, H, F, S, D,
+                                       _ptr(workspace), workspace.numel(), _stream(stream))
+    _raise(st, "la_gdn_interval_composite")
+    return out
+
+
+def la_gdn_compose_prefix(composites, state_in=None, starts=None, state_out=None, stream=None):
+    """Exclusive prefix over interval composites.  composites: [n, 2, B, H, D, D]
+    float32 (T_r, U_r of interval r, as la_gdn_interval_composite writes them
+    and as an all-gather stacks them).  Returns starts [n, B, H, D, D], the
+    initial state of every interval; state_out (if given) gets the state
+    after all n intervals."""
+    n, two, B, H, D, D2 = composites.shape
+    if two != 2 or D2 != D:
+        raise ValueError(f"composites must be [n, 2, B, H, D, D], got {tuple(composites.shape)}")
+    _check(composites, "composites", None, torch.float32)
+    _check(state_in, "state_in", (B, H, D, D), torch.float32)
+    _check(state_out, "state_out", (B, H, D, D), torch.float32)
+    if starts is None:
+        starts = torch.empty((n, B, H, D, D), dtype=torch.float32, device=composites.device)
+    _check(starts, "starts", (n, B, H, D, D), torch.float32)
+    one = B * H * D * D
+    st = lib.la_gdn_compose_prefix(_ptr(composites), _ptr(composites[0, 1]), 2 * one,
+                                   _ptr(state_in), _ptr(starts), _ptr(state_out), n, B, H, D,
+                                   _stream(stream))
+    _raise(st, "la_gdn_compose_prefix")
+    return starts
 
 
 def la_state_step(mode: int, k, v, alpha=None, beta=None, k_scale: float = 1.0,

@@ -43,6 +43,8 @@ struct ScanArgs {
     int mode;                // LA_MODE_RELU / LA_MODE_GDN
     int bf16;                // 1 if q,k,v,o are bf16
     int rev_chunk;           // > 0: reversed GDN scan reset every rev_chunk frames
+    float* trans_out;        // GDN interval composite: the transition A_F ... A_1 of the
+                             // interval goes here (and the input composite to state_out)
     void* ws;
     size_t ws_bytes;
 };
@@ -80,6 +82,7 @@ cudaError_t ensure_dyn_smem(const void* kernel, int bytes);
 
 // Launchers (host side), each returns cudaGetLastError() of its launches.
 cudaError_t launch_simt(const ScanArgs& a, cudaStream_t st);
+int simt_kernel_count(const ScanArgs& a);
 size_t simt_workspace_bytes(const ScanArgs& a);
 
 // Tensor-core path: bf16 inputs, 64 <= D <= 128, F > 0.
@@ -93,6 +96,12 @@ bool wide_eligible(const ScanArgs& a);
 size_t wide_workspace_bytes(const ScanArgs& a);
 int wide_kernel_count(const ScanArgs& a);
 cudaError_t launch_wide(const ScanArgs& a, cudaStream_t st);
+
+// Exclusive prefix over GDN interval composites (composite.cu).
+// T and U of interval r start at T + r * stride and U + r * stride (floats).
+cudaError_t launch_compose_prefix(const float* T, const float* U, size_t stride, const float* m0,
+                                  float* starts, float* mout, int n, int B, int H, int D,
+                                  cudaStream_t st);
 
 // Fused persistent tensor-core path (one cooperative launch).
 bool fused_eligible(const ScanArgs& a);

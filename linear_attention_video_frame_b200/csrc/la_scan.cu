@@ -59,7 +59,10 @@ bool use_tc(const ScanArgs& a) { return !force_simt() && tc_eligible(a); }
 
 // The reversed scan and the per-token gate run on the three-kernel tensor-core
 // path or the SIMT kernel.
-bool special(const ScanArgs& a) { return a.rev_chunk != 0 || a.beta_tok != nullptr; }
+// So do the interval composites (one chunk, chain on 2 BH blocks).
+bool special(const ScanArgs& a) {
+    return a.rev_chunk != 0 || a.beta_tok != nullptr || a.trans_out != nullptr;
+}
 
 bool use_wide(const ScanArgs& a) { return !force_simt() && !special(a) && wide_eligible(a); }
 
@@ -98,7 +101,7 @@ la_status validate(const ScanArgs& a, bool need_q) {
     la_status s = check_device(&dev);
     if (s != LA_OK) return s;
     const void* ptrs[] = {a.q, a.k, a.v, a.o, a.alpha, a.beta, a.beta_tok, a.state_in, a.z_in,
-                          a.state_out, a.z_out, a.ws};
+                          a.state_out, a.z_out, a.trans_out, a.ws};
     for (const void* p : ptrs)
         if ((s = check_ptr(p, dev)) != LA_OK) return s;
     if (a.o) {
@@ -121,6 +124,15 @@ la_status run(const ScanArgs& a, cudaStream_t st) {
                                   : launch_simt(a, st);
     if (e != cudaSuccess) { cudaGetLastError(); return LA_ERR_CUDA; }
     return LA_OK;
+}
+
+// Arguments of a size or plan query for `mode`: the variants are marked by
+// non-NULL placeholders that are never dereferenced.
+void mark_mode(ScanArgs& a, la_mode mode) {
+    a.mode = mode == LA_MODE_RELU ? LA_MODE_RELU : LA_MODE_GDN;
+    a.rev_chunk = mode == LA_MODE_GDN_REVERSE ? 1 : 0;
+    if (mode == LA_MODE_GDN_TOKEN_BETA) a.beta_tok = reinterpret_cast<const float*>(uintptr_t(16));
+    if (mode == LA_MODE_GDN_COMPOSITE) a.trans_out = reinterpret_cast<float*>(uintptr_t(16));
 }
 
 ScanArgs base_args(const void* k, const void* v, la_dtype dt, int B, int H, int F, int S, int D,
@@ -224,13 +236,66 @@ extern "C" la_status la_state_step(la_mode mode, const void* k, const void* v, l
     return run(a, stream);
 }
 
+extern "C" la_status la_gdn_interval_composite(const void* k, const void* v, la_dtype dt,
+                                               const float* alpha, const float* beta,
+                                               float k_scale, float* transition_out,
+                                               float* input_out, int B, int H, int F, int S,
+                                               int D, void* workspace, size_t workspace_bytes,
+                                               cudaStream_t stream) {
+    if (dt != LA_F32 && dt != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (!transition_out || !input_out) return LA_ERR_INVALID_ARG;
+    ScanArgs a = base_args(k, v, dt, B, H, F, S, D, workspace, workspace_bytes);
+    a.mode = LA_MODE_GDN;
+    a.alpha = alpha; a.beta = beta; a.k_scale = k_scale;
+    a.state_out = input_out;
+    a.trans_out = transition_out;
+    if (B > 0 && H > 0 && D > 0) {
+        const size_t n = (size_t)B * H * D * D * sizeof(float);
+        if (overlaps(transition_out, n, input_out, n)) return LA_ERR_INVALID_ARG;
+    }
+    const la_status s = validate(a, false);
+    if (s != LA_OK) return s;
+    return run(a, stream);
+}
+
+extern "C" la_status la_gdn_compose_prefix(const float* transitions, const float* inputs,
+                                           size_t interval_stride, const float* state_in,
+                                           float* starts_out, float* state_out, int n, int B,
+                                           int H, int D, cudaStream_t stream) {
+    if (n < 1 || B < 1 || H < 1 || B > 65535 || H > 65535) return LA_ERR_INVALID_ARG;
+    if ((double)B * H > 65535.0) return LA_ERR_INVALID_ARG;
+    if (!shape_supported(D)) return LA_ERR_UNSUPPORTED;
+    if (!transitions || !inputs || !starts_out) return LA_ERR_INVALID_ARG;
+    const size_t one_n = (size_t)B * H * D * D;              // floats of one [B, H, D, D]
+    if (interval_stride < one_n) return LA_ERR_INVALID_ARG;
+    int dev = 0;
+    la_status s = check_device(&dev);
+    if (s != LA_OK) return s;
+    const void* ptrs[] = {transitions, inputs, state_in, starts_out, state_out};
+    for (const void* p : ptrs)
+        if ((s = check_ptr(p, dev)) != LA_OK) return s;
+    const size_t one = one_n * sizeof(float);
+    const size_t span = ((size_t)(n - 1) * interval_stride + one_n) * sizeof(float);
+    const size_t all = one * n;
+    const void* ins[] = {transitions, inputs, state_in};
+    const size_t in_n[] = {span, span, one};
+    for (int i = 0; i < 3; ++i)
+        if (overlaps(starts_out, all, ins[i], in_n[i]) || overlaps(state_out, one, ins[i], in_n[i]))
+            return LA_ERR_INVALID_ARG;
+    if (overlaps(starts_out, all, state_out, one)) return LA_ERR_INVALID_ARG;
+    if (launch_compose_prefix(transitions, inputs, interval_stride, state_in, starts_out,
+                              state_out, n, B, H, D, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return LA_ERR_CUDA;
+    }
+    return LA_OK;
+}
+
 extern "C" size_t la_workspace_size(la_mode mode, int B, int H, int F, int S, int D) {
     if (B < 1 || H < 1 || F < 0 || S < 1 || !shape_supported(D)) return 0;
-    if (mode < LA_MODE_RELU || mode > LA_MODE_GDN_TOKEN_BETA) return 0;
+    if (mode < LA_MODE_RELU || mode > LA_MODE_GDN_COMPOSITE) return 0;
     ScanArgs a = base_args(nullptr, nullptr, LA_BF16, B, H, F, S, D, nullptr, 0);
-    a.mode = mode == LA_MODE_RELU ? LA_MODE_RELU : LA_MODE_GDN;
-    a.rev_chunk = mode == LA_MODE_GDN_REVERSE ? 1 : 0;
-    if (mode == LA_MODE_GDN_TOKEN_BETA) a.beta_tok = reinterpret_cast<const float*>(uintptr_t(16));
+    mark_mode(a, mode);
     size_t n = workspace_needed(a);
     a.bf16 = 0;
     size_t n32 = workspace_needed(a);
@@ -251,13 +316,12 @@ extern "C" la_status la_query_device_status(void* workspace, cudaStream_t stream
 extern "C" const char* la_plan(la_mode mode, la_dtype dt, int B, int H, int F, int S, int D,
                                int* kernels) {
     if (B < 1 || H < 1 || F < 0 || S < 1 || !shape_supported(D)) return nullptr;
-    if (mode < LA_MODE_RELU || mode > LA_MODE_GDN_TOKEN_BETA || (dt != LA_F32 && dt != LA_BF16))
+    if (mode < LA_MODE_RELU || mode > LA_MODE_GDN_COMPOSITE || (dt != LA_F32 && dt != LA_BF16))
         return nullptr;
     ScanArgs a = base_args(nullptr, nullptr, dt, B, H, F, S, D, nullptr, 0);
-    a.mode = mode == LA_MODE_RELU ? LA_MODE_RELU : LA_MODE_GDN;
-    a.rev_chunk = mode == LA_MODE_GDN_REVERSE ? 1 : 0;
-    if (mode == LA_MODE_GDN_TOKEN_BETA) a.beta_tok = reinterpret_cast<const float*>(uintptr_t(16));
-    a.o = reinterpret_cast<void*>(uintptr_t(1));    // a scan (with outputs)
+    mark_mode(a, mode);
+    if (mode != LA_MODE_GDN_COMPOSITE)
+        a.o = reinterpret_cast<void*>(uintptr_t(1));    // a scan (with outputs)
     if (use_fused(a)) {
         if (kernels) *kernels = 1;
         return "tcgen05_fused";
@@ -270,7 +334,7 @@ extern "C" const char* la_plan(la_mode mode, la_dtype dt, int B, int H, int F, i
         if (kernels) *kernels = wide_kernel_count(a);
         return "tcgen05_wide";
     }
-    if (kernels) *kernels = 1;
+    if (kernels) *kernels = simt_kernel_count(a);
     return "simt_f32";
 }
 

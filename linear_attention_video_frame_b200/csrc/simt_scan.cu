@@ -14,7 +14,12 @@
 // ReLU mode accumulates the additive block state and normaliser of the
 // SANA-Video block KV cache (talk, block KV cache segment).  With
 // rev_chunk > 0 the GDN frames are taken in the reversed, chunk-reset order
-// of the SANA-WM paper summary (section 3, "Chunk-causal deployment").
+// of the SANA-WM paper summary (section 3, "Chunk-causal deployment").  With
+// trans_out set (the interval composites of that summary's context-parallel
+// training, appendix C.1) a second set of blocks runs the same GDN
+// recurrence from the identity with V = 0, which leaves the transition
+// composite A_F ... A_1; the first set, from a zero state, leaves the input
+// composite.
 #include "common.cuh"
 
 namespace la {
@@ -56,7 +61,10 @@ simt_scan_kernel(ScanArgs a) {
     float* sden = smem + L.den;
 
     const int j0 = blockIdx.x * kDJ;
-    const int h = blockIdx.y, b = blockIdx.z;
+    // With trans_out set, blocks z >= B compute the interval's transition
+    // composite A_F ... A_1: the same recurrence from the identity with V = 0.
+    const bool trans = a.trans_out && (int)blockIdx.z >= a.B;
+    const int h = blockIdx.y, b = trans ? (int)blockIdx.z - a.B : (int)blockIdx.z;
     const int tid = threadIdx.x;
     const int jj = tid % kDJ;          // this thread's state column within the slice
     const int rr = tid / kDJ;          // row phase 0..7
@@ -66,7 +74,8 @@ simt_scan_kernel(ScanArgs a) {
     // ---- initial state slice (and normaliser) ----
     for (int i = tid; i < D * kDJ; i += kThreads) {
         int d = i / kDJ, j = i % kDJ;
-        sM[i] = (a.state_in && j0 + j < D) ? a.state_in[(bh * D + d) * D + j0 + j] : 0.f;
+        if (trans) sM[i] = (d == j0 + j) ? 1.f : 0.f;
+        else sM[i] = (a.state_in && j0 + j < D) ? a.state_in[(bh * D + d) * D + j0 + j] : 0.f;
     }
     if (relu)
         for (int d = tid; d < D; d += kThreads) sz[d] = a.z_in ? a.z_in[bh * D + d] : 0.f;
@@ -104,7 +113,7 @@ simt_scan_kernel(ScanArgs a) {
             }
             for (int i = tid; i < kT * kDJ; i += kThreads) {
                 int t = i / kDJ, j = i % kDJ;
-                sV[i] = (t < nt && j0 + j < D)
+                sV[i] = (!trans && t < nt && j0 + j < D)
                             ? load_elem(a.v, (frame + t0 + t) * D + j0 + j, a.bf16) : 0.f;
             }
             __syncthreads();
@@ -177,11 +186,12 @@ simt_scan_kernel(ScanArgs a) {
         }
     }
 
-    // ---- final state ----
-    if (a.state_out)
+    // ---- final state (or transition composite) ----
+    float* out = trans ? a.trans_out : a.state_out;
+    if (out)
         for (int i = tid; i < D * kDJ; i += kThreads) {
             int d = i / kDJ, j = i % kDJ;
-            if (j0 + j < D) a.state_out[(bh * D + d) * D + j0 + j] = sM[i];
+            if (j0 + j < D) out[(bh * D + d) * D + j0 + j] = sM[i];
         }
     if (relu && a.z_out && blockIdx.x == 0)
         for (int d = tid; d < D; d += kThreads) a.z_out[bh * D + d] = sz[d];
@@ -191,12 +201,14 @@ simt_scan_kernel(ScanArgs a) {
 
 size_t simt_workspace_bytes(const ScanArgs&) { return kWsHeaderBytes; }
 
+int simt_kernel_count(const ScanArgs&) { return 1; }
+
 cudaError_t launch_simt(const ScanArgs& a, cudaStream_t st) {
     const size_t smem = (size_t)simt_smem(a.D).total * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(simt_scan_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((a.D + kDJ - 1) / kDJ, a.H, a.B);
+    dim3 grid((a.D + kDJ - 1) / kDJ, a.H, a.B * (a.trans_out ? 2 : 1));
     simt_scan_kernel<<<grid, kThreads, smem, st>>>(a);
     return cudaGetLastError();
 }

@@ -22,7 +22,11 @@
 // exchanges (appendix C.1) -- and the block-causal ReLU linear attention of
 // the SANA-Video talk (block KV cache segment).
 //
-// Variants.  The reversed GDN scan reset at chunk boundaries (SANA-WM paper
+// Variants.  Interval composites (SANA-WM paper summary, appendix C.1,
+// context-parallel training) run the gram once and the chain on 2 BH
+// blocks: from a zero state (input composite) and, without the input term,
+// from the identity (transition composite).
+// The reversed GDN scan reset at chunk boundaries (SANA-WM paper
 // summary, section 3, "Chunk-causal deployment") changes only the chain:
 // its frame order and a zero state at each chunk start.  The per-token
 // update gate (section 3, "Hybrid GDN/Softmax Attention") changes only the
@@ -87,6 +91,8 @@ struct TcParams {
     int rev_chunk;          // > 0: reversed GDN scan reset every rev_chunk frames
     const float* beta_tok;  // per-token update gate [BHF][S] (GDN), or NULL
     int f0, Fc;             // this launch covers frames [f0, f0 + Fc) of every head
+    float* trans_out;       // GDN interval composite: chain blocks BH .. 2 BH - 1 leave
+                            // the transition A_F ... A_1 here, or NULL
 };
 
 // Global frame index (into q, k, v, o, the gates and the per-frame workspace
@@ -366,7 +372,12 @@ tc_chain_kernel(const TcParams p) {
     uint32_t* abort_flag = tmem_slot + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bh = blockIdx.x;
+    // Interval composites (trans_out set): blocks BH .. 2 BH - 1 run the same
+    // recurrence from the identity without the input term, which leaves the
+    // transition composite A_F ... A_1; blocks 0 .. BH - 1 leave the input
+    // composite (the state from zero).
+    const bool trans = p.trans_out && (int)blockIdx.x >= p.BH;
+    const int bh = trans ? (int)blockIdx.x - p.BH : (int)blockIdx.x;
     const int F = p.F, D = p.D;
     const int nsteps = p.Fc;                // steps of this launch: clip steps f0 .. f0 + Fc - 1
     if (threadIdx.x == 0) {
@@ -397,11 +408,13 @@ tc_chain_kernel(const TcParams p) {
                 if (!mbar_wait(&empty[s], ph ^ 1, ab, 0x201)) break;
                 const size_t frame = (size_t)bh * F + step_frame(p.f0 + f, F, p.rev_chunk);
                 uint8_t* st = ring + s * kStage;
-                mbar_expect_tx(&full[s], kStage);
                 if (!RELU) {
+                    mbar_expect_tx(&full[s], trans ? kImg : kStage);
                     bulk_load(st, p.gimg + frame * kImg, kImg, &full[s]);
-                    bulk_load(st + kImg, p.bmat + frame * (kQuadMat / 4), kQuadMat, &full[s]);
+                    if (!trans)
+                        bulk_load(st + kImg, p.bmat + frame * (kQuadMat / 4), kQuadMat, &full[s]);
                 } else {
+                    mbar_expect_tx(&full[s], kStage);
                     bulk_load(st, p.bmat + frame * (kQuadMat / 4), kQuadMat, &full[s]);
                     bulk_load(st + kQuadMat, p.dz + frame * 128, 512, &full[s]);
                 }
@@ -439,7 +452,9 @@ tc_chain_kernel(const TcParams p) {
             float v[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e)
-                v[e] = (p.state_in && live) ? p.state_in[((size_t)bh * D + row) * D + c0 + e] : 0.f;
+                v[e] = trans ? (row == c0 + e ? 1.f : 0.f)
+                             : ((p.state_in && live) ? p.state_in[((size_t)bh * D + row) * D + c0 + e]
+                                                     : 0.f);
             tmem_st16(tl + c0, v);
             store_row16_bf16(mimg, row, c0, v);
         }
@@ -468,13 +483,16 @@ tc_chain_kernel(const TcParams p) {
             if (issuer && p.want_output) bulk_wait_read<0>();   // image free for rewriting
             named_bar_sync(1, kEpiThreads);
             const bool last = (f == nsteps - 1);
+            float* sout = trans ? p.trans_out : p.state_out;
             for (int c0 = 0; c0 < D && ok; c0 += 16) {
                 float v[16];
                 tmem_ld16(tl + c0, v);
                 tmem_wait_ld();
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const float4 b = *reinterpret_cast<const float4*>(bq + ((c0 / 4 + u) * 128 + row) * 4);
+                    const float4 b = trans ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                           : *reinterpret_cast<const float4*>(
+                                                 bq + ((c0 / 4 + u) * 128 + row) * 4);
                     const float ae = reset ? 0.f : al;
                     v[4 * u] = reset ? b.x : fmaf(ae, v[4 * u], b.x);
                     v[4 * u + 1] = reset ? b.y : fmaf(ae, v[4 * u + 1], b.y);
@@ -483,10 +501,10 @@ tc_chain_kernel(const TcParams p) {
                 }
                 tmem_st16(tl + c0, v);
                 store_row16_bf16(mimg, row, c0, v);
-                if (last && p.state_out && live)
+                if (last && sout && live)
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
-                        *reinterpret_cast<float4*>(p.state_out + ((size_t)bh * D + row) * D + c0 + 4 * u) =
+                        *reinterpret_cast<float4*>(sout + ((size_t)bh * D + row) * D + c0 + 4 * u) =
                             make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
             }
             if (RELU && ok) {
@@ -772,6 +790,7 @@ static_assert(smem_out <= 232448, "output smem");
 // than half of the SMs.
 int tc_chunk(const ScanArgs& a, int nsm) {
     int c = a.F;
+    if (a.trans_out) return std::max(1, a.F);     // interval composites: one chunk
     if (a.F >= 32 && 2 * a.B * a.H <= nsm) c = std::max(16, (a.F + 7) / 8);
     if (a.rev_chunk > 0) c = (c + a.rev_chunk - 1) / a.rev_chunk * a.rev_chunk;
     if (const char* e = std::getenv("LA_TC_CHUNK")) {
@@ -826,6 +845,7 @@ cudaError_t launch_tc_mode(const ScanArgs& a, cudaStream_t st) {
     p.want_output = a.o != nullptr;
     p.rev_chunk = a.rev_chunk;
     p.beta_tok = a.beta_tok;
+    p.trans_out = a.trans_out;
 
     const uint64_t bhf = (uint64_t)p.BH * p.F;
     CUtensorMap mK, mV, mQ, mO;
@@ -872,7 +892,8 @@ cudaError_t launch_tc_mode(const ScanArgs& a, cudaStream_t st) {
         set_chunk(0);
         const int grid_f = (int)std::min<uint64_t>(bhf, (uint64_t)nsm);
         gram(grid_f, st);
-        tc_chain_kernel<RELU><<<p.BH, 192, RELU ? smem_chain_relu : smem_chain_gdn, st>>>(p);
+        tc_chain_kernel<RELU><<<p.BH * (p.trans_out ? 2 : 1), 192,
+                                RELU ? smem_chain_relu : smem_chain_gdn, st>>>(p);
         if (p.want_output) tc_output_kernel<RELU><<<grid_f, thr, smem_out, st>>>(p, mQ, mO);
         return cudaGetLastError();
     }

@@ -22,7 +22,8 @@ def test_header_declares_the_abi():
         "la_scan_relu", "la_scan_gdn", "la_state_step", "la_workspace_size",
         "la_query_device_status", "la_status_string", "la_plan", "la_scan_gdn_noalloc",
         "la_scan_host", "la_host_workspace_size", "la_host_chunk_frames",
-        "la_scan_gdn_reverse", "la_scan_gdn_token_beta", "la_query_noalloc_status"])
+        "la_scan_gdn_reverse", "la_scan_gdn_token_beta", "la_query_noalloc_status",
+        "la_gdn_interval_composite", "la_gdn_compose_prefix"])
 
 
 def test_library_exports_every_declared_symbol():
@@ -127,7 +128,7 @@ def test_token_gate_scan_argument_errors_and_plan():
     assert ws >= 256 and ws % 256 == 0
     assert la.la_plan(la.LA_MODE_GDN_TOKEN_BETA, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05", 24)
     assert la.la_plan(la.LA_MODE_GDN_TOKEN_BETA, la.LA_F32, 1, 2, 8, 64, 32)[0] == "simt_f32"
-    assert la.la_workspace_size(4, 1, 1, 4, 16, 64) == 0
+    assert la.la_workspace_size(5, 1, 1, 4, 16, 64) == 0      # no mode 5
     args = lambda bt=P(), D=64, w=ws: (P(), P(), P(), P(), la.LA_BF16, P(), bt, 0.1, None, None,
                                        1, 1, 4, 16, D, P(), w, None)
     assert L.la_scan_gdn_token_beta(*args(bt=None)) == la.LA_ERR_INVALID_ARG
@@ -230,3 +231,32 @@ def test_noalloc_scratch_limit_matches_its_documentation():
     assert la.la_workspace_size(la.LA_MODE_GDN, 1, 63, 8, 880, 128) > lim
     # float32 inputs and D < 64 need only the header
     assert la.la_workspace_size(la.LA_MODE_GDN, 4, 20, 181, 880, 32) < 4096
+
+
+def test_composite_and_prefix_argument_errors_and_plan():
+    L = la.lib
+    P = _fake
+    ws = la.la_workspace_size(la.LA_MODE_GDN_COMPOSITE, 1, 2, 5, 64, 128)
+    assert ws >= 256 and ws % 256 == 0
+    # one gram plus one chain launch of 2 B H blocks on the tensor-core path
+    assert la.la_plan(la.LA_MODE_GDN_COMPOSITE, la.LA_BF16, 1, 20, 45, 880, 128) == ("tcgen05", 2)
+    assert la.la_plan(la.LA_MODE_GDN_COMPOSITE, la.LA_F32, 1, 20, 45, 880, 128) == ("simt_f32", 1)
+    assert la.la_plan(la.LA_MODE_GDN_COMPOSITE, la.LA_BF16, 1, 16, 8, 1024, 256)[0] == "simt_f32"
+    # both outputs are required; they must not overlap; sizes and head dims are checked
+    assert L.la_gdn_interval_composite(P(), P(), la.LA_BF16, P(), P(), 0.1, None, P(0x20000),
+                                       1, 2, 5, 64, 128, P(), ws, None) == la.LA_ERR_INVALID_ARG
+    assert L.la_gdn_interval_composite(P(), P(), la.LA_BF16, P(), P(), 0.1, P(0x20000),
+                                       P(0x20000), 1, 2, 5, 64, 128, P(), ws, None) == \
+        la.LA_ERR_INVALID_ARG
+    assert L.la_gdn_interval_composite(P(), P(), la.LA_BF16, P(), P(), 0.1, P(0x20000),
+                                       P(0x90000), 1, 2, 5, 64, 24, P(), ws, None) == \
+        la.LA_ERR_UNSUPPORTED
+    one = 2 * 3 * 64 * 64
+    assert L.la_gdn_compose_prefix(P(), P(), one, None, P(), None, 0, 2, 3, 64, None) == \
+        la.LA_ERR_INVALID_ARG
+    assert L.la_gdn_compose_prefix(P(), P(), one - 1, None, P(), None, 2, 2, 3, 64, None) == \
+        la.LA_ERR_INVALID_ARG
+    assert L.la_gdn_compose_prefix(P(), P(), one, None, None, None, 2, 2, 3, 64, None) == \
+        la.LA_ERR_INVALID_ARG
+    assert L.la_gdn_compose_prefix(P(), P(), one, None, P(), None, 2, 2, 3, 40, None) == \
+        la.LA_ERR_UNSUPPORTED
