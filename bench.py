@@ -53,6 +53,8 @@ WORKLOADS = {
     "gdn_720p_60s_reverse8": ("gdn_720p_60s", "gdn_reverse"),
     # per-token update gate on the 720p 60 s clip
     "gdn_720p_60s_token_beta": ("gdn_720p_60s", "gdn_token_beta"),
+    # raw q, k with RMSNorm, ReLU and 3D RoPE fused into the scan (22 x 40 grid)
+    "gdn_720p_60s_prep": ("gdn_720p_60s_raw", "gdn_prep"),
     "tiny_gdn": ("tiny_fp32", "gdn"),
     "tiny_relu": ("tiny_fp32", "relu"),
 }
@@ -65,6 +67,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # Algorithmic counts (fixed formulas, whatever the kernels do)
 # ----------------------------------------------------------------------------
 REVERSE_CHUNK = 8      # frames per chunk of the reversed-scan workload
+PREP_NORM_EPS = 1e-6   # RMSNorm epsilon of the fused input preparation
 
 
 def frame_flops(mode: str, S: int, D: int) -> int:
@@ -82,10 +85,11 @@ def call_bytes(mode: str, B: int, H: int, F: int, S: int, D: int, elem: int,
     reversed scan has no state in or out)."""
     per_frame = 4 * S * D * elem + (8 if mode != "relu" else 0) + \
         (4 * (S - 1) if mode == "gdn_token_beta" else 0)
+    per_bh_prep = 2 * D * 4 if mode == "gdn_prep" else 0     # the two RMSNorm weight rows
     per_bh = D * D * 4 * (2 if state_in else 1) if mode != "gdn_reverse" else 0
     if mode == "relu":
         per_bh += D * 4 * (2 if state_in else 1)
-    return B * H * (F * per_frame + per_bh)
+    return B * H * (F * per_frame + per_bh + per_bh_prep)
 
 
 def step_plan(spec, mode):
@@ -254,6 +258,11 @@ def time_oracle_sample(spec, mode, budget_s: float, max_heads=None):
             oracle.gdn_scan_reverse_chunked(q, k, v, a, bt, spec.k_scale, REVERSE_CHUNK)
         elif mode == "gdn_token_beta":
             oracle.gdn_scan_token_beta(q, k, v, a, btok_all[b:b + 1, h:h + 1], spec.k_scale)
+        elif mode == "gdn_prep":
+            gh, gw = spec.grid
+            oracle.gdn_scan_prep(q, k, v, a, bt, spec.k_scale,
+                                 synth.norm_weights(spec, "q")[h:h + 1],
+                                 synth.norm_weights(spec, "k")[h:h + 1], PREP_NORM_EPS, gh, gw)
         else:
             oracle.gdn_scan(q, k, v, a, bt, spec.k_scale)
         t_total += time.perf_counter() - t0
@@ -269,7 +278,7 @@ def time_oracle_sample(spec, mode, budget_s: float, max_heads=None):
 def workload_label(spec_name: str, mode: str) -> str:
     """config.workload of a JSON line: the workload's name, plus the variant."""
     return spec_name + {"gdn_reverse": f"_reverse{REVERSE_CHUNK}",
-                        "gdn_token_beta": "_token_beta"}.get(mode, "")
+                        "gdn_token_beta": "_token_beta", "gdn_prep": "_prep"}.get(mode, "")
 
 
 def run_reference(args):
@@ -358,7 +367,12 @@ def run_ours(args):
     plan = step_plan(spec, mode)
     mode_c = {"gdn": la.LA_MODE_GDN, "relu": la.LA_MODE_RELU,
               "gdn_reverse": la.LA_MODE_GDN_REVERSE,
-              "gdn_token_beta": la.LA_MODE_GDN_TOKEN_BETA}[mode]
+              "gdn_token_beta": la.LA_MODE_GDN_TOKEN_BETA,
+              "gdn_prep": la.LA_MODE_GDN_PREP}[mode]
+    prep = None
+    if mode == "gdn_prep":
+        prep_w = [torch.from_numpy(synth.norm_weights(spec, n)).to(dev) for n in ("q", "k")]
+        prep = la.make_prep(prep_w[0], prep_w[1], PREP_NORM_EPS, True, spec.grid)
     if mode == "gdn_token_beta":
         host["beta"] = torch.from_numpy(synth.token_gates(spec)).pin_memory()
         dev_in["beta"] = host["beta"].to(dev)
@@ -381,6 +395,9 @@ def run_ours(args):
             if mode == "gdn_token_beta":
                 la.la_scan_gdn_token_beta(q, k, v, al, be, spec.k_scale, o=oo, state_out=state,
                                           workspace=ws, stream=stream)
+            elif mode == "gdn_prep":
+                la.la_scan_gdn_prep(q, k, v, al, be, spec.k_scale, prep, o=oo, state_out=state,
+                                    workspace=ws, stream=stream)
             elif mode == "gdn_reverse":
                 la.la_scan_gdn_reverse(q, k, v, al, be, spec.k_scale, REVERSE_CHUNK, o=oo,
                                        workspace=ws, stream=stream)
@@ -470,7 +487,7 @@ def run_ours(args):
     ins = ("q", "k", "v") if mode == "relu" else ("q", "k", "v", "alpha", "beta")
     if mode == "gdn_reverse":
         so_host = None          # the reversed scan has no state out
-    special = mode in ("gdn_reverse", "gdn_token_beta")
+    special = mode in ("gdn_reverse", "gdn_token_beta", "gdn_prep")
     h2d = sum(host[x].numel() * host[x].element_size() for x in ins)
     d2h = sum(t.numel() * t.element_size() for t in (o_host, so_host, zo_host) if t is not None)
     e2e_call = "la_scan_host"
@@ -487,6 +504,11 @@ def run_ours(args):
                 la.la_scan_gdn_reverse(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"],
                                        dev_in["beta"], spec.k_scale, REVERSE_CHUNK, o=o,
                                        workspace=ws, stream=stream)
+            elif mode == "gdn_prep":
+                la.la_scan_gdn_prep(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"],
+                                    dev_in["beta"], spec.k_scale, prep, o=o, state_out=state,
+                                    workspace=ws, stream=stream)
+                so_host.copy_(state, non_blocking=True)
             else:
                 la.la_scan_gdn_token_beta(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["alpha"],
                                           dev_in["beta"], spec.k_scale, o=o, state_out=state,

@@ -91,8 +91,36 @@ typedef enum la_mode {
     LA_MODE_GDN = 1,
     LA_MODE_GDN_REVERSE = 2,     /* la_scan_gdn_reverse (for la_workspace_size, la_plan) */
     LA_MODE_GDN_TOKEN_BETA = 3,  /* la_scan_gdn_token_beta (for la_workspace_size, la_plan) */
-    LA_MODE_GDN_COMPOSITE = 4    /* la_gdn_interval_composite (for la_workspace_size, la_plan) */
+    LA_MODE_GDN_COMPOSITE = 4,   /* la_gdn_interval_composite (for la_workspace_size, la_plan) */
+    LA_MODE_GDN_PREP = 5,        /* la_scan_gdn_prep (for la_workspace_size, la_plan) */
+    LA_MODE_RELU_PREP = 6        /* la_scan_relu_prep (for la_workspace_size, la_plan) */
 } la_mode;
+
+/*
+ * Input preparation fused into the scan: RMSNorm, ReLU and 3D RoPE of q and
+ * k.  Source: SANA-WM digest, method details, "Context-Parallel + Fused
+ * Triton" paragraph -- RMSNorm, ReLU, key scaling, UCPE/RoPE and the GDN
+ * scan run as one kernel; SANA-WM paper summary, appendix C.1 (the fused
+ * kernel combines normalization, activation, scaling, positional
+ * preparation and recurrent scanning); SANA-Video talk, 3D RoPE for the
+ * linear attention.  The pages give the order, not the formulas; reading:
+ *   y  = x / sqrt(mean_d x_d^2 + norm_eps) * weight[h]   (per token, per head)
+ *   y  = max(y, 0)
+ *   y~ = RoPE(y): channel pairs (2i, 2i+1); the first D/2 - 2 floor(D/6)
+ *        pairs are temporal, the next floor(D/6) height, the last floor(D/6)
+ *        width; pair i of a group of n pairs turns by pos * rope_base^(-i/n),
+ *        pos = frame_offset + frame, s / grid_w or s % grid_w for token s.
+ * The key scale k_scale is still applied inside the scan.
+ */
+typedef struct la_prep {
+    const float* q_weight;  /* [H, D] f32 RMSNorm weight of q, or NULL (ones)              */
+    const float* k_weight;  /* [H, D] f32 RMSNorm weight of k, or NULL (ones)              */
+    float norm_eps;         /* RMSNorm epsilon, finite and >= 0 (1e-6 is usual)            */
+    int rope;               /* non-zero: 3D RoPE after the ReLU                            */
+    int grid_h, grid_w;     /* latent grid of a frame (rope only): S == grid_h * grid_w    */
+    int frame_offset;       /* temporal position of frame 0 (a chunk of a longer clip), >= 0 */
+    float rope_base;        /* RoPE base, finite and > 1 (10000 is usual)                   */
+} la_prep;
 
 /*
  * Block-causal ReLU linear attention with normaliser over latent frames.
@@ -183,6 +211,45 @@ LA_API la_status la_scan_gdn_token_beta(const void* q, const void* k, const void
                                         int B, int H, int F, int S, int D,
                                         void* workspace, size_t workspace_bytes,
                                         cudaStream_t stream);
+
+/*
+ * Frame-wise GDN on raw q and k with the input preparation (la_prep) fused
+ * into the scan: q~ = RoPE(ReLU(RMSNorm(q))), k~ = RoPE(ReLU(RMSNorm(k))), then
+ * the recurrence of la_scan_gdn with Kh = k_scale k~ and O_f = Q~_f M_f.
+ * Arguments as for la_scan_gdn plus `prep` (required).  Workspace:
+ * la_workspace_size(LA_MODE_GDN_PREP, ...).  bf16 inputs with
+ * 64 <= D <= 128 on the single-kernel path (B*H <= SMs/3), when the RoPE
+ * tables of the grid fit in shared memory (about (grid_h + grid_w) * D / 6
+ * entries of 8 bytes, at most 24 KiB), prepare the tiles in shared memory
+ * between the TMA loads and the tensor core; other shapes run on the
+ * float32 SIMT kernel.
+ */
+LA_API la_status la_scan_gdn_prep(const void* q, const void* k, const void* v, void* o,
+                                  la_dtype dt, const float* alpha, const float* beta,
+                                  float k_scale, const la_prep* prep,
+                                  const float* state_in, float* state_out,
+                                  int B, int H, int F, int S, int D,
+                                  void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Block-causal ReLU linear attention on raw q and k with the input
+ * preparation fused: phi_x = ReLU(RMSNorm(x)); RoPE (if prep->rope) enters
+ * the numerator only, the normaliser keeps the unrotated features (reading:
+ * rotated features can be negative, which would remove the positivity the
+ * normaliser relies on):
+ *   M_f = M_{f-1} + RoPE(phi_k)^T V_f,   z_f = z_{f-1} + sum_t phi_k[t]
+ *   O_f[t] = RoPE(phi_q)[t] M_f / (phi_q[t] . z_f + eps)
+ * Arguments as for la_scan_relu plus `prep` (required).  Workspace:
+ * la_workspace_size(LA_MODE_RELU_PREP, ...).  Runs on the float32 SIMT
+ * kernel.
+ */
+LA_API la_status la_scan_relu_prep(const void* q, const void* k, const void* v, void* o,
+                                   la_dtype dt, const la_prep* prep,
+                                   const float* state_in, const float* z_in,
+                                   float* state_out, float* z_out,
+                                   int B, int H, int F, int S, int D, float eps,
+                                   void* workspace, size_t workspace_bytes,
+                                   cudaStream_t stream);
 
 /*
  * Advance the cached state over finished frames without producing outputs:

@@ -28,15 +28,25 @@ __all__ = [
     "la_scan_gdn_noalloc", "la_query_noalloc_status", "LA_NOALLOC_SCRATCH_BYTES", "la_scan_host",
     "la_host_workspace_size", "la_host_chunk_frames", "host_workspace_for",
     "LA_MODE_GDN_COMPOSITE", "la_gdn_interval_composite", "la_gdn_compose_prefix",
+    "LA_MODE_GDN_PREP", "LA_MODE_RELU_PREP", "LaPrep", "make_prep", "la_scan_gdn_prep",
+    "la_scan_relu_prep",
 ]
 
 LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CUDA, LA_ERR_TIMEOUT = 0, 1, 2, 3, 4
 LA_F32, LA_BF16 = 0, 1
 LA_MODE_RELU, LA_MODE_GDN, LA_MODE_GDN_REVERSE, LA_MODE_GDN_TOKEN_BETA = 0, 1, 2, 3
-LA_MODE_GDN_COMPOSITE = 4
+LA_MODE_GDN_COMPOSITE, LA_MODE_GDN_PREP, LA_MODE_RELU_PREP = 4, 5, 6
 LA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "liblavf.so")
+
+
+class LaPrep(ctypes.Structure):
+    """The C struct la_prep (fused input preparation of q and k)."""
+    _fields_ = [("q_weight", ctypes.c_void_p), ("k_weight", ctypes.c_void_p),
+                ("norm_eps", ctypes.c_float), ("rope", ctypes.c_int),
+                ("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int),
+                ("frame_offset", ctypes.c_int), ("rope_base", ctypes.c_float)]
 
 
 class LaScanError(RuntimeError):
@@ -83,6 +93,12 @@ def _load() -> ctypes.CDLL:
     L.la_gdn_interval_composite.restype = I
     L.la_gdn_compose_prefix.argtypes = [P, P, Z, P, P, P, I, I, I, I, P]
     L.la_gdn_compose_prefix.restype = I
+    L.la_scan_gdn_prep.argtypes = [P, P, P, P, I, P, P, F, ctypes.POINTER(LaPrep), P, P,
+                                   I, I, I, I, I, P, Z, P]
+    L.la_scan_gdn_prep.restype = I
+    L.la_scan_relu_prep.argtypes = [P, P, P, P, I, ctypes.POINTER(LaPrep), P, P, P, P,
+                                    I, I, I, I, I, F, P, Z, P]
+    L.la_scan_relu_prep.restype = I
     L.la_status_string.argtypes = [I]
     L.la_status_string.restype = ctypes.c_char_p
     return L
@@ -296,6 +312,60 @@ def la_gdn_compose_prefix(composites, state_in=None, starts=None, state_out=None
                                    _stream(stream))
     _raise(st, "la_gdn_compose_prefix")
     return starts
+
+
+def make_prep(q_weight=None, k_weight=None, norm_eps: float = 1e-6, rope: bool = True,
+              grid=(1, 1), frame_offset: int = 0, rope_base: float = 10000.0) -> LaPrep:
+    """An la_prep struct; q_weight / k_weight are [H, D] float32 CUDA tensors or None.
+    The struct holds raw pointers: keep the weight tensors alive while it is used."""
+    for t, n in ((q_weight, "q_weight"), (k_weight, "k_weight")):
+        _check(t, n, None, torch.float32)
+    return LaPrep(_ptr(q_weight), _ptr(k_weight), float(norm_eps), int(bool(rope)),
+                  int(grid[0]), int(grid[1]), int(frame_offset), float(rope_base))
+
+
+def la_scan_gdn_prep(q, k, v, alpha, beta, k_scale: float, prep: LaPrep, o=None, state_in=None,
+                     state_out=None, workspace=None, stream=None):
+    """la_scan_gdn on raw q, k with RMSNorm, ReLU and 3D RoPE fused (see la_prep)."""
+    B, H, F, S, D = k.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _check(t, n, (B, H, F, S, D), k.dtype)
+    for t, n in ((alpha, "alpha"), (beta, "beta")):
+        _check(t, n, (B, H, F), torch.float32)
+    for t, n in ((state_in, "state_in"), (state_out, "state_out")):
+        _check(t, n, (B, H, D, D), torch.float32)
+    if o is None:
+        o = torch.empty_like(q)
+    if workspace is None:
+        workspace = workspace_for(LA_MODE_GDN_PREP, B, H, F, S, D, q.device)
+    st = lib.la_scan_gdn_prep(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _dtype_code(k), _ptr(alpha),
+                              _ptr(beta), float(k_scale), ctypes.byref(prep), _ptr(state_in),
+                              _ptr(state_out), B, H, F, S, D, _ptr(workspace), workspace.numel(),
+                              _stream(stream))
+    _raise(st, "la_scan_gdn_prep")
+    return o
+
+
+def la_scan_relu_prep(q, k, v, prep: LaPrep, o=None, state_in=None, z_in=None, state_out=None,
+                      z_out=None, eps: float = 1e-6, workspace=None, stream=None):
+    """la_scan_relu on raw q, k with RMSNorm, ReLU and (numerator) 3D RoPE fused."""
+    B, H, F, S, D = k.shape
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _check(t, n, (B, H, F, S, D), k.dtype)
+    for t, n in ((state_in, "state_in"), (state_out, "state_out")):
+        _check(t, n, (B, H, D, D), torch.float32)
+    for t, n in ((z_in, "z_in"), (z_out, "z_out")):
+        _check(t, n, (B, H, D), torch.float32)
+    if o is None:
+        o = torch.empty_like(q)
+    if workspace is None:
+        workspace = workspace_for(LA_MODE_RELU_PREP, B, H, F, S, D, q.device)
+    st = lib.la_scan_relu_prep(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _dtype_code(k),
+                               ctypes.byref(prep), _ptr(state_in), _ptr(z_in), _ptr(state_out),
+                               _ptr(z_out), B, H, F, S, D, float(eps), _ptr(workspace),
+                               workspace.numel(), _stream(stream))
+    _raise(st, "la_scan_relu_prep")
+    return o
 
 
 def la_state_step(mode: int, k, v, alpha=None, beta=None, k_scale: float = 1.0,

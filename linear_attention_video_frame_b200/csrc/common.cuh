@@ -45,6 +45,8 @@ struct ScanArgs {
     int rev_chunk;           // > 0: reversed GDN scan reset every rev_chunk frames
     float* trans_out;        // GDN interval composite: the transition A_F ... A_1 of the
                              // interval goes here (and the input composite to state_out)
+    int has_prep;            // 1: RMSNorm, ReLU and (prep.rope) 3D RoPE of q and k in the scan
+    la_prep prep;
     void* ws;
     size_t ws_bytes;
 };
@@ -61,6 +63,22 @@ __host__ __device__ inline int step_frame(int s, int F, int C) {
 }
 __host__ __device__ inline bool step_resets(int s, int C) { return C > 0 && s % C == 0; }
 
+// 3D RoPE (fused input preparation).  Pairs of a head of D channels: the
+// first rope_nt(D) are temporal, then rope_nhw(D) height, then rope_nhw(D)
+// width pairs; pair i of a group of n pairs turns by pos * base^(-i / n).
+__host__ __device__ inline int rope_nhw(int D) { return (D / 2) / 3; }
+__host__ __device__ inline int rope_nt(int D) { return D / 2 - 2 * rope_nhw(D); }
+
+// cos and sin of pos * base^(-i / n).  The angle is formed and reduced
+// modulo 2 pi in double, so that positions up to 2^24 keep float accuracy.
+__device__ inline void rope_cos_sin(int pos, int i, int n, double log2_base, float& c, float& s) {
+    const double th = exp2(-(double)i / (double)n * log2_base);
+    double ang = (double)pos * th;
+    const double two_pi = 6.283185307179586476925286766559;
+    ang -= two_pi * rint(ang / two_pi);
+    sincosf((float)ang, &s, &c);
+}
+
 // Element access for the two storage types.
 __device__ __forceinline__ float load_elem(const void* p, size_t i, int bf16) {
     if (bf16) return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[i]);
@@ -76,8 +94,9 @@ __device__ __forceinline__ void store_elem(void* p, size_t i, float x, int bf16)
 constexpr int kDefaultSmCount = 148;   // B200; used only when no device is visible
 int current_device();                   // current device, or -1
 int device_sm_count();                  // SMs of the current device (cached per device)
-// Opt `kernel` in to `bytes` of dynamic shared memory on the current device
-// (once per device and kernel); returns the CUDA error of the first failure.
+// Opt `kernel` in to at least `bytes` of dynamic shared memory on the
+// current device (the limit is raised when a call asks for more than any
+// earlier one, never lowered); returns the CUDA error of a failure.
 cudaError_t ensure_dyn_smem(const void* kernel, int bytes);
 
 // Launchers (host side), each returns cudaGetLastError() of its launches.
@@ -105,6 +124,8 @@ cudaError_t launch_compose_prefix(const float* T, const float* U, size_t stride,
 
 // Fused persistent tensor-core path (one cooperative launch).
 bool fused_eligible(const ScanArgs& a);
+// The fused kernel prepares q and k itself (GDN) when its RoPE tables fit.
+bool fused_prep_fits(const ScanArgs& a);
 size_t fused_workspace_bytes(const ScanArgs& a);
 cudaError_t launch_fused(const ScanArgs& a, cudaStream_t st);
 

@@ -1,8 +1,8 @@
 // Facts and one-time set-up that belong to a device, not to the process: a
 // process may drive several GPUs, and both a kernel's shared-memory opt-in
 // (cudaFuncSetAttribute) and the SM count are properties of one device.
+#include <map>
 #include <mutex>
-#include <set>
 #include <utility>
 
 #include "common.cuh"
@@ -13,7 +13,8 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_dev_mu;
 int g_sm_count[kMaxDevices] = {};
-std::set<std::pair<int, const void*>> g_smem_done;   // (device, kernel) pairs set up
+// Largest dynamic shared memory each (device, kernel) has been opted in to.
+std::map<std::pair<int, const void*>, int> g_smem_set;
 
 }  // namespace
 
@@ -47,14 +48,17 @@ cudaError_t ensure_dyn_smem(const void* kernel, int bytes) {
     if (dev < 0) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(g_dev_mu);
     const std::pair<int, const void*> key(dev, kernel);
-    if (g_smem_done.count(key)) return cudaSuccess;
+    auto it = g_smem_set.find(key);
+    if (it != g_smem_set.end() && it->second >= bytes) return cudaSuccess;
+    // A kernel whose shared memory depends on the call's shape (D) may ask
+    // for more than an earlier call did: raise the limit, never lower it.
     const cudaError_t e =
         cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) {
         cudaGetLastError();
         return e;
     }
-    g_smem_done.insert(key);
+    g_smem_set[key] = bytes;
     return cudaSuccess;
 }
 

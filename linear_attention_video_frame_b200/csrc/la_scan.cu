@@ -55,13 +55,15 @@ bool force_simt() {
     return e && e[0] == '1';
 }
 
-bool use_tc(const ScanArgs& a) { return !force_simt() && tc_eligible(a); }
+// Calls with a fused input preparation take the single-kernel path (GDN) or
+// the SIMT kernel, never the three-kernel or wide paths.
+bool use_tc(const ScanArgs& a) { return !force_simt() && tc_eligible(a) && !a.has_prep; }
 
 // The reversed scan and the per-token gate run on the three-kernel tensor-core
 // path or the SIMT kernel.
 // So do the interval composites (one chunk, chain on 2 BH blocks).
 bool special(const ScanArgs& a) {
-    return a.rev_chunk != 0 || a.beta_tok != nullptr || a.trans_out != nullptr;
+    return a.rev_chunk != 0 || a.beta_tok != nullptr || a.trans_out != nullptr || a.has_prep;
 }
 
 bool use_wide(const ScanArgs& a) { return !force_simt() && !special(a) && wide_eligible(a); }
@@ -70,13 +72,30 @@ bool use_wide(const ScanArgs& a) { return !force_simt() && !special(a) && wide_e
 // compare the two).
 bool use_fused(const ScanArgs& a) {
     const char* e = std::getenv("LA_SCAN_NO_FUSE");
-    return use_tc(a) && !special(a) && !(e && e[0] == '1') && fused_eligible(a);
+    if (e && e[0] == '1') return false;
+    if (a.has_prep)
+        return !force_simt() && tc_eligible(a) && a.mode == LA_MODE_GDN && a.rev_chunk == 0 &&
+               !a.beta_tok && !a.trans_out && fused_eligible(a) && fused_prep_fits(a);
+    return use_tc(a) && !special(a) && fused_eligible(a);
 }
 
 size_t workspace_needed(const ScanArgs& a) {
     if (use_fused(a)) return fused_workspace_bytes(a);
     if (use_tc(a)) return tc_workspace_bytes(a);
     return use_wide(a) ? wide_workspace_bytes(a) : simt_workspace_bytes(a);
+}
+
+// The fused input preparation's own arguments (no CUDA call).
+la_status validate_prep(const ScanArgs& a) {
+    const la_prep& p = a.prep;
+    if (!(std::isfinite(p.norm_eps) && p.norm_eps >= 0.f)) return LA_ERR_INVALID_ARG;
+    if (p.frame_offset < 0 || (double)p.frame_offset + a.F > 16777216.0) return LA_ERR_INVALID_ARG;
+    if (p.rope) {
+        if (!(std::isfinite(p.rope_base) && p.rope_base > 1.f)) return LA_ERR_INVALID_ARG;
+        if (p.grid_h < 1 || p.grid_w < 1 || (long long)p.grid_h * p.grid_w != a.S)
+            return LA_ERR_INVALID_ARG;
+    }
+    return LA_OK;
 }
 
 // Validation common to every entry point.  `need_q` is false for a state step.
@@ -88,6 +107,10 @@ la_status validate(const ScanArgs& a, bool need_q) {
     if (elems > 9.0e15) return LA_ERR_INVALID_ARG;
     if (a.mode == LA_MODE_RELU && !(std::isfinite(a.eps) && a.eps >= 0.f)) return LA_ERR_INVALID_ARG;
     if (a.mode == LA_MODE_GDN && !std::isfinite(a.k_scale)) return LA_ERR_INVALID_ARG;
+    if (a.has_prep) {
+        const la_status ps = validate_prep(a);
+        if (ps != LA_OK) return ps;
+    }
     if (!a.ws) return LA_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(a.ws) & 255u) != 0) return LA_ERR_INVALID_ARG;
     if (a.ws_bytes < workspace_needed(a)) return LA_ERR_INVALID_ARG;
@@ -101,7 +124,9 @@ la_status validate(const ScanArgs& a, bool need_q) {
     la_status s = check_device(&dev);
     if (s != LA_OK) return s;
     const void* ptrs[] = {a.q, a.k, a.v, a.o, a.alpha, a.beta, a.beta_tok, a.state_in, a.z_in,
-                          a.state_out, a.z_out, a.trans_out, a.ws};
+                          a.state_out, a.z_out, a.trans_out, a.ws,
+                          a.has_prep ? a.prep.q_weight : nullptr,
+                          a.has_prep ? a.prep.k_weight : nullptr};
     for (const void* p : ptrs)
         if ((s = check_ptr(p, dev)) != LA_OK) return s;
     if (a.o) {
@@ -129,7 +154,15 @@ la_status run(const ScanArgs& a, cudaStream_t st) {
 // Arguments of a size or plan query for `mode`: the variants are marked by
 // non-NULL placeholders that are never dereferenced.
 void mark_mode(ScanArgs& a, la_mode mode) {
-    a.mode = mode == LA_MODE_RELU ? LA_MODE_RELU : LA_MODE_GDN;
+    a.mode = (mode == LA_MODE_RELU || mode == LA_MODE_RELU_PREP) ? LA_MODE_RELU : LA_MODE_GDN;
+    if (mode == LA_MODE_GDN_PREP || mode == LA_MODE_RELU_PREP) {
+        // sizes and plans assume a grid whose RoPE tables fit the fused kernel
+        a.has_prep = 1;
+        a.prep.rope = 1;
+        a.prep.grid_h = 1;
+        a.prep.grid_w = 1;
+        a.prep.rope_base = 10000.f;
+    }
     a.rev_chunk = mode == LA_MODE_GDN_REVERSE ? 1 : 0;
     if (mode == LA_MODE_GDN_TOKEN_BETA) a.beta_tok = reinterpret_cast<const float*>(uintptr_t(16));
     if (mode == LA_MODE_GDN_COMPOSITE) a.trans_out = reinterpret_cast<float*>(uintptr_t(16));
@@ -175,6 +208,44 @@ extern "C" la_status la_scan_gdn(const void* q, const void* k, const void* v, vo
     ScanArgs a = base_args(k, v, dt, B, H, F, S, D, workspace, workspace_bytes);
     a.q = q; a.o = o; a.mode = LA_MODE_GDN; a.k_scale = k_scale;
     a.alpha = alpha; a.beta = beta; a.state_in = state_in; a.state_out = state_out;
+    la_status s = validate(a, true);
+    if (s != LA_OK) return s;
+    return run(a, stream);
+}
+
+extern "C" la_status la_scan_gdn_prep(const void* q, const void* k, const void* v, void* o,
+                                      la_dtype dt, const float* alpha, const float* beta,
+                                      float k_scale, const la_prep* prep,
+                                      const float* state_in, float* state_out,
+                                      int B, int H, int F, int S, int D,
+                                      void* workspace, size_t workspace_bytes,
+                                      cudaStream_t stream) {
+    if (dt != LA_F32 && dt != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (!prep) return LA_ERR_INVALID_ARG;
+    ScanArgs a = base_args(k, v, dt, B, H, F, S, D, workspace, workspace_bytes);
+    a.q = q; a.o = o; a.mode = LA_MODE_GDN; a.k_scale = k_scale;
+    a.alpha = alpha; a.beta = beta; a.state_in = state_in; a.state_out = state_out;
+    a.has_prep = 1;
+    a.prep = *prep;
+    la_status s = validate(a, true);
+    if (s != LA_OK) return s;
+    return run(a, stream);
+}
+
+extern "C" la_status la_scan_relu_prep(const void* q, const void* k, const void* v, void* o,
+                                       la_dtype dt, const la_prep* prep,
+                                       const float* state_in, const float* z_in,
+                                       float* state_out, float* z_out,
+                                       int B, int H, int F, int S, int D, float eps,
+                                       void* workspace, size_t workspace_bytes,
+                                       cudaStream_t stream) {
+    if (dt != LA_F32 && dt != LA_BF16) return LA_ERR_INVALID_ARG;
+    if (!prep) return LA_ERR_INVALID_ARG;
+    ScanArgs a = base_args(k, v, dt, B, H, F, S, D, workspace, workspace_bytes);
+    a.q = q; a.o = o; a.mode = LA_MODE_RELU; a.eps = eps;
+    a.state_in = state_in; a.z_in = z_in; a.state_out = state_out; a.z_out = z_out;
+    a.has_prep = 1;
+    a.prep = *prep;
     la_status s = validate(a, true);
     if (s != LA_OK) return s;
     return run(a, stream);
@@ -293,7 +364,7 @@ extern "C" la_status la_gdn_compose_prefix(const float* transitions, const float
 
 extern "C" size_t la_workspace_size(la_mode mode, int B, int H, int F, int S, int D) {
     if (B < 1 || H < 1 || F < 0 || S < 1 || !shape_supported(D)) return 0;
-    if (mode < LA_MODE_RELU || mode > LA_MODE_GDN_COMPOSITE) return 0;
+    if (mode < LA_MODE_RELU || mode > LA_MODE_RELU_PREP) return 0;
     ScanArgs a = base_args(nullptr, nullptr, LA_BF16, B, H, F, S, D, nullptr, 0);
     mark_mode(a, mode);
     size_t n = workspace_needed(a);
@@ -316,7 +387,7 @@ extern "C" la_status la_query_device_status(void* workspace, cudaStream_t stream
 extern "C" const char* la_plan(la_mode mode, la_dtype dt, int B, int H, int F, int S, int D,
                                int* kernels) {
     if (B < 1 || H < 1 || F < 0 || S < 1 || !shape_supported(D)) return nullptr;
-    if (mode < LA_MODE_RELU || mode > LA_MODE_GDN_COMPOSITE || (dt != LA_F32 && dt != LA_BF16))
+    if (mode < LA_MODE_RELU || mode > LA_MODE_RELU_PREP || (dt != LA_F32 && dt != LA_BF16))
         return nullptr;
     ScanArgs a = base_args(nullptr, nullptr, dt, B, H, F, S, D, nullptr, 0);
     mark_mode(a, mode);

@@ -32,15 +32,18 @@ constexpr int kRowsPerPass = kThreads / kDJ;   // 8
 
 struct SimtSmem {
     // offsets in floats
-    int M, K, V, U, z, den;
+    int M, K, Kn, V, U, z, den;
     int total;
 };
 
-__host__ __device__ inline SimtSmem simt_smem(int D) {
+// Kn holds the unrotated features of a tile (ReLU with RoPE: the normaliser
+// reads them, the numerator the rotated ones in K).
+__host__ __device__ inline SimtSmem simt_smem(int D, bool kn) {
     SimtSmem s;
     s.M = 0;                    // [D][kDJ]
     s.K = s.M + D * kDJ;        // [kT][D]   keys (GDN: scaled) or queries
-    s.V = s.K + kT * D;         // [kT][kDJ]
+    s.Kn = s.K + kT * D;        // [kT][D]   unrotated features (ReLU with RoPE)
+    s.V = s.Kn + (kn ? kT * D : 0);   // [kT][kDJ]
     s.U = s.V + kT * kDJ;       // [kT][kDJ] residual (GDN)
     s.z = s.U + kT * kDJ;       // [D]       normaliser (ReLU)
     s.den = s.z + D;            // [kT]
@@ -48,13 +51,70 @@ __host__ __device__ inline SimtSmem simt_smem(int D) {
     return s;
 }
 
+__host__ __device__ inline bool simt_needs_kn(const ScanArgs& a) {
+    return a.has_prep && a.prep.rope && a.mode == LA_MODE_RELU;
+}
+
+// Fused input preparation of a tile of raw rows x[t][D] (t < nt, tokens
+// t0 .. t0 + nt - 1 of frame f): RMSNorm with weight w (NULL = ones), ReLU,
+// then (prep.rope) 3D RoPE, and finally a factor `post` (the GDN key scale).
+// x receives the prepared rows; xn (if not NULL) the unrotated ones.  Eight
+// threads share a row (D / 8 consecutive channels each, an even count).
+__device__ void simt_prep_rows(const ScanArgs& a, float* x, float* xn, int nt, int t0, int f,
+                               const float* w, float post) {
+    const int D = a.D, tid = threadIdx.x;
+    const int row = tid >> 3, part = tid & 7, span = D / 8, c0 = part * span;
+    const bool live = row < nt;
+    float ss = 0.f;
+    if (live)
+        for (int c = c0; c < c0 + span; ++c) ss = fmaf(x[row * D + c], x[row * D + c], ss);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 4);
+    if (!live) {               // rows past the frame's last token stay zero in both copies
+        if (xn)
+            for (int c = c0; c < c0 + span; ++c) xn[row * D + c] = 0.f;
+        return;
+    }
+    const float r = rsqrtf(ss / (float)D + a.prep.norm_eps);
+    const int nt_p = rope_nt(D), nhw = rope_nhw(D);
+    const int s = t0 + row;
+    const double l2b = log2((double)a.prep.rope_base);
+    for (int c = c0; c < c0 + span; c += 2) {
+        float y0 = x[row * D + c] * r * (w ? w[c] : 1.f);
+        float y1 = x[row * D + c + 1] * r * (w ? w[c + 1] : 1.f);
+        y0 = fmaxf(y0, 0.f);
+        y1 = fmaxf(y1, 0.f);
+        if (xn) {
+            xn[row * D + c] = y0;
+            xn[row * D + c + 1] = y1;
+        }
+        if (a.prep.rope) {
+            const int i = c / 2;
+            int pos, ig, n;
+            if (i < nt_p) { pos = a.prep.frame_offset + f; ig = i; n = nt_p; }
+            else if (i < nt_p + nhw) { pos = s / a.prep.grid_w; ig = i - nt_p; n = nhw; }
+            else { pos = s % a.prep.grid_w; ig = i - nt_p - nhw; n = nhw; }
+            float cs, sn;
+            rope_cos_sin(pos, ig, n, l2b, cs, sn);
+            const float r0 = y0 * cs - y1 * sn, r1 = y0 * sn + y1 * cs;
+            y0 = r0;
+            y1 = r1;
+        }
+        x[row * D + c] = y0 * post;
+        x[row * D + c + 1] = y1 * post;
+    }
+}
+
 __global__ void __launch_bounds__(kThreads)
 simt_scan_kernel(ScanArgs a) {
     extern __shared__ float smem[];
     const int D = a.D, S = a.S, F = a.F;
-    const SimtSmem L = simt_smem(D);
+    const bool kn = simt_needs_kn(a);
+    const SimtSmem L = simt_smem(D, kn);
     float* sM = smem + L.M;
     float* sK = smem + L.K;
+    float* sKn = kn ? smem + L.Kn : sK;     // features the normaliser reads (ReLU)
     float* sV = smem + L.V;
     float* sU = smem + L.U;
     float* sz = smem + L.z;
@@ -109,7 +169,13 @@ simt_scan_kernel(ScanArgs a) {
                 int t = i / D;
                 float x = 0.f;
                 if (t < nt) x = load_elem(a.k, (frame + t0) * D + i, a.bf16);
-                sK[i] = relu ? fmaxf(x, 0.f) : x * a.k_scale;
+                sK[i] = a.has_prep ? x : (relu ? fmaxf(x, 0.f) : x * a.k_scale);
+            }
+            if (a.has_prep) {
+                __syncthreads();
+                simt_prep_rows(a, sK, kn ? sKn : nullptr, nt, t0, f,
+                               a.prep.k_weight ? a.prep.k_weight + (size_t)h * D : nullptr,
+                               relu ? 1.f : a.k_scale);
             }
             for (int i = tid; i < kT * kDJ; i += kThreads) {
                 int t = i / kDJ, j = i % kDJ;
@@ -141,7 +207,7 @@ simt_scan_kernel(ScanArgs a) {
             }
             if (relu && tid < D) {
                 float s = dz;
-                for (int t = 0; t < kT; ++t) s += sK[t * D + tid];
+                for (int t = 0; t < kT; ++t) s += sKn[t * D + tid];
                 dz = s;
             }
             __syncthreads();
@@ -166,12 +232,18 @@ simt_scan_kernel(ScanArgs a) {
                     int t = i / D;
                     float x = 0.f;
                     if (t < nt) x = load_elem(a.q, (frame + t0) * D + i, a.bf16);
-                    sK[i] = relu ? fmaxf(x, 0.f) : x;
+                    sK[i] = (relu && !a.has_prep) ? fmaxf(x, 0.f) : x;
                 }
                 __syncthreads();
+                if (a.has_prep) {
+                    simt_prep_rows(a, sK, kn ? sKn : nullptr, nt, t0, f,
+                                   a.prep.q_weight ? a.prep.q_weight + (size_t)h * D : nullptr,
+                                   1.f);
+                    __syncthreads();
+                }
                 if (relu && tid < kT) {
                     float s = 0.f;
-                    for (int d = 0; d < D; ++d) s = fmaf(sK[tid * D + d], sz[d], s);
+                    for (int d = 0; d < D; ++d) s = fmaf(sKn[tid * D + d], sz[d], s);
                     sden[tid] = s + a.eps;
                 }
                 __syncthreads();
@@ -204,7 +276,7 @@ size_t simt_workspace_bytes(const ScanArgs&) { return kWsHeaderBytes; }
 int simt_kernel_count(const ScanArgs&) { return 1; }
 
 cudaError_t launch_simt(const ScanArgs& a, cudaStream_t st) {
-    const size_t smem = (size_t)simt_smem(a.D).total * sizeof(float);
+    const size_t smem = (size_t)simt_smem(a.D, simt_needs_kn(a)).total * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(simt_scan_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -145,7 +145,33 @@ struct FusedParams {
     int heads_per_chain;
     int lag;
     int skip_publish;          // test hook: frame of head 0 whose gram_ready is never set
+    // fused input preparation (GDN, PREP instantiation): RMSNorm, ReLU, 3D RoPE of K and Q
+    int H;
+    const float* q_weight;     // [H, D] or NULL
+    const float* k_weight;     // [H, D] or NULL
+    float norm_eps;
+    int rope, grid_w, grid_max, frame_offset;
+    float rope_base;
 };
+
+// Shared memory of the input preparation, after the worker's own layout:
+// the RMSNorm weight row of the current item (D floats), the temporal
+// cos/sin of its frame, and the height/width cos/sin table (the two groups
+// have the same pair count and frequencies, so one table indexed by
+// position serves both).
+constexpr uint32_t kPrepSmem = 24576;
+constexpr uint32_t kPrepTabEntries = (kPrepSmem - 512 - 512) / 8;   // float2 entries
+
+constexpr size_t kWorkerSmem = kWStages * 32768 + kImg + kWStg * 16384 + 2048 + 512 + 2048 + 512 +
+                               (kIQ + 2) * sizeof(Item) + 16 +
+                               (3 * kWStages + 2 + 12 + 2 * kIQ) * 8 + 8;
+constexpr size_t kChainSmem = kCStages * 2 * kImg + 2 * kImg + 1024 + 8 + 12 * 8 + 8 + 8;
+constexpr size_t kFusedSmem = 1024 + (kWorkerSmem > kChainSmem ? kWorkerSmem : kChainSmem);
+static_assert(kFusedSmem <= 232448, "fused kernel shared memory");
+// the preparation region starts at align_up(kWorkerSmem, 16) after the 1024-byte alignment slack
+constexpr size_t kFusedSmemPrep =
+    1024 + ((kWorkerSmem > kChainSmem ? kWorkerSmem : kChainSmem) + 15) / 16 * 16 + kPrepSmem;
+static_assert(kFusedSmemPrep <= 232448, "fused kernel shared memory with the input preparation");
 
 __device__ __forceinline__ Item decode_ticket(const FusedParams& p, uint32_t t) {
     const uint32_t BH = p.BH, F = p.F;
@@ -173,7 +199,7 @@ __device__ __forceinline__ Item decode_ticket(const FusedParams& p, uint32_t t) 
 // ============================================================================
 // worker blocks
 // ============================================================================
-template <bool RELU>
+template <bool RELU, bool PREP>
 __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                                             const CUtensorMap* mK, const CUtensorMap* mV,
                                             const CUtensorMap* mQ, const CUtensorMap* mO) {
@@ -216,7 +242,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
         }
         for (int i = 0; i < kIQ; ++i) {
             mbar_init(&iqfull[i], 1);
-            mbar_init(&iqempty[i], RELU ? 3 : 2);
+            mbar_init(&iqempty[i], (RELU || PREP) ? 3 : 2);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -224,6 +250,18 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
     if (RELU)
         for (int i = threadIdx.x; i < 2048 / 4; i += blockDim.x)
             reinterpret_cast<uint32_t*>(ones)[i] = 0x3F803F80u;
+    // input preparation: weight row, temporal cos/sin, height/width table
+    float* prep_w = reinterpret_cast<float*>(smem + align_up(kWorkerSmem, 16));
+    float2* prep_t = reinterpret_cast<float2*>(prep_w + 128);
+    float2* prep_hw = prep_t + 64;
+    const int nhw = rope_nhw(p.D), ntp = rope_nt(p.D);
+    const double l2b = PREP ? log2((double)p.rope_base) : 0.0;
+    if (PREP && p.rope)
+        for (int i = threadIdx.x; i < p.grid_max * nhw; i += blockDim.x) {
+            float c, sn;
+            rope_cos_sin(i / nhw, i % nhw, nhw, l2b, c, sn);
+            prep_hw[i] = make_float2(c, sn);
+        }
     if (warp == 1) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
@@ -339,7 +377,8 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                     tc_fence_after();
                     const uint32_t dG = tbase + qa * 128, dW = tbase + qb * 128;
                     for (int t = 0; t < ntg && ok; ++t) {
-                        if (!(ok = mbar_wait(RELU ? &xform[s] : &full[s], ph, ab, 0x414))) break;
+                        if (!(ok = mbar_wait((RELU || PREP) ? &xform[s] : &full[s], ph, ab, 0x414)))
+                            break;
                         tc_fence_after();
                         const uint32_t sk = smem_u32(ring + s * 32768), sv = sk + 16384;
 #pragma unroll
@@ -370,7 +409,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                     for (int t = 0; t < nto && ok; ++t) {
                         const uint32_t qa = qctr & 3;
                         ok = mbar_wait(&qempty[qa], ((qctr >> 2) & 1) ^ 1, ab, 0x416) &&
-                             mbar_wait(RELU ? &xform[s] : &full[s], ph, ab, 0x417);
+                             mbar_wait((RELU || PREP) ? &xform[s] : &full[s], ph, ab, 0x417);
                         ++qctr;
                         if (!ok) break;
                         tc_fence_after();
@@ -538,6 +577,124 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
             }
         }
         if (leader) bulk_wait_all<0>();
+    } else if (PREP && warp < 10) {
+        // ---------------- input preparation of K (gram) and Q (output) tiles ----------------
+        // RMSNorm with the head's weight, ReLU and 3D RoPE, in place on the
+        // bf16 tile between its TMA load and the MMA (SANA-WM digest, method
+        // details: RMSNorm + ReLU + key scaling + RoPE fused with the scan;
+        // the key scale stays on the fp32 accumulators).  Thread tl owns the
+        // 16-byte column chunk tl % 16 (8 channels, 4 RoPE pairs) of 8
+        // consecutive rows, so its weights, pair groups and temporal cos/sin
+        // live in registers for a whole item; the 16 lanes that share a row
+        // combine its sum of squares with 4 shuffles.
+        const int tl = threadIdx.x - 192;          // 0..127
+        const bool leader = (tl == 0);
+        const int chunk = tl & 15, rgrp = tl >> 4; // rows 8 rgrp .. 8 rgrp + 7 of each 64
+        const bool live_c = chunk < D / 8;
+        // pair e2 of the chunk: group 0 temporal, 1 height, 2 width; index in its group
+        int grp[4], gj[4];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+            const int i = 4 * chunk + e2;
+            grp[e2] = i < ntp ? 0 : (i < ntp + nhw ? 1 : 2);
+            gj[e2] = i < ntp ? i : (i < ntp + nhw ? i - ntp : i - ntp - nhw);
+        }
+        uint32_t iq = 0, ph = 0, bcn = 0;
+        int s = 0;
+        bool ok = true;
+        int* bc2 = bc_ok + 2;
+        while (true) {
+            if (leader) {
+                const int qi = iq % kIQ;
+                Item it{kItemStop, 0, 0, 0};
+                ok = ok && mbar_wait(&iqfull[qi], (iq / kIQ) & 1, ab, 0x441);
+                if (ok) {
+                    it = items[qi];
+                    mbar_arrive(&iqempty[qi]);
+                }
+                bc_item[1] = it;
+            }
+            ++iq;
+            named_bar_sync(2, 128);
+            const Item it = bc_item[1];
+            if (it.type == kItemStop) break;
+            const bool gram = it.type == kItemGram;
+            // per-item constants of this thread's chunk: weights and temporal cos/sin
+            const float* wsrc = gram ? p.k_weight : p.q_weight;
+            const size_t wrow = (size_t)(it.bh % p.H) * D + 8 * chunk;
+            float w[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w[e] = (wsrc && live_c) ? __ldg(wsrc + wrow + e) : 1.f;
+            float2 tcs[4];
+#pragma unroll
+            for (int e2 = 0; e2 < 4; ++e2) {
+                tcs[e2] = make_float2(1.f, 0.f);
+                if (p.rope && live_c && grp[e2] == 0) {
+                    float c, sn;
+                    rope_cos_sin(p.frame_offset + it.f, gj[e2], ntp, l2b, c, sn);
+                    tcs[e2] = make_float2(c, sn);
+                }
+            }
+            const int ntile = gram ? ntg : nto;
+            const int rows = gram ? kTokG : kTokO;
+            const uint32_t box = gram ? kBoxG : kBoxO;
+            uint8_t* const cbase = ring + (chunk >> 3) * box;      // + stage + row offset
+            for (int t = 0; t < ntile; ++t) {
+                if (leader) {
+                    ok = ok && mbar_wait(&full[s], ph, ab, 0x442);
+                    bc2[bcn & 1] = ok;
+                }
+                named_bar_sync(2, 128);
+                if (bc2[(bcn++) & 1]) {
+                    for (int r0 = 8 * rgrp; r0 < rows; r0 += 64) {
+                        uint4 x[8];
+                        float ss[8];
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            x[j] = *reinterpret_cast<const uint4*>(cbase + s * 32768 +
+                                                                   sw128_off(r0 + j, chunk & 7));
+                            const float a0 = bf16_lo(x[j].x), a1 = bf16_hi(x[j].x);
+                            const float a2 = bf16_lo(x[j].y), a3 = bf16_hi(x[j].y);
+                            const float a4 = bf16_lo(x[j].z), a5 = bf16_hi(x[j].z);
+                            const float a6 = bf16_lo(x[j].w), a7 = bf16_hi(x[j].w);
+                            ss[j] = fmaf(a0, a0, fmaf(a1, a1, fmaf(a2, a2, a3 * a3))) +
+                                    fmaf(a4, a4, fmaf(a5, a5, fmaf(a6, a6, a7 * a7)));
+                        }
+#pragma unroll
+                        for (int m = 1; m < 16; m <<= 1)
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) ss[j] += __shfl_xor_sync(0xffffffffu, ss[j], m);
+                        if (!live_c) continue;                       // padding channels stay zero
+                        int tok = t * rows + r0;                     // token of the first row
+                        int hp = tok / p.grid_w, wp = tok - hp * p.grid_w;
+#pragma unroll
+                        for (int j = 0; j < 8; ++j) {
+                            const float ms = ss[j] / (float)D + p.norm_eps;
+                            const float r = ms > 0.f ? rsqrtf(ms) : 0.f;   // a zero row stays zero
+                            const bool real = tok + j < p.S;
+                            const uint32_t in[4] = {x[j].x, x[j].y, x[j].z, x[j].w};
+                            uint32_t out[4];
+#pragma unroll
+                            for (int e2 = 0; e2 < 4; ++e2) {
+                                const float y0 = fmaxf(bf16_lo(in[e2]) * w[2 * e2], 0.f) * r;
+                                const float y1 = fmaxf(bf16_hi(in[e2]) * w[2 * e2 + 1], 0.f) * r;
+                                float2 cs = tcs[e2];
+                                if (p.rope && grp[e2] != 0 && real)
+                                    cs = prep_hw[(grp[e2] == 1 ? hp : wp) * nhw + gj[e2]];
+                                out[e2] = pack_bf16x2(y0 * cs.x - y1 * cs.y, y0 * cs.y + y1 * cs.x);
+                            }
+                            *reinterpret_cast<uint4*>(cbase + s * 32768 + sw128_off(r0 + j, chunk & 7)) =
+                                make_uint4(out[0], out[1], out[2], out[3]);
+                            if (++wp == p.grid_w) { wp = 0; ++hp; }   // next token of the grid
+                        }
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xform[s]);
+                if (++s == kWStages) { s = 0; ph ^= 1; }
+            }
+        }
     } else if (RELU && warp < 10) {
         // ---------------- ReLU transforms: phi(K), phi(Q) and denominators ----------------
         const int tl = threadIdx.x - 192;          // 0..127
@@ -954,7 +1111,7 @@ __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) 
     if (warp == 1) tmem_dealloc(tM, 128);
 }
 
-template <bool RELU>
+template <bool RELU, bool PREP>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_fused_kernel(const FusedParams p, const __grid_constant__ CUtensorMap mK,
                 const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mQ,
@@ -964,7 +1121,7 @@ tc_fused_kernel(const FusedParams p, const __grid_constant__ CUtensorMap mK,
     if ((int)blockIdx.x < p.n_chain)
         chain_role<RELU>(p, smem);
     else
-        worker_role<RELU>(p, smem, &mK, &mV, &mQ, &mO);
+        worker_role<RELU, PREP>(p, smem, &mK, &mV, &mQ, &mO);
 }
 
 // ----------------------------------------------------------------------------
@@ -1001,14 +1158,9 @@ FusedLayout fused_layout(const ScanArgs& a) {
     return L;
 }
 
-constexpr size_t kWorkerSmem = kWStages * 32768 + kImg + kWStg * 16384 + 2048 + 512 + 2048 + 512 +
-                               (kIQ + 2) * sizeof(Item) + 16 +
-                               (3 * kWStages + 2 + 12 + 2 * kIQ) * 8 + 8;
-constexpr size_t kChainSmem = kCStages * 2 * kImg + 2 * kImg + 1024 + 8 + 12 * 8 + 8 + 8;
-constexpr size_t kFusedSmem = 1024 + (kWorkerSmem > kChainSmem ? kWorkerSmem : kChainSmem);
-static_assert(kFusedSmem <= 232448, "fused kernel shared memory");
 
-template <bool RELU>
+
+template <bool RELU, bool PREP>
 cudaError_t launch_fused_mode(const ScanArgs& a, cudaStream_t st) {
     const FusedLayout L = fused_layout(a);
     uint8_t* ws = reinterpret_cast<uint8_t*>(a.ws);
@@ -1037,6 +1189,15 @@ cudaError_t launch_fused_mode(const ScanArgs& a, cudaStream_t st) {
     p.want_output = a.o != nullptr;
     p.lag = LA_FUSED_LAG;
     if (const char* e = std::getenv("LA_SCAN_LAG")) p.lag = std::max(1, std::min(std::atoi(e), kRG + kRM - 1));
+    p.H = a.H;
+    p.q_weight = a.has_prep ? a.prep.q_weight : nullptr;
+    p.k_weight = a.has_prep ? a.prep.k_weight : nullptr;
+    p.norm_eps = a.prep.norm_eps;
+    p.rope = a.has_prep && a.prep.rope;
+    p.grid_w = p.rope ? a.prep.grid_w : 1;
+    p.grid_max = p.rope ? std::max(a.prep.grid_h, a.prep.grid_w) : 0;
+    p.frame_offset = a.prep.frame_offset;
+    p.rope_base = p.rope ? a.prep.rope_base : 10000.f;
     p.skip_publish = -1;
     if (const char* e = std::getenv("LA_SCAN_TEST_SKIP_PUBLISH")) p.skip_publish = std::atoi(e);
     const int nsm = device_sm_count();
@@ -1061,19 +1222,20 @@ cudaError_t launch_fused_mode(const ScanArgs& a, cudaStream_t st) {
     cudaError_t e = cudaMemsetAsync(a.ws, 0, L.flags_end, st);
     if (e != cudaSuccess) return e;
 
-    e = ensure_dyn_smem(reinterpret_cast<const void*>(tc_fused_kernel<RELU>), (int)kFusedSmem);
+    const size_t smem = PREP ? kFusedSmemPrep : kFusedSmem;
+    e = ensure_dyn_smem(reinterpret_cast<const void*>(tc_fused_kernel<RELU, PREP>), (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(nsm);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = kFusedSmem;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, tc_fused_kernel<RELU>, p, mK, mV, mQ, mO);
+    e = cudaLaunchKernelEx(&cfg, tc_fused_kernel<RELU, PREP>, p, mK, mV, mQ, mO);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -1097,9 +1259,17 @@ bool fused_eligible(const ScanArgs& a) {
 
 size_t fused_workspace_bytes(const ScanArgs& a) { return fused_layout(a).total; }
 
+// The height/width cos/sin table holds max(grid_h, grid_w) x D/6 entries.
+bool fused_prep_fits(const ScanArgs& a) {
+    if (!a.prep.rope) return true;
+    const long n = (long)std::max(a.prep.grid_h, a.prep.grid_w) * rope_nhw(a.D);
+    return n <= (long)kPrepTabEntries && rope_nt(a.D) <= 64;
+}
+
 cudaError_t launch_fused(const ScanArgs& a, cudaStream_t st) {
-    return a.mode == LA_MODE_RELU ? launch_fused_mode<true>(a, st)
-                                  : launch_fused_mode<false>(a, st);
+    if (a.has_prep) return launch_fused_mode<false, true>(a, st);     // GDN only
+    return a.mode == LA_MODE_RELU ? launch_fused_mode<true, false>(a, st)
+                                  : launch_fused_mode<false, false>(a, st);
 }
 
 }  // namespace la

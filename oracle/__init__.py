@@ -59,6 +59,30 @@ beta_f Kh^T Kh and beta_f Kh^T V become Kh^T diag(beta_f) Kh and
 Kh^T diag(beta_f) V:
     M_f = alpha_f (M_{f-1} - Kh_f^T diag(beta_f) Kh_f M_{f-1}) + Kh_f^T diag(beta_f) V_f
 
+Fused input preparation -- SANA-WM digest, method details, "Context-Parallel
++ Fused Triton" paragraph (RMSNorm + ReLU + key scaling + UCPE/RoPE + GDN
+scan fused into one kernel); SANA-WM paper summary, appendix C.1 (the fused
+kernel combines normalization, activation, scaling, positional preparation
+and recurrent scanning); SANA-Video talk, 3D RoPE for the linear attention.
+Readings (the pages give the order of the steps, no formulas):
+  - RMSNorm over the head dimension of each token, with a per-head weight:
+        y = x / sqrt(mean_d x_d^2 + eps_n) * w
+  - then phi = ReLU, then 3D RoPE over (latent frame, row, column): the D/2
+    adjacent channel pairs (2i, 2i+1) are split into a temporal group (the
+    first D/2 - 2 floor(D/6) pairs), a height group and a width group
+    (floor(D/6) pairs each); pair i of a group of n pairs turns by
+    pos * base^(-i / n), pos being the token's frame (plus a frame offset),
+    row or column on the latent grid (token s of a frame sits at row
+    s // grid_w, column s % grid_w);
+  - the key scale stays inside the scan (k_scale), as before;
+  - GDN: q~ = RoPE(phi(RMSNorm(q))), k~ = RoPE(phi(RMSNorm(k))) enter the scan;
+  - ReLU: the numerator uses the rotated features and the normaliser the
+    unrotated ones (rotated ReLU features can be negative, which would
+    remove the positivity the normaliser relies on):
+        M_f = M_{f-1} + RoPE(phi_k)^T V_f,   z_f = z_{f-1} + sum_t phi_k[t]
+        O_f[t] = RoPE(phi_q)[t] M_f / (phi_q[t] . z_f + eps),
+    with phi_x = phi(RMSNorm(x)).
+
 Array layout: q, k, v, o are [B, H, F, S, D]; alpha, beta are [B, H, F];
 state is [B, H, D, D] (key-major); z is [B, H, D].  Every input is widened
 to float64 first (bf16 and fp32 widen exactly).
@@ -72,7 +96,8 @@ import numpy as np
 __all__ = [
     "relu_scan", "gdn_scan", "relu_state_step", "gdn_state_step",
     "gdn_interval_composite", "compose_exclusive_prefix", "gdn_scan_reverse_chunked",
-    "gdn_scan_token_beta",
+    "gdn_scan_token_beta", "rms_norm", "rope3d_groups", "rope3d_angles", "rope3d_apply",
+    "prep_features", "gdn_scan_prep", "relu_scan_prep",
 ]
 
 
@@ -283,3 +308,111 @@ def compose_exclusive_prefix(composites: Sequence[Tuple[np.ndarray, np.ndarray]]
         starts.append(M.copy())
         M = T @ M + U
     return starts
+
+
+# ----------------------------------------------------------------------------
+# Fused input preparation: RMSNorm, ReLU, 3D RoPE
+# ----------------------------------------------------------------------------
+def rms_norm(x, weight=None, eps: float = 1e-6):
+    """RMSNorm of every token over the head dimension (the last axis):
+    x / sqrt(mean(x^2) + eps) * weight.  weight: [D] or None (ones)."""
+    x = _f64(x)
+    y = x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    return y if weight is None else y * _f64(weight)
+
+
+def rope3d_groups(D: int) -> Tuple[int, int, int]:
+    """Channel pairs of the temporal, height and width groups of 3D RoPE."""
+    P = D // 2
+    n_hw = P // 3
+    return P - 2 * n_hw, n_hw, n_hw
+
+
+def rope3d_angles(F: int, grid_h: int, grid_w: int, D: int, frame_offset: int = 0,
+                  base: float = 10000.0) -> np.ndarray:
+    """Rotation angle of every (frame, token, channel pair): [F, grid_h*grid_w, D/2].
+    Pair i of a group of n pairs turns by pos * base^(-i/n)."""
+    n_t, n_h, n_w = rope3d_groups(D)
+    S = grid_h * grid_w
+    shape = (F, S)
+    f_pos = np.broadcast_to((np.arange(F) + frame_offset)[:, None].astype(np.float64), shape)
+    r_pos = np.broadcast_to((np.arange(S) // grid_w)[None, :].astype(np.float64), shape)
+    c_pos = np.broadcast_to((np.arange(S) % grid_w)[None, :].astype(np.float64), shape)
+    ang = np.zeros((F, S, D // 2))
+    col = 0
+    for n, pos in ((n_t, f_pos), (n_h, r_pos), (n_w, c_pos)):
+        for i in range(n):
+            ang[:, :, col + i] = pos * base ** (-i / n)
+        col += n
+    return ang
+
+
+def rope3d_apply(x, angles) -> np.ndarray:
+    """Turn each channel pair (2i, 2i+1) of x [..., F, S, D] by angles [F, S, D/2]."""
+    x = _f64(x)
+    c, s = np.cos(angles), np.sin(angles)
+    x0, x1 = x[..., 0::2], x[..., 1::2]
+    y = np.empty_like(x)
+    y[..., 0::2] = x0 * c - x1 * s
+    y[..., 1::2] = x0 * s + x1 * c
+    return y
+
+
+def prep_features(x, weight, norm_eps: float, grid_h: int, grid_w: int,
+                  frame_offset: int = 0, base: float = 10000.0, relu: bool = True,
+                  rope: bool = True):
+    """The prepared features of x [B, H, F, S, D]: RMSNorm (weight [H, D] or
+    None), then ReLU, then 3D RoPE.  Returns (rotated, unrotated)."""
+    x = _f64(x)
+    B, H, F, S, D = x.shape
+    if grid_h * grid_w != S:
+        raise ValueError("S must equal grid_h * grid_w")
+    y = np.empty_like(x)
+    for h in range(H):
+        y[:, h] = rms_norm(x[:, h], None if weight is None else _f64(weight)[h], norm_eps)
+    if relu:
+        y = _phi(y)
+    if not rope:
+        return y, y
+    return rope3d_apply(y, rope3d_angles(F, grid_h, grid_w, D, frame_offset, base)), y
+
+
+def gdn_scan_prep(q, k, v, alpha, beta, k_scale: float, q_weight, k_weight,
+                  norm_eps: float, grid_h: int, grid_w: int, frame_offset: int = 0,
+                  base: float = 10000.0, relu: bool = True, rope: bool = True,
+                  state_in=None):
+    """Frame-wise GDN on prepared queries and keys (the fused kernel of the
+    SANA-WM digest: RMSNorm + ReLU + key scaling + RoPE + GDN scan).
+    Returns (o, M_F)."""
+    qt, _ = prep_features(q, q_weight, norm_eps, grid_h, grid_w, frame_offset, base, relu, rope)
+    kt, _ = prep_features(k, k_weight, norm_eps, grid_h, grid_w, frame_offset, base, relu, rope)
+    return gdn_scan(qt, kt, v, alpha, beta, k_scale, state_in)
+
+
+def relu_scan_prep(q, k, v, eps: float, q_weight, k_weight, norm_eps: float, grid_h: int,
+                   grid_w: int, frame_offset: int = 0, base: float = 10000.0,
+                   rope: bool = True, state_in=None, z_in=None):
+    """Block-causal ReLU linear attention on prepared features: RoPE on the
+    numerator's features only, the normaliser on the unrotated ones.
+    Returns (o, M_F, z_F)."""
+    qr, qn = prep_features(q, q_weight, norm_eps, grid_h, grid_w, frame_offset, base, True, rope)
+    kr, kn = prep_features(k, k_weight, norm_eps, grid_h, grid_w, frame_offset, base, True, rope)
+    v = _f64(v)
+    B, H, F, S, D = v.shape
+    o = np.zeros((B, H, F, S, D))
+    m_out = np.zeros((B, H, D, D))
+    z_out = np.zeros((B, H, D))
+    m0, z0 = _f64(state_in), _f64(z_in)
+    for b in range(B):
+        for h in range(H):
+            M = np.zeros((D, D)) if m0 is None else m0[b, h].copy()
+            z = np.zeros(D) if z0 is None else z0[b, h].copy()
+            for f in range(F):
+                M = M + kr[b, h, f].T @ v[b, h, f]        # rotated keys in the state
+                z = z + kn[b, h, f].sum(axis=0)          # unrotated keys in the normaliser
+                num = qr[b, h, f] @ M
+                den = qn[b, h, f] @ z
+                o[b, h, f] = num / (den + eps)[:, None]
+            m_out[b, h] = M
+            z_out[b, h] = z
+    return o, m_out, z_out

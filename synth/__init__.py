@@ -31,7 +31,7 @@ from typing import Optional, Tuple
 import numpy as np
 
 TENSOR_IDS = {"q": 0, "k": 1, "v": 2, "alpha": 10, "beta": 11, "beta_token": 12,
-              "outlier": 20, "state": 30, "z": 31}
+              "outlier": 20, "state": 30, "z": 31, "q_weight": 40, "k_weight": 41}
 
 
 # ----------------------------------------------------------------------------
@@ -73,6 +73,7 @@ class Spec:
     beta: Tuple = ("uniform", 0.0, 1.0)
     eps: float = 1e-6               # ReLU-mode normaliser epsilon
     chunk_frames: int = 0           # >0: streamed in chunks of this many frames
+    grid: Optional[Tuple[int, int]] = None   # latent grid (rows, columns) of a frame, S = rows * cols
 
     @property
     def k_scale(self) -> float:
@@ -93,17 +94,24 @@ WORKLOADS = {
             seed=0, modes=("relu", "gdn"), alpha=("uniform", 0.9, 1.0),
             beta=("uniform", 0.0, 1.0)),
     "relu_480p": Spec("relu_480p_B1_H20_D112_F21_S1560", B=1, H=20, F=21, S=1560, D=112,
-            dtype="bf16", seed=1, modes=("relu",)),
+            dtype="bf16", seed=1, modes=("relu",), grid=(30, 52)),
     "gdn_720p_60s": Spec("gdn_720p_60s_B1_H20_D128_F181_S880", B=1, H=20, F=181, S=880, D=128,
             dtype="bf16", seed=2, modes=("gdn",), keys_l2=True,
-            alpha=("sigmoid_normal", 3.0, 1.0), beta=("sigmoid_normal", 0.0, 1.0)),
+            alpha=("sigmoid_normal", 3.0, 1.0), beta=("sigmoid_normal", 0.0, 1.0),
+            grid=(22, 40)),
+    # the 720p clip with raw keys, for the scan with the input preparation
+    # fused (RMSNorm replaces the harness's L2 normalisation of the keys)
+    "gdn_720p_60s_raw": Spec("gdn_720p_60s_raw_B1_H20_D128_F181_S880", B=1, H=20, F=181, S=880,
+            D=128, dtype="bf16", seed=2, modes=("gdn",), keys_l2=False,
+            alpha=("sigmoid_normal", 3.0, 1.0), beta=("sigmoid_normal", 0.0, 1.0),
+            grid=(22, 40)),
     "gdn_stream": Spec("gdn_stream_B4_H20_D128_8x8frames_S880", B=4, H=20, F=64, S=880, D=128,
             dtype="bf16", seed=3, modes=("gdn",), keys_l2=True,
             alpha=("sigmoid_normal", 3.0, 1.0), beta=("sigmoid_normal", 0.0, 1.0),
-            chunk_frames=8),
+            chunk_frames=8, grid=(22, 40)),
     "stress_d256": Spec("stress_B1_H16_D256_F512_S1024", B=1, H=16, F=512, S=1024, D=256,
             dtype="bf16", seed=4, modes=("relu", "gdn"), outlier_frac=0.01,
-            alpha=("uniform", 0.8, 1.0), beta=("uniform", 0.0, 1.0)),
+            alpha=("uniform", 0.8, 1.0), beta=("uniform", 0.0, 1.0), grid=(32, 32)),
 }
 
 
@@ -227,6 +235,14 @@ def token_gates(spec: Spec) -> np.ndarray:
     workload's beta distribution (one value per token instead of per frame)."""
     shape = (spec.B, spec.H, spec.F, spec.S)
     return _draw_gate(spec.beta, _rng(spec.seed, TENSOR_IDS["beta_token"]), shape)
+
+
+def norm_weights(spec: Spec, tensor: str) -> np.ndarray:
+    """Per-head RMSNorm weight of q or k for the fused input preparation,
+    float32 [H, D] drawn from U(0.5, 1.5) (random-init stand-in for a
+    trained weight)."""
+    rng = _rng(spec.seed, TENSOR_IDS[tensor + "_weight"])
+    return rng.uniform(0.5, 1.5, size=(spec.H, spec.D)).astype(np.float32)
 
 
 def random_state(spec: Spec, scale: float = 1.0) -> Tuple[np.ndarray, np.ndarray]:

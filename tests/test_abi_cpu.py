@@ -23,7 +23,8 @@ def test_header_declares_the_abi():
         "la_query_device_status", "la_status_string", "la_plan", "la_scan_gdn_noalloc",
         "la_scan_host", "la_host_workspace_size", "la_host_chunk_frames",
         "la_scan_gdn_reverse", "la_scan_gdn_token_beta", "la_query_noalloc_status",
-        "la_gdn_interval_composite", "la_gdn_compose_prefix"])
+        "la_gdn_interval_composite", "la_gdn_compose_prefix", "la_scan_gdn_prep",
+        "la_scan_relu_prep"])
 
 
 def test_library_exports_every_declared_symbol():
@@ -128,7 +129,7 @@ def test_token_gate_scan_argument_errors_and_plan():
     assert ws >= 256 and ws % 256 == 0
     assert la.la_plan(la.LA_MODE_GDN_TOKEN_BETA, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05", 24)
     assert la.la_plan(la.LA_MODE_GDN_TOKEN_BETA, la.LA_F32, 1, 2, 8, 64, 32)[0] == "simt_f32"
-    assert la.la_workspace_size(5, 1, 1, 4, 16, 64) == 0      # no mode 5
+    assert la.la_workspace_size(7, 1, 1, 4, 16, 64) == 0      # no mode 7
     args = lambda bt=P(), D=64, w=ws: (P(), P(), P(), P(), la.LA_BF16, P(), bt, 0.1, None, None,
                                        1, 1, 4, 16, D, P(), w, None)
     assert L.la_scan_gdn_token_beta(*args(bt=None)) == la.LA_ERR_INVALID_ARG
@@ -260,3 +261,32 @@ def test_composite_and_prefix_argument_errors_and_plan():
         la.LA_ERR_INVALID_ARG
     assert L.la_gdn_compose_prefix(P(), P(), one, None, P(), None, 2, 2, 3, 40, None) == \
         la.LA_ERR_UNSUPPORTED
+
+
+def test_prep_argument_errors_return_before_any_cuda_call():
+    L = la.lib
+    P = _fake
+    ws = la.la_workspace_size(la.LA_MODE_GDN_PREP, 1, 2, 4, 12, 64)
+    assert ws >= la.la_workspace_size(la.LA_MODE_GDN, 1, 2, 4, 12, 64)
+    # single-kernel path for bf16 GDN with the preparation; ReLU with it on SIMT
+    assert la.la_plan(la.LA_MODE_GDN_PREP, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05_fused", 1)
+    assert la.la_plan(la.LA_MODE_RELU_PREP, la.LA_BF16, 1, 20, 21, 1560, 112) == ("simt_f32", 1)
+    assert la.la_plan(la.LA_MODE_GDN_PREP, la.LA_F32, 1, 2, 4, 12, 64) == ("simt_f32", 1)
+
+    def gdn(prep):
+        return L.la_scan_gdn_prep(P(), P(), P(), P(), la.LA_BF16, P(), P(), 0.1,
+                                  None if prep is None else ctypes.byref(prep), None, None,
+                                  1, 2, 4, 12, 64, P(), ws, None)
+
+    assert gdn(None) == la.LA_ERR_INVALID_ARG
+    mk = lambda **kw: la.LaPrep(None, None, kw.get("eps", 1e-6), kw.get("rope", 1),
+                                kw.get("gh", 3), kw.get("gw", 4), kw.get("off", 0),
+                                kw.get("base", 1e4))
+    assert gdn(mk(gh=5)) == la.LA_ERR_INVALID_ARG              # 5 x 4 != 12 tokens
+    assert gdn(mk(gh=0, gw=12)) == la.LA_ERR_INVALID_ARG
+    assert gdn(mk(base=0.5)) == la.LA_ERR_INVALID_ARG
+    assert gdn(mk(eps=float("nan"))) == la.LA_ERR_INVALID_ARG
+    assert gdn(mk(off=-3)) == la.LA_ERR_INVALID_ARG
+    assert gdn(mk(off=1 << 24)) == la.LA_ERR_INVALID_ARG       # positions stay below 2^24
+    assert L.la_scan_relu_prep(P(), P(), P(), P(), la.LA_BF16, None, None, None, None, None,
+                               1, 2, 4, 12, 64, 1e-6, P(), ws, None) == la.LA_ERR_INVALID_ARG

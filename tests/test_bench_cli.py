@@ -50,7 +50,7 @@ def test_every_bench_workload_names_a_synthetic_workload():
     import synth
     for name, (wname, mode) in bench.WORKLOADS.items():
         spec = synth.workload(wname)
-        assert mode in ("relu", "gdn", "gdn_reverse", "gdn_token_beta"), name
+        assert mode in ("relu", "gdn", "gdn_reverse", "gdn_token_beta", "gdn_prep"), name
         assert spec.F > 0 and spec.S > 0
 
 

@@ -71,7 +71,12 @@ def test_outlier_tokens_recipe():
 
 
 def test_config_table_shapes():
-    assert [synth.workload(n).D for n in synth.WORKLOAD_NAMES] == [32, 112, 128, 128, 256]
+    assert [synth.workload(n).D for n in synth.WORKLOAD_NAMES] == [32, 112, 128, 128, 128, 256]
+    for n in synth.WORKLOAD_NAMES:
+        spec = synth.workload(n)
+        assert spec.grid is None or spec.grid[0] * spec.grid[1] == spec.S, n
+    raw, l2 = synth.workload("gdn_720p_60s_raw"), synth.workload("gdn_720p_60s")
+    assert raw.with_(name=l2.name, keys_l2=True) == l2     # the same clip, raw keys
     assert synth.workload("relu_480p").S == 30 * 52 and synth.workload("gdn_720p_60s").S == 22 * 40
     assert synth.workload("gdn_stream").chunk_frames * 8 == synth.workload("gdn_stream").F
 
