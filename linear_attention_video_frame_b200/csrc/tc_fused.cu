@@ -160,7 +160,7 @@ struct FusedParams {
 // have the same pair count and frequencies, so one table indexed by
 // position serves both).
 constexpr uint32_t kPrepSmem = 24576;
-constexpr uint32_t kPrepTabEntries = (kPrepSmem - 512 - 512) / 8;   // float2 entries
+constexpr uint32_t kPrepTabEntries = (kPrepSmem - 512 - 512 - 1536) / 8;   // float2 entries
 
 constexpr size_t kWorkerSmem = kWStages * 32768 + kImg + kWStg * 16384 + 2048 + 512 + 2048 + 512 +
                                (kIQ + 2) * sizeof(Item) + 16 +
@@ -231,7 +231,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
         for (int s = 0; s < kWStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-            mbar_init(&xform[s], 4);
+            mbar_init(&xform[s], PREP ? 6 : 4);
         }
         mbar_init(mfull, 1);
         mbar_init(mempty, RELU ? 5 : 1);
@@ -251,6 +251,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
         for (int i = threadIdx.x; i < 2048 / 4; i += blockDim.x)
             reinterpret_cast<uint32_t*>(ones)[i] = 0x3F803F80u;
     // input preparation: weight row, temporal cos/sin, height/width table
+    // [weights 128 floats][temporal 64 float2][row partial sums 2 x 3 x 64 floats][h/w table]
     float* prep_w = reinterpret_cast<float*>(smem + align_up(kWorkerSmem, 16));
     float2* prep_t = reinterpret_cast<float2*>(prep_w + 128);
     float2* prep_hw = prep_t + 64;
@@ -260,7 +261,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
         for (int i = threadIdx.x; i < p.grid_max * nhw; i += blockDim.x) {
             float c, sn;
             rope_cos_sin(i / nhw, i % nhw, nhw, l2b, c, sn);
-            prep_hw[i] = make_float2(c, sn);
+            prep_hw[192 + i] = make_float2(c, sn);            // past the row partial sums
         }
     if (warp == 1) {
         tmem_alloc(tmem_slot, 512);
@@ -577,32 +578,30 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
             }
         }
         if (leader) bulk_wait_all<0>();
-    } else if (PREP && warp < 10) {
+    } else if (PREP && warp >= 6) {
         // ---------------- input preparation of K (gram) and Q (output) tiles ----------------
         // RMSNorm with the head's weight, ReLU and 3D RoPE, in place on the
         // bf16 tile between its TMA load and the MMA (SANA-WM digest, method
         // details: RMSNorm + ReLU + key scaling + RoPE fused with the scan;
-        // the key scale stays on the fp32 accumulators).  Thread tl owns the
-        // 16-byte column chunk tl % 16 (8 channels, 4 RoPE pairs) of 8
-        // consecutive rows, so its weights, pair groups and temporal cos/sin
-        // live in registers for a whole item; the 16 lanes that share a row
-        // combine its sum of squares with 4 shuffles.
-        const int tl = threadIdx.x - 192;          // 0..127
+        // the key scale stays on the fp32 accumulators).  Six warps; in each
+        // block of 64 rows, thread tl owns row tl % 64 and one third of its
+        // 16-byte chunks (part tl / 64), so every warp works on the same
+        // channels of 32 consecutive tokens: weights, pair groups and the
+        // temporal cos/sin are broadcast reads, the width cos/sin of
+        // consecutive tokens hit distinct banks.  The three partial sums of
+        // squares of a row meet in shared memory.
+        const int tl = threadIdx.x - 192;          // 0..191
         const bool leader = (tl == 0);
-        const int chunk = tl & 15, rgrp = tl >> 4; // rows 8 rgrp .. 8 rgrp + 7 of each 64
-        const bool live_c = chunk < D / 8;
-        // pair e2 of the chunk: group 0 temporal, 1 height, 2 width; index in its group
-        int grp[4], gj[4];
-#pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-            const int i = 4 * chunk + e2;
-            grp[e2] = i < ntp ? 0 : (i < ntp + nhw ? 1 : 2);
-            gj[e2] = i < ntp ? i : (i < ntp + nhw ? i - ntp : i - ntp - nhw);
-        }
-        uint32_t iq = 0, ph = 0, bcn = 0;
+        const int prow = tl & 63, part = tl >> 6;
+        const int nch = D / 8;
+        const int c_lo = (part * nch + 2) / 3, c_hi = ((part + 1) * nch + 2) / 3;   // <= 6 chunks
+        float* ssp = reinterpret_cast<float*>(prep_t + 64);   // [2][3][64] partial sums
+        float2* prep_tab = prep_hw + 192;                     // height/width table (moved past ssp)
+        uint32_t iq = 0, ph = 0, bcn = 0, blk_par = 0;
         int s = 0;
         bool ok = true;
         int* bc2 = bc_ok + 2;
+        const float inv_d = 1.f / (float)D;
         while (true) {
             if (leader) {
                 const int qi = iq % kIQ;
@@ -615,77 +614,83 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                 bc_item[1] = it;
             }
             ++iq;
-            named_bar_sync(2, 128);
+            named_bar_sync(2, 192);
             const Item it = bc_item[1];
             if (it.type == kItemStop) break;
             const bool gram = it.type == kItemGram;
-            // per-item constants of this thread's chunk: weights and temporal cos/sin
             const float* wsrc = gram ? p.k_weight : p.q_weight;
-            const size_t wrow = (size_t)(it.bh % p.H) * D + 8 * chunk;
-            float w[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) w[e] = (wsrc && live_c) ? __ldg(wsrc + wrow + e) : 1.f;
-            float2 tcs[4];
-#pragma unroll
-            for (int e2 = 0; e2 < 4; ++e2) {
-                tcs[e2] = make_float2(1.f, 0.f);
-                if (p.rope && live_c && grp[e2] == 0) {
+            const size_t wrow = (size_t)(it.bh % p.H) * D;
+            for (int i = tl; i < D; i += 192) prep_w[i] = wsrc ? __ldg(wsrc + wrow + i) : 1.f;
+            if (p.rope)
+                for (int i = tl; i < ntp; i += 192) {
                     float c, sn;
-                    rope_cos_sin(p.frame_offset + it.f, gj[e2], ntp, l2b, c, sn);
-                    tcs[e2] = make_float2(c, sn);
+                    rope_cos_sin(p.frame_offset + it.f, i, ntp, l2b, c, sn);
+                    prep_t[i] = make_float2(c, sn);
                 }
-            }
+            named_bar_sync(2, 192);
             const int ntile = gram ? ntg : nto;
             const int rows = gram ? kTokG : kTokO;
             const uint32_t box = gram ? kBoxG : kBoxO;
-            uint8_t* const cbase = ring + (chunk >> 3) * box;      // + stage + row offset
             for (int t = 0; t < ntile; ++t) {
                 if (leader) {
                     ok = ok && mbar_wait(&full[s], ph, ab, 0x442);
                     bc2[bcn & 1] = ok;
                 }
-                named_bar_sync(2, 128);
+                named_bar_sync(2, 192);
                 if (bc2[(bcn++) & 1]) {
-                    for (int r0 = 8 * rgrp; r0 < rows; r0 += 64) {
-                        uint4 x[8];
-                        float ss[8];
+                    uint8_t* const tile = ring + s * 32768;
+                    for (int r0 = 0; r0 < rows; r0 += 64, blk_par ^= 1) {
+                        const int row = r0 + prow;
+                        float* sp = ssp + blk_par * 192;
+                        uint4 x[6];
+                        float ss = 0.f;
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            x[j] = *reinterpret_cast<const uint4*>(cbase + s * 32768 +
-                                                                   sw128_off(r0 + j, chunk & 7));
-                            const float a0 = bf16_lo(x[j].x), a1 = bf16_hi(x[j].x);
-                            const float a2 = bf16_lo(x[j].y), a3 = bf16_hi(x[j].y);
-                            const float a4 = bf16_lo(x[j].z), a5 = bf16_hi(x[j].z);
-                            const float a6 = bf16_lo(x[j].w), a7 = bf16_hi(x[j].w);
-                            ss[j] = fmaf(a0, a0, fmaf(a1, a1, fmaf(a2, a2, a3 * a3))) +
-                                    fmaf(a4, a4, fmaf(a5, a5, fmaf(a6, a6, a7 * a7)));
-                        }
+                        for (int u = 0; u < 6; ++u) {
+                            const int c = c_lo + u;
+                            if (c < c_hi) {
+                                x[u] = *reinterpret_cast<const uint4*>(tile + (c >> 3) * box +
+                                                                       sw128_off(row, c & 7));
+                                const uint32_t wv[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
 #pragma unroll
-                        for (int m = 1; m < 16; m <<= 1)
-#pragma unroll
-                            for (int j = 0; j < 8; ++j) ss[j] += __shfl_xor_sync(0xffffffffu, ss[j], m);
-                        if (!live_c) continue;                       // padding channels stay zero
-                        int tok = t * rows + r0;                     // token of the first row
-                        int hp = tok / p.grid_w, wp = tok - hp * p.grid_w;
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const float ms = ss[j] / (float)D + p.norm_eps;
-                            const float r = ms > 0.f ? rsqrtf(ms) : 0.f;   // a zero row stays zero
-                            const bool real = tok + j < p.S;
-                            const uint32_t in[4] = {x[j].x, x[j].y, x[j].z, x[j].w};
-                            uint32_t out[4];
-#pragma unroll
-                            for (int e2 = 0; e2 < 4; ++e2) {
-                                const float y0 = fmaxf(bf16_lo(in[e2]) * w[2 * e2], 0.f) * r;
-                                const float y1 = fmaxf(bf16_hi(in[e2]) * w[2 * e2 + 1], 0.f) * r;
-                                float2 cs = tcs[e2];
-                                if (p.rope && grp[e2] != 0 && real)
-                                    cs = prep_hw[(grp[e2] == 1 ? hp : wp) * nhw + gj[e2]];
-                                out[e2] = pack_bf16x2(y0 * cs.x - y1 * cs.y, y0 * cs.y + y1 * cs.x);
+                                for (int e2 = 0; e2 < 4; ++e2) {
+                                    const float a0 = bf16_lo(wv[e2]), a1 = bf16_hi(wv[e2]);
+                                    ss = fmaf(a0, a0, fmaf(a1, a1, ss));
+                                }
                             }
-                            *reinterpret_cast<uint4*>(cbase + s * 32768 + sw128_off(r0 + j, chunk & 7)) =
-                                make_uint4(out[0], out[1], out[2], out[3]);
-                            if (++wp == p.grid_w) { wp = 0; ++hp; }   // next token of the grid
+                        }
+                        sp[part * 64 + prow] = ss;
+                        named_bar_sync(2, 192);
+                        const float ms = fmaf(sp[prow] + sp[64 + prow] + sp[128 + prow], inv_d,
+                                              p.norm_eps);
+                        const float r = ms > 0.f ? rsqrtf(ms) : 0.f;   // a zero row stays zero
+                        const int tok = t * rows + row;
+                        const bool real = tok < p.S;
+                        const int hp = real ? tok / p.grid_w : 0, wp = real ? tok - hp * p.grid_w : 0;
+#pragma unroll
+                        for (int u = 0; u < 6; ++u) {
+                            const int c = c_lo + u;
+                            if (c < c_hi) {
+                                const uint32_t wv[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+                                const float4 wa = *reinterpret_cast<const float4*>(prep_w + 8 * c);
+                                const float4 wb = *reinterpret_cast<const float4*>(prep_w + 8 * c + 4);
+                                const float wt[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+                                uint32_t out[4];
+#pragma unroll
+                                for (int e2 = 0; e2 < 4; ++e2) {
+                                    const int i = 4 * c + e2;               // channel pair
+                                    float2 cs = make_float2(1.f, 0.f);
+                                    if (p.rope && real)
+                                        cs = i < ntp ? prep_t[i]
+                                           : i < ntp + nhw ? prep_tab[hp * nhw + (i - ntp)]
+                                                           : prep_tab[wp * nhw + (i - ntp - nhw)];
+                                    const float rc = r * cs.x, rs = r * cs.y;
+                                    const float y0 = fmaxf(bf16_lo(wv[e2]) * wt[2 * e2], 0.f);
+                                    const float y1 = fmaxf(bf16_hi(wv[e2]) * wt[2 * e2 + 1], 0.f);
+                                    out[e2] = pack_bf16x2(fmaf(y0, rc, -y1 * rs), fmaf(y0, rs, y1 * rc));
+                                }
+                                *reinterpret_cast<uint4*>(tile + (c >> 3) * box + sw128_off(row, c & 7)) =
+                                    make_uint4(out[0], out[1], out[2], out[3]);
+                            }
                         }
                     }
                 }
