@@ -144,6 +144,8 @@ struct FusedParams {
     int n_chain;
     int heads_per_chain;
     int lag;
+    int den_col;               // ReLU, D <= 112: z_f rides in column D (hi) and D + 1 (lo) of
+                               // the state image, so one MMA gives numerator and denominator
     int skip_publish;          // test hook: frame of head 0 whose gram_ready is never set
     // fused input preparation (GDN, PREP instantiation): RMSNorm, ReLU, 3D RoPE of K and Q
     int H;
@@ -357,7 +359,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
         if (lane == 0) {
             const uint32_t idKK = idesc_bf16(128, D, true, true);
             const uint32_t idZ = idesc_bf16(128, 16, true, false);
-            const uint32_t idO = idesc_bf16(128, D, false, true);
+            const uint32_t idO = idesc_bf16(128, p.den_col ? D + 16 : D, false, true);
             const uint64_t ones_d = sdesc_sw128(smem_u32(ones), 16, 1024);
             uint32_t iq = 0, ph = 0, qctr = 0, nout = 0;
             int s = 0;
@@ -535,7 +537,8 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                     const uint32_t qa = qctr & 3;
                     if (leader) {
                         ok = ok && mbar_wait(&qfull[qa], (qctr >> 2) & 1, ab, 0x424);
-                        if (RELU) ok = ok && mbar_wait(&denready[qa], (dpar >> qa) & 1, ab, 0x425);
+                        if (RELU && !p.den_col)
+                            ok = ok && mbar_wait(&denready[qa], (dpar >> qa) & 1, ab, 0x425);
                         *bc_ok = ok;
                     }
                     dpar ^= 1u << qa;
@@ -543,7 +546,17 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                     named_bar_sync(1, 128);
                     const bool go = *bc_ok;
                     tc_fence_after();
-                    const float inv = (RELU && go) ? 1.f / denbuf[qa * 128 + row] : 1.f;
+                    float inv = 1.f;
+                    if (RELU && go) {
+                        if (p.den_col) {             // phi(Q) z_hi and phi(Q) z_lo from the MMA
+                            float dv[16];
+                            tmem_ld16(tbase + lanebase + qa * 128 + D, dv);
+                            tmem_wait_ld();
+                            inv = 1.f / (dv[0] + dv[1] + p.eps);
+                        } else {
+                            inv = 1.f / denbuf[qa * 128 + row];
+                        }
+                    }
                     // one 64-column block (16 KB) at a time through staging
                     for (int blk = 0; blk < nblk; ++blk) {
                         if (leader) bulk_wait_read<kWStg - 1>();
@@ -754,13 +767,23 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                 for (int t = 0; t < nto; ++t) {
                     const uint32_t qa = qctr & 3;
                     if (leader) {
-                        ok = ok && mbar_wait(&qempty[qa], ((qctr >> 2) & 1) ^ 1, ab, 0x434) &&
-                             mbar_wait(&full[s], ph, ab, 0x435);
+                        if (!p.den_col)
+                            ok = ok && mbar_wait(&qempty[qa], ((qctr >> 2) & 1) ^ 1, ab, 0x434);
+                        ok = ok && mbar_wait(&full[s], ph, ab, 0x435);
                         bc2[bcn & 1] = ok;
                     }
                     ++qctr;
                     named_bar_sync(2, 128);
-                    if (bc2[(bcn++) & 1]) {
+                    if (bc2[(bcn++) & 1] && p.den_col) {
+                        // phi(Q) only: the MMA forms the denominator from z in the image
+                        uint4* qt = reinterpret_cast<uint4*>(ring + s * 32768);
+                        for (int i = tl; i < 2 * (int)kBoxO / 16; i += 128) {
+                            uint4 x = qt[i];
+                            x.x = relu_bf16x2(x.x); x.y = relu_bf16x2(x.y);
+                            x.z = relu_bf16x2(x.z); x.w = relu_bf16x2(x.w);
+                            qt[i] = x;
+                        }
+                    } else if (bc2[(bcn - 1) & 1]) {
                         uint8_t* st = ring + s * 32768;
                         float den = 0.f;
                         for (int blk = 0; blk < 2 && blk * 64 < D; ++blk) {
@@ -787,7 +810,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                     __syncwarp();
                     if (lane == 0) {
                         mbar_arrive(&xform[s]);
-                        mbar_arrive(&denready[qa]);
+                        if (!p.den_col) mbar_arrive(&denready[qa]);
                     }
                     if (++s == kWStages) { s = 0; ph ^= 1; }
                 }
@@ -1034,6 +1057,12 @@ __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) 
                     if (RELU && h == 0) {
                         z += reinterpret_cast<const float*>(stage + s * 2 * kImg)[row];
                         zst[ib * 128 + row] = z;
+                        if (p.den_col) {
+                            float zv[16] = {};
+                            zv[0] = z;                                          // rounds to z_hi
+                            zv[1] = z - __bfloat162float(__float2bfloat16_rn(z));   // z_lo
+                            store_row16_bf16(img, row, D, zv);
+                        }
                         if (!more && p.z_out && live) p.z_out[(size_t)bh * D + row] = z;
                     }
                 }
@@ -1193,6 +1222,7 @@ cudaError_t launch_fused_mode(const ScanArgs& a, cudaStream_t st) {
     p.D = a.D;
     p.want_output = a.o != nullptr;
     p.lag = LA_FUSED_LAG;
+    p.den_col = (RELU && a.D <= 112) ? 1 : 0;
     if (const char* e = std::getenv("LA_SCAN_LAG")) p.lag = std::max(1, std::min(std::atoi(e), kRG + kRM - 1));
     p.H = a.H;
     p.q_weight = a.has_prep ? a.prep.q_weight : nullptr;
