@@ -76,6 +76,9 @@ bool use_fused(const ScanArgs& a) {
     if (a.has_prep)
         return !force_simt() && tc_eligible(a) && a.mode == LA_MODE_GDN && a.rev_chunk == 0 &&
                !a.beta_tok && !a.trans_out && fused_eligible(a) && fused_prep_fits(a);
+    // the reversed scan and the per-token gate (GDN) run in the fused kernel too
+    if (a.rev_chunk || a.beta_tok)
+        return use_tc(a) && a.mode == LA_MODE_GDN && !a.trans_out && fused_eligible(a);
     return use_tc(a) && !special(a) && fused_eligible(a);
 }
 

@@ -144,6 +144,9 @@ struct FusedParams {
     int n_chain;
     int heads_per_chain;
     int lag;
+    int rev_chunk;             // > 0: reversed GDN scan reset every rev_chunk frames (steps
+                               // are processed in scan order; step j is frame step_frame(j))
+    const float* beta_tok;     // per-token update gate [BH][F][S] (TOKB instantiation)
     int den_col;               // ReLU, D <= 112: z_f rides in column D (hi) and D + 1 (lo) of
                                // the state image, so one MMA gives numerator and denominator
     int skip_publish;          // test hook: frame of head 0 whose gram_ready is never set
@@ -155,6 +158,11 @@ struct FusedParams {
     int rope, grid_w, grid_max, frame_offset;
     float rope_base;
 };
+
+// What the worker's transform warps do to the tiles between TMA and the MMA
+// (besides phi in ReLU mode): nothing, the fused input preparation, or the
+// per-token update gate's sqrt(beta) row scaling of the gram tiles.
+constexpr int kXfNone = 0, kXfPrep = 1, kXfTokB = 2;
 
 // Shared memory of the input preparation, after the worker's own layout:
 // the RMSNorm weight row of the current item (D floats), the temporal
@@ -201,10 +209,11 @@ __device__ __forceinline__ Item decode_ticket(const FusedParams& p, uint32_t t) 
 // ============================================================================
 // worker blocks
 // ============================================================================
-template <bool RELU, bool PREP>
+template <bool RELU, int XF>
 __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                                             const CUtensorMap* mK, const CUtensorMap* mV,
                                             const CUtensorMap* mQ, const CUtensorMap* mO) {
+    constexpr bool PREP = XF == kXfPrep, TOKB = XF == kXfTokB;
     uint8_t* ring = smem;                                  // kWStages x 32 KB
     uint8_t* mbuf = ring + kWStages * 32768;               // M image of the current output item
     uint8_t* stg = mbuf + kImg;                            // kWStg x 16 KB epilogue staging
@@ -244,7 +253,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
         }
         for (int i = 0; i < kIQ; ++i) {
             mbar_init(&iqfull[i], 1);
-            mbar_init(&iqempty[i], (RELU || PREP) ? 3 : 2);
+            mbar_init(&iqempty[i], (RELU || PREP || TOKB) ? 3 : 2);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -302,7 +311,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                 mbar_arrive(&iqfull[qi]);
                 ++iq;
                 if (it.type == kItemStop) break;
-                const int frame = it.bh * F + it.f;
+                const int frame = it.bh * F + step_frame(it.f, F, p.rev_chunk);
                 LA_TRACE_EVENT(it.type == kItemGram ? 1 : 2, frame);
                 if (it.type == kItemGram) {
                     if (it.f >= kRG)
@@ -380,7 +389,8 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                     tc_fence_after();
                     const uint32_t dG = tbase + qa * 128, dW = tbase + qb * 128;
                     for (int t = 0; t < ntg && ok; ++t) {
-                        if (!(ok = mbar_wait((RELU || PREP) ? &xform[s] : &full[s], ph, ab, 0x414)))
+                        if (!(ok = mbar_wait((RELU || PREP || TOKB) ? &xform[s] : &full[s], ph, ab,
+                                             0x414)))
                             break;
                         tc_fence_after();
                         const uint32_t sk = smem_u32(ring + s * 32768), sv = sk + 16384;
@@ -457,7 +467,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
             named_bar_sync(1, 128);
             const Item it = bc_item[0];
             if (it.type == kItemStop) break;
-            const int frame = it.bh * F + it.f;
+            const int frame = it.bh * F + step_frame(it.f, F, p.rev_chunk);
             const int nblk = D > 64 ? 2 : 1;
             if (it.type == kItemGram) {
                 const uint32_t qa = qctr & 3, qb = (qctr + 1) & 3;
@@ -475,8 +485,10 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                 // GDN: G'' = -alpha beta kappa^2 K^T K (A operand of the chain's MMA),
                 //      B~  = beta kappa K^T V (added by the chain through an identity MMA).
                 // ReLU: B~ = phi(K)^T V, and dz = phi(K)^T 1 in fp32.
-                const float al = RELU ? 1.f : p.alpha[frame];
-                const float bt = RELU ? 1.f : p.beta[frame];
+                // a step that starts a chunk of the reversed scan has a zero decay:
+                // G'' = 0 and the chain's carried state is zero
+                const float al = RELU ? 1.f : (step_resets(it.f, p.rev_chunk) ? 0.f : p.alpha[frame]);
+                const float bt = (RELU || TOKB) ? 1.f : p.beta[frame];   // TOKB: in the rows
                 const float sg = -al * bt * p.k_scale * p.k_scale;
                 const float sw = RELU ? 1.f : bt * p.k_scale;
                 for (int im = RELU ? 1 : 0; im < 2; ++im) {
@@ -705,6 +717,71 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                                     make_uint4(out[0], out[1], out[2], out[3]);
                             }
                         }
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xform[s]);
+                if (++s == kWStages) { s = 0; ph ^= 1; }
+            }
+        }
+    } else if (TOKB && warp < 10) {
+        // ---------------- per-token update gate: sqrt(beta_t) on K and V rows ----------------
+        // Every token row of a gram item's K and V tiles is scaled by
+        // sqrt(beta_t) in shared memory (bf16), so the unchanged contractions
+        // give Kh^T diag(beta) Kh and Kh^T diag(beta) V (SANA-WM paper
+        // summary, section 3, "Hybrid GDN/Softmax Attention", per-token update
+        // gate).  Thread tl scales row tl % 64 of K (tl < 64) or of V; output
+        // tiles pass untouched (through the same barrier protocol).
+        const int tl = threadIdx.x - 192;          // 0..127
+        const bool leader = (tl == 0);
+        const int row = tl & 63;
+        const int nch = D / 8;
+        uint32_t iq = 0, ph = 0, bcn = 0;
+        int s = 0;
+        bool ok = true;
+        int* bc2 = bc_ok + 2;
+        while (true) {
+            if (leader) {
+                const int qi = iq % kIQ;
+                Item it{kItemStop, 0, 0, 0};
+                ok = ok && mbar_wait(&iqfull[qi], (iq / kIQ) & 1, ab, 0x451);
+                if (ok) {
+                    it = items[qi];
+                    mbar_arrive(&iqempty[qi]);
+                }
+                bc_item[1] = it;
+            }
+            ++iq;
+            named_bar_sync(2, 128);
+            const Item it = bc_item[1];
+            if (it.type == kItemStop) break;
+            // Output tiles are not touched, but they pass through the same
+            // wait / arrive protocol: every use of a ring stage completes one
+            // phase of its xform barrier, whose parity the MMA tracks by stage use.
+            const bool gram = it.type == kItemGram;
+            const float* bsrc =
+                p.beta_tok + ((size_t)it.bh * F + step_frame(it.f, F, p.rev_chunk)) * p.S;
+            for (int t = 0; t < (gram ? ntg : nto); ++t) {
+                const int tok = t * kTokG + row;
+                const float bv = (gram && tok < p.S) ? __ldg(bsrc + tok) : 0.f;   // before the wait
+                if (leader) {
+                    ok = ok && mbar_wait(&full[s], ph, ab, 0x452);
+                    bc2[bcn & 1] = ok;
+                }
+                named_bar_sync(2, 128);
+                if (bc2[(bcn++) & 1] && gram) {
+                    const float sb = sqrtf(fmaxf(bv, 0.f));
+                    const __nv_bfloat162 g = __floats2bfloat162_rn(sb, sb);
+                    uint8_t* const base = ring + s * 32768 + (tl >> 6) * 16384;   // K or V
+#pragma unroll 4
+                    for (int c = 0; c < nch; ++c) {
+                        uint4* pc = reinterpret_cast<uint4*>(base + (c >> 3) * kBoxG + sw128_off(row, c & 7));
+                        uint4 x = *pc;
+                        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&x);
+                        h[0] = __hmul2(h[0], g); h[1] = __hmul2(h[1], g);
+                        h[2] = __hmul2(h[2], g); h[3] = __hmul2(h[3], g);
+                        *pc = x;
                     }
                 }
                 fence_proxy_async_smem();
@@ -955,8 +1032,14 @@ __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) 
         if (active) {
             // alpha_{f+1} is read two frames ahead from the gate array (a read-only input)
             const float* ap = p.alpha + (size_t)bh * F;
-            float a_cur = (!RELU && F > 0) ? __ldg(ap) : 1.f;       // alpha_0
-            float a_nxt = (!RELU && F > 1) ? __ldg(ap + 1) : 1.f;   // alpha_1
+            // decay of scan step j (frame step_frame(j)); zero where the reversed
+            // scan starts a chunk, so that the carried state restarts from zero
+            auto alpha_at = [&](int j) -> float {
+                if (RELU || j >= F) return 1.f;
+                return step_resets(j, p.rev_chunk) ? 0.f : __ldg(ap + step_frame(j, F, p.rev_chunk));
+            };
+            float a_cur = alpha_at(0);                               // step 0
+            float a_nxt = alpha_at(1);                               // step 1
             // initial state: image of M_0 (buffer 1 = "frame -1") and TMEM alpha_0 M_0
             float z = 0.f;
             for (int c0 = c_lo; c0 < c_hi; c0 += 16) {
@@ -998,7 +1081,7 @@ __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) 
                 const bool go = bc_ok[h];
                 const float an = abc[h];
                 tc_fence_after();
-                if (leader) a_nxt = (!RELU && f + 2 < F) ? __ldg(ap + f + 2) : 1.f;
+                if (leader) a_nxt = alpha_at(f + 2);
                 if (go) {
                     const uint8_t* bimg = stage + s * 2 * kImg + kImg + h * 16384;
                     uint8_t* img = imgs + ib * kImg;
@@ -1145,7 +1228,7 @@ __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) 
     if (warp == 1) tmem_dealloc(tM, 128);
 }
 
-template <bool RELU, bool PREP>
+template <bool RELU, int XF>
 __global__ void __launch_bounds__(kThreads, 1)
 tc_fused_kernel(const FusedParams p, const __grid_constant__ CUtensorMap mK,
                 const __grid_constant__ CUtensorMap mV, const __grid_constant__ CUtensorMap mQ,
@@ -1155,7 +1238,7 @@ tc_fused_kernel(const FusedParams p, const __grid_constant__ CUtensorMap mK,
     if ((int)blockIdx.x < p.n_chain)
         chain_role<RELU>(p, smem);
     else
-        worker_role<RELU, PREP>(p, smem, &mK, &mV, &mQ, &mO);
+        worker_role<RELU, XF>(p, smem, &mK, &mV, &mQ, &mO);
 }
 
 // ----------------------------------------------------------------------------
@@ -1194,8 +1277,9 @@ FusedLayout fused_layout(const ScanArgs& a) {
 
 
 
-template <bool RELU, bool PREP>
+template <bool RELU, int XF>
 cudaError_t launch_fused_mode(const ScanArgs& a, cudaStream_t st) {
+    constexpr bool PREP = XF == kXfPrep;
     const FusedLayout L = fused_layout(a);
     uint8_t* ws = reinterpret_cast<uint8_t*>(a.ws);
     FusedParams p;
@@ -1223,6 +1307,8 @@ cudaError_t launch_fused_mode(const ScanArgs& a, cudaStream_t st) {
     p.want_output = a.o != nullptr;
     p.lag = LA_FUSED_LAG;
     p.den_col = (RELU && a.D <= 112) ? 1 : 0;
+    p.rev_chunk = a.rev_chunk;
+    p.beta_tok = a.beta_tok;
     if (const char* e = std::getenv("LA_SCAN_LAG")) p.lag = std::max(1, std::min(std::atoi(e), kRG + kRM - 1));
     p.H = a.H;
     p.q_weight = a.has_prep ? a.prep.q_weight : nullptr;
@@ -1258,7 +1344,7 @@ cudaError_t launch_fused_mode(const ScanArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
 
     const size_t smem = PREP ? kFusedSmemPrep : kFusedSmem;
-    e = ensure_dyn_smem(reinterpret_cast<const void*>(tc_fused_kernel<RELU, PREP>), (int)smem);
+    e = ensure_dyn_smem(reinterpret_cast<const void*>(tc_fused_kernel<RELU, XF>), (int)smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(nsm);
@@ -1270,7 +1356,7 @@ cudaError_t launch_fused_mode(const ScanArgs& a, cudaStream_t st) {
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, tc_fused_kernel<RELU, PREP>, p, mK, mV, mQ, mO);
+    e = cudaLaunchKernelEx(&cfg, tc_fused_kernel<RELU, XF>, p, mK, mV, mQ, mO);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -1302,9 +1388,10 @@ bool fused_prep_fits(const ScanArgs& a) {
 }
 
 cudaError_t launch_fused(const ScanArgs& a, cudaStream_t st) {
-    if (a.has_prep) return launch_fused_mode<false, true>(a, st);     // GDN only
-    return a.mode == LA_MODE_RELU ? launch_fused_mode<true, false>(a, st)
-                                  : launch_fused_mode<false, false>(a, st);
+    if (a.has_prep) return launch_fused_mode<false, kXfPrep>(a, st);      // GDN only
+    if (a.beta_tok) return launch_fused_mode<false, kXfTokB>(a, st);      // GDN only
+    return a.mode == LA_MODE_RELU ? launch_fused_mode<true, kXfNone>(a, st)
+                                  : launch_fused_mode<false, kXfNone>(a, st);
 }
 
 }  // namespace la

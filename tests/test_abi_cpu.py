@@ -107,10 +107,14 @@ def test_reverse_scan_argument_errors_and_sizes():
     P = _fake
     ws = la.la_workspace_size(la.LA_MODE_GDN_REVERSE, 1, 1, 4, 16, 64)
     assert ws >= 256 and ws % 256 == 0
-    # the reversed scan never takes the fused path, so it needs per-frame buffers
-    assert la.la_workspace_size(la.LA_MODE_GDN_REVERSE, 1, 20, 181, 880, 128) > \
+    # few heads: the reversed scan runs in the single fused kernel, with the
+    # forward scan's per-head rings (no per-frame buffers)
+    assert la.la_workspace_size(la.LA_MODE_GDN_REVERSE, 1, 20, 181, 880, 128) == \
         la.la_workspace_size(la.LA_MODE_GDN, 1, 20, 181, 880, 128)
-    assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05", 24)
+    assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 1, 20, 181, 880, 128) == \
+        ("tcgen05_fused", 1)
+    # many heads: the three-kernel path with per-frame buffers
+    assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 4, 20, 64, 880, 128)[0] == "tcgen05"
     assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 1, 16, 512, 1024, 256)[0] == "simt_f32"
     args = lambda C, D=64, w=ws: (P(), P(), P(), P(), la.LA_BF16, P(), P(), 0.1, C,
                                   1, 1, 4, 16, D, P(), w, None)
@@ -127,7 +131,9 @@ def test_token_gate_scan_argument_errors_and_plan():
     P = _fake
     ws = la.la_workspace_size(la.LA_MODE_GDN_TOKEN_BETA, 1, 1, 4, 16, 64)
     assert ws >= 256 and ws % 256 == 0
-    assert la.la_plan(la.LA_MODE_GDN_TOKEN_BETA, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05", 24)
+    assert la.la_plan(la.LA_MODE_GDN_TOKEN_BETA, la.LA_BF16, 1, 20, 181, 880, 128) == \
+        ("tcgen05_fused", 1)
+    assert la.la_plan(la.LA_MODE_GDN_TOKEN_BETA, la.LA_BF16, 4, 20, 64, 880, 128)[0] == "tcgen05"
     assert la.la_plan(la.LA_MODE_GDN_TOKEN_BETA, la.LA_F32, 1, 2, 8, 64, 32)[0] == "simt_f32"
     assert la.la_workspace_size(7, 1, 1, 4, 16, 64) == 0      # no mode 7
     args = lambda bt=P(), D=64, w=ws: (P(), P(), P(), P(), la.LA_BF16, P(), bt, 0.1, None, None,
@@ -195,9 +201,11 @@ def test_python_binding_refuses_cpu_tensors():
 
 
 @pytest.mark.parametrize("F,chunks", [(8, 1), (31, 1), (32, 2), (40, 3), (181, 8), (512, 8)])
-def test_three_kernel_path_chunk_count(F, chunks):
+def test_three_kernel_path_chunk_count(F, chunks, monkeypatch):
     """Clips of 32+ frames with few heads run as a pipeline of frame chunks of
-    max(16, ceil(F / 8)) frames, three kernels per chunk (two without output)."""
+    max(16, ceil(F / 8)) frames, three kernels per chunk (two without output)
+    (LA_SCAN_NO_FUSE keeps few heads off the single-kernel path)."""
+    monkeypatch.setenv("LA_SCAN_NO_FUSE", "1")
     assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 1, 4, F, 64, 128) == ("tcgen05", 3 * chunks)
 
 
@@ -206,9 +214,10 @@ def test_three_kernel_pipeline_needs_free_sms():
     assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 4, 20, 64, 880, 128) == ("tcgen05", 3)
 
 
-def test_reversed_scan_chunks_align_with_pipeline_chunks():
+def test_reversed_scan_chunks_align_with_pipeline_chunks(monkeypatch):
     # F = 181 -> pipeline chunks of 23 frames, rounded up to whole 8-frame reversed
     # chunks (24 frames): 8 launches of three kernels
+    monkeypatch.setenv("LA_SCAN_NO_FUSE", "1")
     assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05", 24)
 
 

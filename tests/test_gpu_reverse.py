@@ -3,7 +3,8 @@
 
 Bars as for the forward scan: 1e-4 for float32 inputs, 2e-2 for bfloat16
 inputs (max|gpu - ref| / max|ref|).  bf16 heads with 64 <= D <= 128 run on
-the three-kernel tensor-core path, the rest on the SIMT kernel.
+the single-kernel tensor-core path (the three-kernel path for many heads),
+the rest on the SIMT kernel.
 """
 import numpy as np
 import pytest
@@ -65,7 +66,8 @@ def test_reverse_scan_matches_oracle(dtype, D, S, F, C):
 def test_reverse_scan_720p_gdn_all_heads():
     """The 720p 60 s GDN workload (B1 H20 D128 F181 S880) in chunks of 8 frames."""
     spec = synth.workload("gdn_720p_60s")
-    assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05", 24)
+    assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 1, 20, 181, 880, 128) == \
+        ("tcgen05_fused", 1)
     _compare(spec, 8)
 
 
@@ -94,3 +96,20 @@ def test_reverse_chunks_are_independent():
     assert not torch.equal(o1[:, :, 3].view(torch.int16), o2[:, :, 3].view(torch.int16))
     # inside the chunk {3, 4, 5} the reversed scan carries frame 4 back to frame 3, not on to 5
     assert torch.equal(o1[:, :, 5].view(torch.int16), o2[:, :, 5].view(torch.int16))
+
+
+@pytest.mark.parametrize("C", [1, 4, 8])
+def test_reverse_fused_kernel_matches_three_kernel_path(C, monkeypatch):
+    """The single-kernel path (chunk resets as a zero decay at each chunk's
+    first step) against the three-kernel path on the same inputs."""
+    spec = synth.small(B=2, H=3, F=13, S=250, D=128, dtype="bf16", seed=61 + C, keys_l2=True,
+                       alpha=("sigmoid_normal", 3.0, 1.0), beta=("sigmoid_normal", 0.0, 1.0))
+    assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 2, 3, 13, 250, 128)[0] == "tcgen05_fused"
+    inp = device_inputs(spec)
+    o_f = _run(spec, inp, C).clone()
+    monkeypatch.setenv("LA_SCAN_NO_FUSE", "1")
+    o_3 = _run(spec, inp, C)
+    torch.cuda.synchronize()
+    assert rel_err(to_np(o_f), to_np(o_3)) <= TOL_BF16
+    monkeypatch.delenv("LA_SCAN_NO_FUSE")
+    _compare(spec, C)

@@ -2,8 +2,9 @@
 (la_scan_gdn_token_beta) against the CPU oracle.
 
 Bars: 1e-4 for float32 inputs, 2e-2 for bfloat16 inputs.  bf16 heads with
-64 <= D <= 128 run on the three-kernel tensor-core path (K and V token rows
-scaled by sqrt(beta) in shared memory), the rest on the SIMT kernel.
+64 <= D <= 128 run on the single-kernel tensor-core path (the three-kernel
+path for many heads), K and V token rows scaled by sqrt(beta) in shared
+memory; the rest on the SIMT kernel.
 """
 import numpy as np
 import pytest
@@ -72,9 +73,8 @@ def test_token_gate_scan_matches_oracle(dtype, D, S, F):
 def test_token_gate_scan_720p_gdn_all_heads():
     """The 720p 60 s GDN workload with one update gate per token."""
     spec = synth.workload("gdn_720p_60s")
-    # eight pipeline chunks of 23 frames, three kernels each
     assert la.la_plan(la.LA_MODE_GDN_TOKEN_BETA, la.LA_BF16, 1, 20, 181, 880, 128) == \
-        ("tcgen05", 24)
+        ("tcgen05_fused", 1)
     _compare(spec)
 
 
@@ -98,3 +98,22 @@ def test_constant_token_gate_equals_frame_gate():
     o_f = la.la_scan_gdn(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"], spec.k_scale)
     torch.cuda.synchronize()
     assert rel_err(to_np(o_t), to_np(o_f)) <= TOL_BF16
+
+
+def test_token_gate_fused_kernel_matches_three_kernel_path(monkeypatch):
+    spec = synth.small(B=2, H=3, F=9, S=333, D=112, dtype="bf16", seed=67, keys_l2=True,
+                       alpha=("sigmoid_normal", 3.0, 1.0), beta=("sigmoid_normal", 0.0, 1.0))
+    assert la.la_plan(la.LA_MODE_GDN_TOKEN_BETA, la.LA_BF16, 2, 3, 9, 333, 112)[0] == \
+        "tcgen05_fused"
+    inp = device_inputs(spec)
+    btok = torch.from_numpy(synth.token_gates(spec)).cuda()
+    m0 = torch.from_numpy(synth.random_state(spec, 0.05)[0]).cuda()
+    o_f, m_f = _run(spec, inp, btok, m0)
+    o_f, m_f = o_f.clone(), m_f.clone()
+    monkeypatch.setenv("LA_SCAN_NO_FUSE", "1")
+    o_3, m_3 = _run(spec, inp, btok, m0)
+    torch.cuda.synchronize()
+    assert rel_err(to_np(o_f), to_np(o_3)) <= TOL_BF16
+    assert rel_err(to_np(m_f), to_np(m_3)) <= TOL_BF16
+    monkeypatch.delenv("LA_SCAN_NO_FUSE")
+    _compare(spec, with_state=True)
