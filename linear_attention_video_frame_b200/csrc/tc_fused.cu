@@ -762,9 +762,12 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
             const bool gram = it.type == kItemGram;
             const float* bsrc =
                 p.beta_tok + ((size_t)it.bh * F + step_frame(it.f, F, p.rev_chunk)) * p.S;
+            // the gates of a tile are fetched one tile ahead, off the critical path
+            float bv_next = (gram && row < p.S) ? __ldg(bsrc + row) : 0.f;
             for (int t = 0; t < (gram ? ntg : nto); ++t) {
-                const int tok = t * kTokG + row;
-                const float bv = (gram && tok < p.S) ? __ldg(bsrc + tok) : 0.f;   // before the wait
+                const float bv = bv_next;
+                const int tok_n = (t + 1) * kTokG + row;
+                bv_next = (gram && t + 1 < ntg && tok_n < p.S) ? __ldg(bsrc + tok_n) : 0.f;
                 if (leader) {
                     ok = ok && mbar_wait(&full[s], ph, ab, 0x452);
                     bc2[bcn & 1] = ok;
