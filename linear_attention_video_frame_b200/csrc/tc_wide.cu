@@ -109,10 +109,15 @@ __device__ __forceinline__ uint32_t quad_off(int row, int col) {
 // ============================================================================
 // gram: per-frame contractions over tokens, one key-row block per CTA
 // ============================================================================
-// warp 0: TMA producer; warp 1: TMEM owner + MMA issuer; warps 2-5: epilogue;
-// warps 6-9 (ReLU): phi(K) in place before the MMA.
+// warp 0: TMA producer; warp 1: TMEM owner + MMA issuer; warps 6-9 (ReLU):
+// phi(K) in place before the MMA; two epilogue groups of four warps (2-5, and
+// 6-9 or, with ReLU, 10-13) read out the two halves of the 512 accumulator
+// columns side by side (GDN: G'' and B~; ReLU: value columns 0-127 with dz,
+// and 128-255), so the next item's MMAs wait half as long for the TMEM.
+constexpr int wide_gram_threads(bool relu) { return relu ? 448 : 320; }
+
 template <bool RELU>
-__global__ void __launch_bounds__(RELU ? 320 : 192, 1)
+__global__ void __launch_bounds__(wide_gram_threads(RELU), 1)
 wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
                  const __grid_constant__ CUtensorMap mapV) {
     constexpr int kStages = 3;
@@ -138,7 +143,7 @@ wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
             mbar_init(&xform[s], 4);
         }
         mbar_init(accfull, 1);
-        mbar_init(accempty, 4);
+        mbar_init(accempty, 8);                            // both epilogue groups
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -228,64 +233,7 @@ wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
                 if (ok) mma_commit(accfull);
             }
         }
-    } else if (warp < 6) {
-        // ---------------- epilogue: TMEM -> workspace ----------------
-        const int q = warp & 3, row = q * 32 + lane;
-        int li = 0;
-        bool ok = true;
-        for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
-            const int frame = global_frame(p, item >> 1);
-            if (!(ok = mbar_wait(accfull, li & 1, ab, 0x604))) break;
-            tc_fence_after();
-            const uint32_t tl = tbase + (uint32_t(q * 32) << 16);
-            if (!RELU) {
-                const float al = p.alpha[frame], bt = p.beta[frame];
-                const float sg = -al * bt * p.k_scale * p.k_scale, sw = bt * p.k_scale;
-                // the G''[r] image goes straight from registers to its workspace slot
-                uint8_t* gi = p.gimg + (size_t)item * kGImg;
-                for (int c0 = 0; c0 < kDW; c0 += 16) {
-                    float v[16];
-                    tmem_ld16(tl + c0, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) v[e] *= sg;
-                    store_row16(gi, 16384, row, c0, v);
-                }
-                for (int c0 = 0; c0 < kDW; c0 += 16) {
-                    float v[16];
-                    tmem_ld16(tl + 256 + c0, v);
-                    tmem_wait_ld();
-                    uint4* bt = p.btil + ((size_t)item * 2 + (c0 >> 7)) * kBTile;
-                    const int jc = (c0 & 127) >> 3;
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        bt[(jc + h) * 128 + row] = make_uint4(
-                            pack_bf16x2(v[8 * h] * sw, v[8 * h + 1] * sw),
-                            pack_bf16x2(v[8 * h + 2] * sw, v[8 * h + 3] * sw),
-                            pack_bf16x2(v[8 * h + 4] * sw, v[8 * h + 5] * sw),
-                            pack_bf16x2(v[8 * h + 6] * sw, v[8 * h + 7] * sw));
-                }
-            } else {
-                float* bq = p.bmat + (size_t)item * kQuad;
-                for (int c0 = 0; c0 < kDW; c0 += 16) {
-                    float v[16];
-                    tmem_ld16(tl + c0, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        *reinterpret_cast<float4*>(bq + quad_off(row, c0 + 4 * u)) =
-                            make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
-                }
-                float v[16];
-                tmem_ld16(tl + 256, v);
-                tmem_wait_ld();
-                p.dz[(size_t)item * 128 + row] = v[0];
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(accempty);
-        }
-    } else {
+    } else if (RELU && warp >= 6 && warp < 10) {
         // ---------------- ReLU transform: phi(K) in place ----------------
         const int tl = threadIdx.x - 192;          // 0..127
         int s = 0;
@@ -306,6 +254,66 @@ wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
                 if (lane == 0) mbar_arrive(&xform[s]);
                 if (++s == kStages) { s = 0; ph ^= 1; }
             }
+        }
+    } else {
+        // ---------------- epilogue: TMEM -> workspace, two groups ----------------
+        const int q = warp & 3, row = q * 32 + lane;
+        const int g = warp < 6 ? 0 : 1;                 // half of the accumulator columns
+        int li = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
+            const int frame = global_frame(p, item >> 1);
+            if (!(ok = mbar_wait(accfull, li & 1, ab, 0x604))) break;
+            tc_fence_after();
+            const uint32_t tl = tbase + (uint32_t(q * 32) << 16);
+            if (!RELU) {
+                const float al = p.alpha[frame], bt = p.beta[frame];
+                const float sg = -al * bt * p.k_scale * p.k_scale, sw = bt * p.k_scale;
+                // the G''[r] image goes straight from registers to its workspace slot
+                uint8_t* gi = p.gimg + (size_t)item * kGImg;
+                for (int c0 = 0; c0 < kDW && g == 0; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tl + c0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] *= sg;
+                    store_row16(gi, 16384, row, c0, v);
+                }
+                for (int c0 = 0; c0 < kDW && g == 1; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tl + 256 + c0, v);
+                    tmem_wait_ld();
+                    uint4* bt = p.btil + ((size_t)item * 2 + (c0 >> 7)) * kBTile;
+                    const int jc = (c0 & 127) >> 3;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        bt[(jc + h) * 128 + row] = make_uint4(
+                            pack_bf16x2(v[8 * h] * sw, v[8 * h + 1] * sw),
+                            pack_bf16x2(v[8 * h + 2] * sw, v[8 * h + 3] * sw),
+                            pack_bf16x2(v[8 * h + 4] * sw, v[8 * h + 5] * sw),
+                            pack_bf16x2(v[8 * h + 6] * sw, v[8 * h + 7] * sw));
+                }
+            } else {
+                float* bq = p.bmat + (size_t)item * kQuad;
+                for (int c0 = 128 * g; c0 < 128 * g + 128; c0 += 16) {
+                    float v[16];
+                    tmem_ld16(tl + c0, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        *reinterpret_cast<float4*>(bq + quad_off(row, c0 + 4 * u)) =
+                            make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                }
+                if (g == 0) {
+                    float v[16];
+                    tmem_ld16(tl + 256, v);
+                    tmem_wait_ld();
+                    p.dz[(size_t)item * 128 + row] = v[0];
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(accempty);
         }
     }
     tc_fence_before();
@@ -567,47 +575,56 @@ wide_chain_relu_kernel(const WideParams p) {
 }
 
 // ============================================================================
-// output: O_f[:, c] = Q~_f bf16(M_f)[:, c]   (ReLU: / (phi(Q_f) z_f + eps))
+// output: O_f = Q~_f bf16(M_f)   (ReLU: / (phi(Q_f) z_f + eps))
 // ============================================================================
-// warp 0: producer (M image and z by bulk copy, Q tiles by TMA); warp 1: TMEM
-// owner + MMA issuer; warps 2-5: epilogue (TMEM -> bf16 staging -> TMA store,
-// one 64-column box at a time, kOStg staging buffers); warps 6-9 (ReLU):
-// phi(Q) in place and the per-token denominators.
+// One CTA item per (b, h, f) computes all 256 value columns: the whole
+// bf16(M_f) image (128 KB, both value halves) sits in shared memory, Q is
+// streamed in 64-column boxes of 128-token tiles (kQS-stage ring), and each
+// box feeds four N = 256 MMAs into one of two 256-column TMEM accumulators.
+// Q is read once per frame, and the ReLU feature map and denominators are
+// formed once per token.
+// warp 0: producer (the first Q boxes of an item, then its M image (+ z) by
+// bulk copy once the previous item's MMAs are done, then the other boxes);
+// warp 1: TMEM owner + MMA issuer; warps 2-5: epilogue (TMEM -> bf16 ->
+// TMA store, one 64-column box at a time); warps 6-9 (ReLU): phi(Q) in place
+// and the per-token denominators.
+constexpr int kQS = 3;                        // Q box ring stages (16 KB each)
+constexpr int kOutStg = 2;                    // epilogue staging boxes (16 KB each)
+
 template <bool RELU>
 __global__ void __launch_bounds__(RELU ? 320 : 192, 1)
 wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
                    const __grid_constant__ CUtensorMap mapO) {
-    constexpr int kOStg = RELU ? 1 : 2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
-    uint8_t* qring = smem;                                 // 2 x 64 KB Q tiles
-    uint8_t* mbuf = qring + 2 * kOTile;                    // M[:, c] image (64 KB)
-    uint8_t* ostage = mbuf + kMImg;                        // kOStg x 16 KB output boxes
-    float* zbuf = reinterpret_cast<float*>(ostage + kOStg * kBoxO);   // 256 (ReLU)
-    float* denbuf = zbuf + (RELU ? 256 : 0);                          // kOAcc x 128 (ReLU)
-    uint64_t* qfull = reinterpret_cast<uint64_t*>(denbuf + (RELU ? kOAcc * 128 : 0));
-    uint64_t* qempty = qfull + 2;
-    uint64_t* xform = qempty + 2;
-    uint64_t* mfull = xform + 2;
+    uint8_t* mbuf = smem;                                  // bf16(M_f) image, 2 x kMImg
+    uint8_t* qring = mbuf + 2 * kMImg;                     // kQS x 16 KB Q boxes
+    uint8_t* ostage = qring + kQS * kBoxO;                 // kOutStg x 16 KB output boxes
+    float* zbuf = reinterpret_cast<float*>(ostage + kOutStg * kBoxO);   // 256 (ReLU)
+    float* denbuf = zbuf + 256;                            // 2 x 128 (ReLU)
+    uint64_t* qfull = reinterpret_cast<uint64_t*>(denbuf + 256);
+    uint64_t* qempty = qfull + kQS;
+    uint64_t* xform = qempty + kQS;
+    uint64_t* mfull = xform + kQS;
     uint64_t* mempty = mfull + 1;
-    uint64_t* accfull = mempty + 1;
-    uint64_t* accempty = accfull + kOAcc;
-    uint64_t* denready = accempty + kOAcc;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(denready + kOAcc);
+    uint64_t* accfull = mempty + 1;                        // [2]
+    uint64_t* accempty = accfull + 2;                      // [2]
+    uint64_t* denready = accempty + 2;                     // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(denready + 2);
     uint32_t* abort_flag = tmem_slot + 1;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int D = p.D;
-    const int nbx = (D + 63) / 64;
+    const int nbx = (D + 63) / 64;                         // Q boxes per tile (3 or 4)
     if (threadIdx.x == 0) {
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kQS; ++s) {
             mbar_init(&qfull[s], 1);
             mbar_init(&qempty[s], 1);
             mbar_init(&xform[s], 4);
         }
         mbar_init(mfull, 1);
-        mbar_init(mempty, RELU ? 5 : 1);
-        for (int a = 0; a < kOAcc; ++a) {
+        mbar_init(mempty, 1);
+        for (int a = 0; a < 2; ++a) {
             mbar_init(&accfull[a], 1);
             mbar_init(&accempty[a], 4);
             mbar_init(&denready[a], 4);
@@ -615,22 +632,16 @@ wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
         *abort_flag = 0;
         fence_mbar_init();
     }
-    for (int s = 0; s < 2; ++s)
-        for (int b = nbx; b < 4; ++b) {
-            uint4* z = reinterpret_cast<uint4*>(qring + s * kOTile + b * kBoxO);
-            for (int i = threadIdx.x; i < (int)(kBoxO / 16); i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
-        }
     if (warp == 1) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
     const Abort ab{abort_flag, p.status};
-    const int nitems = p.BH * p.Fc * 2;
+    const int nitems = p.BH * p.Fc;
     const int nt = (p.S + kTokO - 1) / kTokO;
 
     if (warp == 0) {
@@ -642,44 +653,54 @@ wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
             uint32_t ph = 0;
             bool ok = true;
             for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
-                const int frame = global_frame(p, item >> 1);
-                if (!(ok = mbar_wait(mempty, (li & 1) ^ 1, ab, 0x801))) break;
-                mbar_expect_tx(mfull, kMImg + (RELU ? 1024 : 0));
-                bulk_load(mbuf, p.mimg + (size_t)item * kMImg, kMImg, mfull);
-                if (RELU) bulk_load(zbuf, p.zf + (size_t)(item >> 1) * 256, 1024, mfull);
-                for (int t = 0; t < nt; ++t) {
-                    if (!(ok = mbar_wait(&qempty[s], ph ^ 1, ab, 0x802))) break;
-                    uint8_t* st = qring + s * kOTile;
-                    mbar_expect_tx(&qfull[s], nbx * kBoxO);
-                    for (int b = 0; b < nbx; ++b)
-                        tma_load_3d(st + b * kBoxO, &mapQ, &qfull[s], 64 * b, t * kTokO, frame, pol);
-                    if (++s == 2) { s = 0; ph ^= 1; }
-                }
+                const int frame = global_frame(p, item);
+                const int nq = nt * nbx;                   // Q boxes of the item
+                auto load_q = [&](int g) {                 // box g = tile g / nbx, column box g % nbx
+                    if (!(ok = ok && mbar_wait(&qempty[s], ph ^ 1, ab, 0x802))) return;
+                    mbar_expect_tx(&qfull[s], kBoxO);
+                    tma_load_3d(qring + s * kBoxO, &mapQ, &qfull[s], 64 * (g % nbx),
+                                (g / nbx) * kTokO, frame, pol);
+                    if (++s == kQS) { s = 0; ph ^= 1; }
+                };
+                const int early = min(nq, kQS);
+                for (int g = 0; g < early; ++g) load_q(g);
+                // the image buffer is free once the previous item's MMAs are done
+                ok = ok && mbar_wait(mempty, (li & 1) ^ 1, ab, 0x801);
+                if (!ok) break;
+                mbar_expect_tx(mfull, 2 * kMImg + (RELU ? 1024 : 0));
+                bulk_load(mbuf, p.mimg + (size_t)item * 2 * kMImg, 2 * kMImg, mfull);
+                if (RELU) bulk_load(zbuf, p.zf + (size_t)item * 256, 1024, mfull);
+                for (int g = early; g < nq; ++g) load_q(g);
             }
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            const uint32_t idO = idesc_bf16(128, 128, false, true);
+            const uint32_t idO = idesc_bf16(128, kDW, false, true);
             const uint32_t mb = smem_u32(mbuf);
             int s = 0, li = 0, gt = 0;
             uint32_t ph = 0;
             bool ok = true;
             for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
                 if (!(ok = mbar_wait(mfull, li & 1, ab, 0x803))) break;
-                for (int t = 0; t < nt; ++t, ++gt) {
-                    const int a = gt % kOAcc;
-                    if (!(ok = mbar_wait(&accempty[a], ((gt / kOAcc) & 1) ^ 1, ab, 0x804))) break;
-                    if (!(ok = mbar_wait(RELU ? &xform[s] : &qfull[s], ph, ab, 0x805))) break;
+                tc_fence_after();
+                for (int t = 0; t < nt && ok; ++t, ++gt) {
+                    const int a = gt & 1;
+                    if (!(ok = mbar_wait(&accempty[a], ((gt >> 1) & 1) ^ 1, ab, 0x804))) break;
                     tc_fence_after();
-                    const uint32_t qa = smem_u32(qring + s * kOTile);
-                    for (int kk = 0; kk < 4 * nbx; ++kk) {
-                        const uint64_t ad = sdesc_sw128(qa + (kk >> 2) * kBoxO + (kk & 3) * 32, 16, 1024);
-                        const uint64_t bd = sdesc_sw128(mb + kk * 2048, 32768, 1024);
-                        mma_bf16(tbase + a * 128, ad, bd, idO, kk > 0 ? 1u : 0u);
+                    for (int b = 0; b < nbx; ++b) {
+                        if (!(ok = mbar_wait(RELU ? &xform[s] : &qfull[s], ph, ab, 0x805))) break;
+                        tc_fence_after();
+                        const uint32_t qa = smem_u32(qring + s * kBoxO);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t ad = sdesc_sw128(qa + kk * 32, 16, 1024);
+                            const uint64_t bd = sdesc_sw128(mb + (4 * b + kk) * 2048, 32768, 1024);
+                            mma_bf16(tbase + a * 256, ad, bd, idO, (b | kk) ? 1u : 0u);
+                        }
+                        mma_commit(&qempty[s]);
+                        if (++s == kQS) { s = 0; ph ^= 1; }
                     }
-                    mma_commit(&qempty[s]);
-                    mma_commit(&accfull[a]);
-                    if (++s == 2) { s = 0; ph ^= 1; }
+                    if (ok) mma_commit(&accfull[a]);
                 }
                 if (ok) mma_commit(mempty);
             }
@@ -691,19 +712,17 @@ wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
         int gt = 0, gb = 0;
         bool ok = true;     // every epilogue warp runs every named barrier, even after an abort
         for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
-            const int frame = global_frame(p, item >> 1), c = item & 1;
+            const int frame = global_frame(p, item);
             for (int t = 0; t < nt; ++t, ++gt) {
-                const int a = gt % kOAcc;
-                ok = ok && mbar_wait(&accfull[a], (gt / kOAcc) & 1, ab, 0x806);
-                if (RELU) ok = ok && mbar_wait(&denready[a], (gt / kOAcc) & 1, ab, 0x807);
+                const int a = gt & 1;
+                ok = ok && mbar_wait(&accfull[a], (gt >> 1) & 1, ab, 0x806);
+                if (RELU) ok = ok && mbar_wait(&denready[a], (gt >> 1) & 1, ab, 0x807);
                 tc_fence_after();
                 const float inv = (RELU && ok) ? 1.f / denbuf[a * 128 + row] : 1.f;
-                const uint32_t tl = tbase + (uint32_t(q * 32) << 16) + a * 128;
-                for (int b = 0; b < 2; ++b, ++gb) {
-                    const int x0 = 128 * c + 64 * b;
-                    if (x0 >= D) break;                       // uniform over the block
-                    uint8_t* os = ostage + (gb % kOStg) * kBoxO;
-                    if (issuer) bulk_wait_read<kOStg - 1>();  // this staging buffer is free
+                const uint32_t tl = tbase + (uint32_t(q * 32) << 16) + a * 256;
+                for (int b = 0; b < nbx; ++b, ++gb) {
+                    uint8_t* os = ostage + (gb % kOutStg) * kBoxO;
+                    if (issuer) bulk_wait_read<kOutStg - 1>();   // this staging box is free
                     named_bar_sync(1, 128);
                     for (int c0 = 0; c0 < 64 && ok; c0 += 16) {
                         float v[16];
@@ -715,16 +734,18 @@ wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
                         }
                         store_row16(os, 16384, row, c0, v);
                     }
+                    if (b == nbx - 1) {                   // the accumulator is read out
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&accempty[a]);
+                    }
                     fence_proxy_async_smem();
                     named_bar_sync(1, 128);
                     if (issuer && ok) {
-                        tma_store_3d(&mapO, os, x0, t * kTokO, frame);
+                        tma_store_3d(&mapO, os, 64 * b, t * kTokO, frame);
                         bulk_commit();
                     }
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&accempty[a]);
             }
         }
         if (issuer) bulk_wait_all<0>();
@@ -736,15 +757,16 @@ wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
         bool ok = true;
         for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
             if (!(ok = mbar_wait(mfull, li & 1, ab, 0x808))) break;
-            for (int t = 0; t < nt; ++t, ++gt) {
-                const int a = gt % kOAcc;
-                if (!(ok = mbar_wait(&qfull[s], ph, ab, 0x809))) break;
-                if (!(ok = mbar_wait(&accempty[a], ((gt / kOAcc) & 1) ^ 1, ab, 0x80a))) break;
-                uint8_t* st = qring + s * kOTile;
+            for (int t = 0; t < nt && ok; ++t, ++gt) {
+                const int a = gt & 1;
+                // denbuf[a] is free once the epilogue has read this accumulator's last use
+                if (!(ok = mbar_wait(&accempty[a], ((gt >> 1) & 1) ^ 1, ab, 0x80a))) break;
                 float den = 0.f;
                 for (int b = 0; b < nbx; ++b) {
+                    if (!(ok = mbar_wait(&qfull[s], ph, ab, 0x809))) break;
+                    uint8_t* st = qring + s * kBoxO;
                     for (int ch = 0; ch < 8; ++ch) {
-                        uint4* pch = reinterpret_cast<uint4*>(st + b * kBoxO + sw128_off(row, ch));
+                        uint4* pch = reinterpret_cast<uint4*>(st + sw128_off(row, ch));
                         uint4 x = *pch;
                         x.x = relu_bf16x2(x.x); x.y = relu_bf16x2(x.y);
                         x.z = relu_bf16x2(x.z); x.w = relu_bf16x2(x.w);
@@ -759,18 +781,16 @@ wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
                         den = fmaf(bf16_lo(x.w), zz[6], den);
                         den = fmaf(bf16_hi(x.w), zz[7], den);
                     }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&xform[s]);
+                    if (++s == kQS) { s = 0; ph ^= 1; }
                 }
+                if (!ok) break;
                 denbuf[a * 128 + row] = den + p.eps;
-                fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&xform[s]);
-                    mbar_arrive(&denready[a]);
-                }
-                if (++s == 2) { s = 0; ph ^= 1; }
+                if (lane == 0) mbar_arrive(&denready[a]);
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(mempty);
         }
     }
     tc_fence_before();
@@ -845,8 +865,7 @@ constexpr size_t kSmemWideGram = 1024 + 3 * 2 * kGTile + 2048 + 256;
 constexpr size_t kSmemWideChain = 1024 + 2 * kGImg + kMImg + 256;
 template <bool RELU>
 constexpr size_t smem_wide_out() {
-    return 1024 + 2 * kOTile + kMImg + (RELU ? 1 : 2) * kBoxO + (RELU ? 1024 + kOAcc * 512 : 0) +
-           256;
+    return 1024 + 2 * kMImg + kQS * kBoxO + kOutStg * kBoxO + 1024 + 1024 + 256;
 }
 static_assert(kSmemWideGram <= 232448, "gram smem");
 static_assert(kSmemWideChain <= 232448, "chain smem");
@@ -963,7 +982,7 @@ cudaError_t launch_wide_mode(const ScanArgs& a, cudaStream_t st) {
         const int grid = std::min(items, share);
         // gram(c) overwrites the buffers chain(c - 2) read
         if (ci >= 2) ok(cudaStreamWaitEvent(st, cx.chain[b], 0));
-        wide_gram_kernel<RELU><<<grid, thr, kSmemWideGram, st>>>(p, mK, mV);
+        wide_gram_kernel<RELU><<<grid, wide_gram_threads(RELU), kSmemWideGram, st>>>(p, mK, mV);
         ok(cudaGetLastError());
         ok(cudaEventRecord(cx.gram[b], st));
         // chain(c) needs gram(c), and overwrites the images output(c - 2) read
@@ -977,7 +996,8 @@ cudaError_t launch_wide_mode(const ScanArgs& a, cudaStream_t st) {
         ok(cudaEventRecord(cx.chain[b], s_chain));
         if (p.want_output) {
             ok(cudaStreamWaitEvent(s_out, cx.chain[b], 0));
-            wide_output_kernel<RELU><<<grid, thr, smem_wide_out<RELU>(), s_out>>>(p, mQ, mO);
+            const int grid_o = std::min(p.BH * p.Fc, share);     // one item per frame
+            wide_output_kernel<RELU><<<grid_o, thr, smem_wide_out<RELU>(), s_out>>>(p, mQ, mO);
             ok(cudaGetLastError());
             ok(cudaEventRecord(cx.out[b], s_out));
         }
