@@ -53,6 +53,9 @@ WORKLOADS = {
     "gdn_720p_60s_reverse8": ("gdn_720p_60s", "gdn_reverse"),
     # per-token update gate on the 720p 60 s clip
     "gdn_720p_60s_token_beta": ("gdn_720p_60s", "gdn_token_beta"),
+    # the same two variants on the stress workload's 256-wide heads
+    "stress_gdn_reverse8": ("stress_d256", "gdn_reverse"),
+    "stress_gdn_token_beta": ("stress_d256", "gdn_token_beta"),
     # raw q, k with RMSNorm, ReLU and 3D RoPE fused into the scan (22 x 40 grid)
     "gdn_720p_60s_prep": ("gdn_720p_60s_raw", "gdn_prep"),
     "tiny_gdn": ("tiny_fp32", "gdn"),
@@ -116,17 +119,17 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-# Sources the dominant (fused) kernel is compiled from.
+# Sources the kernels of a path are compiled from (a traffic record names its own).
 KERNEL_SOURCES = ("tc_fused.cu", "tc_common.cuh", "tmap.cuh", "common.cuh")
 
 
-def kernel_source_hash() -> str:
-    """Hash of the fused kernel's sources, so a committed DRAM-traffic figure
-    is used only while the kernel it was measured on is unchanged.  Lines of
-    the optional event trace are left out: without -DLA_TRACE they compile
-    to nothing."""
+def kernel_source_hash(sources=KERNEL_SOURCES) -> str:
+    """Hash of a kernel's sources, so a committed DRAM-traffic figure is used
+    only while the kernel it was measured on is unchanged.  Lines of the
+    optional event trace are left out: without -DLA_TRACE they compile to
+    nothing."""
     h = hashlib.sha256()
-    for name in KERNEL_SOURCES:
+    for name in sources:
         p = os.path.join(ROOT, "linear_attention_video_frame_b200", "csrc", name)
         for line in open(p, "rb").read().splitlines(keepends=True):
             if b"LA_TRACE" not in line:
@@ -144,7 +147,8 @@ def traffic_record(workload: str):
         d = json.load(open(p)).get(workload)
     except Exception:
         return None
-    if not d or d.get("kernel_source_hash") != kernel_source_hash():
+    if not d or d.get("kernel_source_hash") != kernel_source_hash(
+            tuple(d.get("sources", KERNEL_SOURCES))):
         return None
     return d.get("dram_bytes_per_launch")
 
@@ -180,7 +184,7 @@ class ClockSampler:
     }
 
     def __init__(self, index: int, period_s: float = 0.001):
-        self.samples, self.stamps, self.reasons, self.max_mhz = [], [], 0, None
+        self.samples, self.stamps, self.bits, self.reasons, self.max_mhz = [], [], [], 0, None
         self.period = period_s
         self._stop = threading.Event()
         self._thr = None
@@ -198,8 +202,10 @@ class ClockSampler:
         while not self._stop.is_set():
             try:
                 mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
-                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                bits = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.reasons |= bits
                 self.samples.append(mhz)
+                self.bits.append(bits)
                 self.stamps.append(time.perf_counter())
             except Exception:
                 pass
@@ -218,6 +224,14 @@ class ClockSampler:
     def between(self, t0: float, t1: float):
         """SM clock samples taken between host times t0 and t1."""
         return [m for m, t in zip(self.samples, self.stamps) if t0 <= t <= t1]
+
+    def reasons_between(self, t0: float, t1: float):
+        """Names of the throttle reasons seen between host times t0 and t1."""
+        acc = 0
+        for b, t in zip(self.bits, self.stamps):
+            if t0 <= t <= t1:
+                acc |= b
+        return [n for bit, n in self.REASONS.items() if acc & bit and n != "gpu_idle"]
 
     def summary(self):
         if not self.nv:
@@ -465,7 +479,8 @@ def run_ours(args):
             med = statistics.median(mhz) if mhz else None
             drift.append({"block": blk, "calls": args.drift_calls, "ms_per_call": ms,
                           "sm_mhz_median": med, "sm_mhz_min": min(mhz) if mhz else None,
-                          "samples": len(mhz), "ms_x_ghz": ms * med / 1e3 if med else None})
+                          "samples": len(mhz), "ms_x_ghz": ms * med / 1e3 if med else None,
+                          "reasons": dclk.reasons_between(h0, h1)})
         dclk.stop()
         barrier()
 

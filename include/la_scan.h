@@ -177,8 +177,8 @@ LA_API la_status la_scan_gdn(const void* q, const void* k, const void* v, void* 
  * Arguments and layouts are those of la_scan_gdn, without state in or out;
  * chunk_frames >= 1 (chunk_frames >= F reverses the whole clip).  The
  * workspace is la_workspace_size(LA_MODE_GDN_REVERSE, B, H, F, S, D) bytes.
- * bf16 inputs with 64 <= D <= 128 run on the tensor-core path; other
- * shapes on the float32 SIMT kernel.
+ * bf16 inputs with 64 <= D <= 256 run on tensor cores (a chunk start is a
+ * zero decay at that scan step); other shapes on the float32 SIMT kernel.
  */
 LA_API la_status la_scan_gdn_reverse(const void* q, const void* k, const void* v, void* o,
                                      la_dtype dt, const float* alpha, const float* beta,
@@ -200,9 +200,9 @@ LA_API la_status la_scan_gdn_reverse(const void* q, const void* k, const void* v
  *                  frame f); alpha [B,H,F] as for la_scan_gdn.
  * Everything else as for la_scan_gdn.  The workspace is
  * la_workspace_size(LA_MODE_GDN_TOKEN_BETA, B, H, F, S, D) bytes.  bf16
- * inputs with 64 <= D <= 128 run on the tensor-core path (each token row of
- * K and V is scaled by sqrt(beta) in shared memory, in bf16, before the
- * unchanged contractions); other shapes on the float32 SIMT kernel.
+ * inputs with 64 <= D <= 256 run on tensor cores (each token row of K and V
+ * is scaled by sqrt(beta) in shared memory, in bf16, before the unchanged
+ * contractions); other shapes on the float32 SIMT kernel.
  */
 LA_API la_status la_scan_gdn_token_beta(const void* q, const void* k, const void* v, void* o,
                                         la_dtype dt, const float* alpha,

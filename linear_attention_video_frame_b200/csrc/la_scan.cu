@@ -66,7 +66,15 @@ bool special(const ScanArgs& a) {
     return a.rev_chunk != 0 || a.beta_tok != nullptr || a.trans_out != nullptr || a.has_prep;
 }
 
-bool use_wide(const ScanArgs& a) { return !force_simt() && !special(a) && wide_eligible(a); }
+// The wide path also takes the reversed scan (its chunk resets are a zero decay
+// at each chunk's first step, so its pipeline chunks need not align) and the
+// per-token gate (sqrt(beta) row scaling in the gram kernel), GDN only.
+bool use_wide(const ScanArgs& a) {
+    if (force_simt() || !wide_eligible(a)) return false;
+    if (a.rev_chunk || a.beta_tok)     // reversed scan, per-token gate (GDN)
+        return a.mode == LA_MODE_GDN && !(a.rev_chunk && a.beta_tok) && !a.trans_out && !a.has_prep;
+    return !special(a);
+}
 
 // LA_SCAN_NO_FUSE=1 keeps tensor-core calls on the three-kernel path (tests
 // compare the two).

@@ -77,15 +77,25 @@ struct WideParams {
     float k_scale;
     float eps;
     int BH, F, S, D;        // F: frames of the clip (global frame index = bh F + f)
-    int f0, Fc;             // this launch covers frames [f0, f0 + Fc) of every head
+    int f0, Fc;             // this launch covers scan steps [f0, f0 + Fc) of every head
     int want_output;
+    int rev_chunk;          // > 0: reversed GDN scan reset every rev_chunk frames
+    const float* beta_tok;  // per-token update gate [BH][F][S] (TOKB gram), or NULL
 };
 
-// Global frame index (into q, k, v, o, alpha, beta) of chunk-local frame
-// `loc` = bh * Fc + fl; per-frame workspace buffers are indexed by `loc`.
+// Global frame index (into q, k, v, o, alpha, beta) of chunk-local scan step
+// `loc` = bh * Fc + fl (step f0 + fl covers frame step_frame(f0 + fl)); per-step
+// workspace buffers are indexed by `loc`.
 __device__ __forceinline__ int global_frame(const WideParams& p, int loc) {
     const int bh = loc / p.Fc;
-    return bh * p.F + p.f0 + (loc - bh * p.Fc);
+    return bh * p.F + step_frame(p.f0 + (loc - bh * p.Fc), p.F, p.rev_chunk);
+}
+
+// Decay of chunk-local step `loc`: zero where the reversed scan starts a chunk,
+// which makes G'' zero and restarts the carried state.
+__device__ __forceinline__ float step_alpha(const WideParams& p, int loc) {
+    const int bh = loc / p.Fc;
+    return step_resets(p.f0 + (loc - bh * p.Fc), p.rev_chunk) ? 0.f : p.alpha[global_frame(p, loc)];
 }
 
 // Write 16 consecutive columns [c0, c0 + 16) of row `row` of a swizzled bf16
@@ -114,10 +124,13 @@ __device__ __forceinline__ uint32_t quad_off(int row, int col) {
 // 6-9 or, with ReLU, 10-13) read out the two halves of the 512 accumulator
 // columns side by side (GDN: G'' and B~; ReLU: value columns 0-127 with dz,
 // and 128-255), so the next item's MMAs wait half as long for the TMEM.
-constexpr int wide_gram_threads(bool relu) { return relu ? 448 : 320; }
+// With the per-token update gate (TOKB, GDN), warps 6-9 scale every K and V
+// token row of a tile by sqrt(beta_t) in shared memory (packed bf16) before
+// the unchanged MMAs, which then give Kh^T diag(beta) Kh and Kh^T diag(beta) V.
+constexpr int wide_gram_threads(bool xf) { return xf ? 448 : 320; }
 
-template <bool RELU>
-__global__ void __launch_bounds__(wide_gram_threads(RELU), 1)
+template <bool RELU, bool TOKB = false>
+__global__ void __launch_bounds__(wide_gram_threads(RELU || TOKB), 1)
 wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
                  const __grid_constant__ CUtensorMap mapV) {
     constexpr int kStages = 3;
@@ -209,7 +222,7 @@ wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
                 if (!(ok = mbar_wait(accempty, (li & 1) ^ 1, ab, 0x602))) break;
                 tc_fence_after();
                 for (int t = 0; t < nt; ++t) {
-                    if (!(ok = mbar_wait(RELU ? &xform[s] : &full[s], ph, ab, 0x603))) break;
+                    if (!(ok = mbar_wait((RELU || TOKB) ? &xform[s] : &full[s], ph, ab, 0x603))) break;
                     tc_fence_after();
                     const uint32_t sk = smem_u32(ring + s * 2 * kGTile), sv = sk + kGTile;
 #pragma unroll
@@ -231,6 +244,39 @@ wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
                     if (++s == kStages) { s = 0; ph ^= 1; }
                 }
                 if (ok) mma_commit(accfull);
+            }
+        }
+    } else if (TOKB && warp >= 6 && warp < 10) {
+        // ---------------- per-token gate: sqrt(beta_t) on the K and V rows ----------------
+        const int tl = threadIdx.x - 192;          // 0..127: row tl % 64 of K (tl < 64) or V
+        const int row = tl & 63;
+        const int nch = (D + 7) / 8;
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x) {
+            const float* bsrc = p.beta_tok + (size_t)global_frame(p, item >> 1) * p.S;
+            float bv_next = row < p.S ? __ldg(bsrc + row) : 0.f;    // gates one tile ahead
+            for (int t = 0; t < nt; ++t) {
+                const float bv = bv_next;
+                const int tok_n = (t + 1) * kTokG + row;
+                bv_next = (t + 1 < nt && tok_n < p.S) ? __ldg(bsrc + tok_n) : 0.f;
+                if (!(ok = mbar_wait(&full[s], ph, ab, 0x606))) break;
+                const float sb = sqrtf(fmaxf(bv, 0.f));
+                const __nv_bfloat162 g = __floats2bfloat162_rn(sb, sb);
+                uint8_t* const base = ring + s * 2 * kGTile + (tl >> 6) * kGTile;
+                for (int c = 0; c < nch; ++c) {
+                    uint4* pc = reinterpret_cast<uint4*>(base + (c >> 3) * kBoxG + sw128_off(row, c & 7));
+                    uint4 x = *pc;
+                    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&x);
+                    h[0] = __hmul2(h[0], g); h[1] = __hmul2(h[1], g);
+                    h[2] = __hmul2(h[2], g); h[3] = __hmul2(h[3], g);
+                    *pc = x;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&xform[s]);
+                if (++s == kStages) { s = 0; ph ^= 1; }
             }
         }
     } else if (RELU && warp >= 6 && warp < 10) {
@@ -267,7 +313,7 @@ wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
             tc_fence_after();
             const uint32_t tl = tbase + (uint32_t(q * 32) << 16);
             if (!RELU) {
-                const float al = p.alpha[frame], bt = p.beta[frame];
+                const float al = step_alpha(p, item >> 1), bt = TOKB ? 1.f : p.beta[frame];
                 const float sg = -al * bt * p.k_scale * p.k_scale, sw = bt * p.k_scale;
                 // the G''[r] image goes straight from registers to its workspace slot
                 uint8_t* gi = p.gimg + (size_t)item * kGImg;
@@ -412,10 +458,11 @@ wide_chain_gdn_kernel(const WideParams p) {
         const bool leader = ((threadIdx.x - 64) & 127) == 0;
         const int bar_id = 1 + r;
         const uint32_t tl = tM + (uint32_t(q * 32) << 16) + r * 128;
-        const float* ap = p.alpha + (size_t)bh * p.F + p.f0;
+        // decay of this head's chunk-local step f (the chunk has F = Fc steps)
+        auto alpha_at = [&](int f) { return step_alpha(p, bh * F + f); };
         // initial state: image of M_0 and alpha_0 M_0 in TMEM
         {
-            const float a0 = __ldg(ap);
+            const float a0 = alpha_at(0);
             for (int j0 = 0; j0 < 128; j0 += 16) {
                 float v[16];
 #pragma unroll
@@ -447,7 +494,7 @@ wide_chain_gdn_kernel(const WideParams p) {
         bool ok = true;
         for (int f = 0; f < F; ++f) {
             const bool more = f + 1 < F;
-            const float an = more ? __ldg(ap + f + 1) : 1.f;
+            const float an = more ? alpha_at(f + 1) : 1.f;
             if (leader) {
                 ok = ok && mbar_wait(mdone, f & 1, ab, 0x704);
                 if (f >= 1) ok = ok && mbar_wait(ipub, (f - 1) & 1, ab, 0x705);
@@ -903,6 +950,8 @@ cudaError_t launch_wide_mode(const ScanArgs& a, cudaStream_t st) {
     uint8_t* ws = reinterpret_cast<uint8_t*>(a.ws);
     WideParams p;
     p.alpha = a.alpha;
+    p.rev_chunk = a.rev_chunk;
+    p.beta_tok = a.beta_tok;
     p.beta = a.beta;
     p.status = reinterpret_cast<unsigned int*>(ws);
     p.k_scale = a.k_scale;
@@ -924,7 +973,8 @@ cudaError_t launch_wide_mode(const ScanArgs& a, cudaStream_t st) {
         return cudaErrorInvalidValue;
 
     {
-        const void* kernels[] = {reinterpret_cast<const void*>(wide_gram_kernel<RELU>),
+        const void* kernels[] = {a.beta_tok ? reinterpret_cast<const void*>(wide_gram_kernel<false, true>)
+                                            : reinterpret_cast<const void*>(wide_gram_kernel<RELU>),
                                  reinterpret_cast<const void*>(wide_chain_gdn_kernel),
                                  reinterpret_cast<const void*>(wide_output_kernel<RELU>)};
         const int bytes[] = {(int)kSmemWideGram, (int)kSmemWideChain, (int)smem_wide_out<RELU>()};
@@ -982,7 +1032,10 @@ cudaError_t launch_wide_mode(const ScanArgs& a, cudaStream_t st) {
         const int grid = std::min(items, share);
         // gram(c) overwrites the buffers chain(c - 2) read
         if (ci >= 2) ok(cudaStreamWaitEvent(st, cx.chain[b], 0));
-        wide_gram_kernel<RELU><<<grid, wide_gram_threads(RELU), kSmemWideGram, st>>>(p, mK, mV);
+        if (!RELU && p.beta_tok)
+            wide_gram_kernel<false, true><<<grid, wide_gram_threads(true), kSmemWideGram, st>>>(p, mK, mV);
+        else
+            wide_gram_kernel<RELU><<<grid, wide_gram_threads(RELU), kSmemWideGram, st>>>(p, mK, mV);
         ok(cudaGetLastError());
         ok(cudaEventRecord(cx.gram[b], st));
         // chain(c) needs gram(c), and overwrites the images output(c - 2) read

@@ -115,7 +115,8 @@ def test_reverse_scan_argument_errors_and_sizes():
         ("tcgen05_fused", 1)
     # many heads: the three-kernel path with per-frame buffers
     assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 4, 20, 64, 880, 128)[0] == "tcgen05"
-    assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 1, 16, 512, 1024, 256)[0] == "simt_f32"
+    assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 1, 16, 512, 1024, 256)[0] == \
+        "tcgen05_wide"
     args = lambda C, D=64, w=ws: (P(), P(), P(), P(), la.LA_BF16, P(), P(), 0.1, C,
                                   1, 1, 4, 16, D, P(), w, None)
     assert L.la_scan_gdn_reverse(*args(0)) == la.LA_ERR_INVALID_ARG

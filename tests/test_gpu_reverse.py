@@ -4,7 +4,7 @@
 Bars as for the forward scan: 1e-4 for float32 inputs, 2e-2 for bfloat16
 inputs (max|gpu - ref| / max|ref|).  bf16 heads with 64 <= D <= 128 run on
 the single-kernel tensor-core path (the three-kernel path for many heads),
-the rest on the SIMT kernel.
+128 < D <= 256 on the wide path, the rest on the SIMT kernel.
 """
 import numpy as np
 import pytest
@@ -56,7 +56,7 @@ def _compare(spec, C, heads=None):
     ("bf16", 128, 96, 9, 16),      # chunk longer than the clip
     ("f32", 32, 40, 7, 3),         # SIMT path
     ("f32", 128, 33, 5, 2),
-    ("bf16", 256, 70, 5, 2),       # wide heads: SIMT path
+    ("bf16", 256, 70, 5, 2),       # wide heads: wide tensor-core path
 ])
 def test_reverse_scan_matches_oracle(dtype, D, S, F, C):
     spec = synth.small(B=2, H=2, F=F, S=S, D=D, dtype=dtype, seed=D + F, keys_l2=True)
@@ -113,3 +113,14 @@ def test_reverse_fused_kernel_matches_three_kernel_path(C, monkeypatch):
     assert rel_err(to_np(o_f), to_np(o_3)) <= TOL_BF16
     monkeypatch.delenv("LA_SCAN_NO_FUSE")
     _compare(spec, C)
+
+
+@pytest.mark.parametrize("wide_chunk", ["3", "7", "21"])
+def test_reverse_wide_path_with_unaligned_pipeline_chunks(wide_chunk, monkeypatch):
+    """D = 256 runs on the wide tensor-core path; its pipeline chunks (3, 7 or
+    21 frames) need not line up with the reversed scan's 4-frame chunks, since
+    a chunk start is a zero decay at that step."""
+    spec = synth.small(B=1, H=2, F=21, S=100, D=256, dtype="bf16", seed=97, keys_l2=True)
+    assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 1, 2, 21, 100, 256)[0] == "tcgen05_wide"
+    monkeypatch.setenv("LA_WIDE_CHUNK", wide_chunk)
+    _compare(spec, 4)

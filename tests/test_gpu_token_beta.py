@@ -3,8 +3,8 @@
 
 Bars: 1e-4 for float32 inputs, 2e-2 for bfloat16 inputs.  bf16 heads with
 64 <= D <= 128 run on the single-kernel tensor-core path (the three-kernel
-path for many heads), K and V token rows scaled by sqrt(beta) in shared
-memory; the rest on the SIMT kernel.
+path for many heads) and 128 < D <= 256 on the wide path, K and V token rows
+scaled by sqrt(beta) in shared memory; the rest on the SIMT kernel.
 """
 import numpy as np
 import pytest
@@ -63,7 +63,7 @@ def _compare(spec, heads=None, with_state=False):
     ("bf16", 64, 64, 3),
     ("bf16", 112, 200, 4),
     ("f32", 32, 40, 6),            # SIMT path
-    ("bf16", 256, 70, 3),          # wide heads: SIMT path
+    ("bf16", 256, 70, 3),          # wide heads: wide tensor-core path
 ])
 def test_token_gate_scan_matches_oracle(dtype, D, S, F):
     spec = synth.small(B=2, H=2, F=F, S=S, D=D, dtype=dtype, seed=D + S, keys_l2=True)
@@ -116,4 +116,13 @@ def test_token_gate_fused_kernel_matches_three_kernel_path(monkeypatch):
     assert rel_err(to_np(o_f), to_np(o_3)) <= TOL_BF16
     assert rel_err(to_np(m_f), to_np(m_3)) <= TOL_BF16
     monkeypatch.delenv("LA_SCAN_NO_FUSE")
+    _compare(spec, with_state=True)
+
+
+def test_token_gate_wide_path_matches_oracle_across_pipeline_chunks(monkeypatch):
+    """D = 256 on the wide tensor-core path, clip split into pipeline chunks."""
+    spec = synth.small(B=1, H=2, F=11, S=140, D=256, dtype="bf16", seed=99, keys_l2=True)
+    assert la.la_plan(la.LA_MODE_GDN_TOKEN_BETA, la.LA_BF16, 1, 2, 11, 140, 256)[0] == \
+        "tcgen05_wide"
+    monkeypatch.setenv("LA_WIDE_CHUNK", "4")
     _compare(spec, with_state=True)
