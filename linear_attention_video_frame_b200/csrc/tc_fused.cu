@@ -1045,15 +1045,35 @@ __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) 
             float a_nxt = alpha_at(1);                               // step 1
             // initial state: image of M_0 (buffer 1 = "frame -1") and TMEM alpha_0 M_0
             float z = 0.f;
-            for (int c0 = c_lo; c0 < c_hi; c0 += 16) {
-                float v[16];
+            {
+                // the row's columns c_lo .. c_hi - 1 (at most 64) as float4
+                // loads, all in flight at once
+                const float* src = (p.state_in && live) ? p.state_in + ((size_t)bh * D + row) * D
+                                                        : nullptr;
+                float4 r[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    v[e] = (p.state_in && live) ? p.state_in[((size_t)bh * D + row) * D + c0 + e] : 0.f;
-                store_row16_bf16(imgs + kImg, row, c0, v);
+                for (int u = 0; u < 16; ++u)
+                    r[u] = (src && c_lo + 4 * u < c_hi)
+                               ? __ldg(reinterpret_cast<const float4*>(src + c_lo + 4 * u))
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) v[e] *= a_cur;
-                tmem_st16(tl + c0, v);
+                for (int k = 0; k < 4; ++k) {
+                    const int c0 = c_lo + 16 * k;
+                    if (c0 < c_hi) {
+                        float v[16];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            v[4 * u] = r[4 * k + u].x;
+                            v[4 * u + 1] = r[4 * k + u].y;
+                            v[4 * u + 2] = r[4 * k + u].z;
+                            v[4 * u + 3] = r[4 * k + u].w;
+                        }
+                        store_row16_bf16(imgs + kImg, row, c0, v);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] *= a_cur;
+                        tmem_st16(tl + c0, v);
+                    }
+                }
             }
             if (RELU && h == 0 && p.z_in && live) z = p.z_in[(size_t)bh * D + row];
             tmem_wait_st();

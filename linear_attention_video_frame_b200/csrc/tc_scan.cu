@@ -91,15 +91,17 @@ struct TcParams {
     int rev_chunk;          // > 0: reversed GDN scan reset every rev_chunk frames
     const float* beta_tok;  // per-token update gate [BHF][S] (GDN), or NULL
     int f0, Fc;             // this launch covers frames [f0, f0 + Fc) of every head
+    int bh0;                // ... of heads bh0 .. bh0 + BH - 1 (BH: heads of this launch)
     float* trans_out;       // GDN interval composite: chain blocks BH .. 2 BH - 1 leave
                             // the transition A_F ... A_1 here, or NULL
 };
 
 // Global frame index (into q, k, v, o, the gates and the per-frame workspace
-// buffers, all sized for the whole clip) of launch-local item `it` = bh Fc + fl.
+// buffers, all sized for the whole clip and every head) of launch-local item
+// `it` = bh Fc + fl.
 __device__ __forceinline__ int global_item(const TcParams& p, int it) {
     const int bh = it / p.Fc;
-    return bh * p.F + p.f0 + (it - bh * p.Fc);
+    return (p.bh0 + bh) * p.F + p.f0 + (it - bh * p.Fc);
 }
 
 // ============================================================================
@@ -353,9 +355,11 @@ tc_gram_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapK,
 // chain: the per-(b, h) recurrence, state resident in tensor memory
 // ============================================================================
 // warp 0: bulk loader of the per-frame operands; warp 1: TMEM owner + MMA
-// issuer (GDN); warps 2-5: epilogue (thread <-> state row).
+// issuer (GDN); warps 2-9: epilogue (thread <-> state row and column half).
+constexpr int kChainEpi = 256;
+constexpr int kChainThreads = 64 + kChainEpi;
 template <bool RELU>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kChainThreads, 1)
 tc_chain_kernel(const TcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
@@ -377,16 +381,16 @@ tc_chain_kernel(const TcParams p) {
     // transition composite A_F ... A_1; blocks 0 .. BH - 1 leave the input
     // composite (the state from zero).
     const bool trans = p.trans_out && (int)blockIdx.x >= p.BH;
-    const int bh = trans ? (int)blockIdx.x - p.BH : (int)blockIdx.x;
+    const int bh = p.bh0 + (trans ? (int)blockIdx.x - p.BH : (int)blockIdx.x);
     const int F = p.F, D = p.D;
     const int nsteps = p.Fc;                // steps of this launch: clip steps f0 .. f0 + Fc - 1
     if (threadIdx.x == 0) {
         for (int s = 0; s < kCStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], RELU ? 4 : 5);     // epilogue warps (+ the MMA for GDN)
+            mbar_init(&empty[s], RELU ? 8 : 9);     // epilogue warps (+ the MMA for GDN)
         }
         mbar_init(mdone, 1);
-        mbar_init(mready, 4);
+        mbar_init(mready, 8);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -442,30 +446,62 @@ tc_chain_kernel(const TcParams p) {
             }
         }
     } else {
-        // ---------------- epilogue: thread <-> state row ----------------
+        // ------------- epilogue: thread <-> (state row, column half) -------------
+        // warps 2-9: TMEM lane quadrant q = warp % 4 (the rows it may access),
+        // column half h; two 16-column TMEM loads in flight per wait
         const int q = warp & 3, row = q * 32 + lane;
+        const int h = (warp - 2) >> 2;
+        const int c_mid = ((D / 16 + 1) / 2) * 16;
+        const int c_lo = h ? c_mid : 0, c_hi = h ? D : c_mid;
         const bool issuer = (threadIdx.x == 64);
         const uint32_t tl = tM + (uint32_t(q * 32) << 16);
         const bool live = row < D;
-        // initial state: TMEM (fp32) and operand image (bf16)
-        for (int c0 = 0; c0 < D; c0 += 16) {
-            float v[16];
+        // initial state: TMEM (fp32) and operand image (bf16); the row's
+        // columns c_lo .. c_hi - 1 (at most 64) arrive as float4 loads, all
+        // in flight at once
+        {
+            const float* src = (!trans && p.state_in && live)
+                                   ? p.state_in + ((size_t)bh * D + row) * D : nullptr;
+            float4 r[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-                v[e] = trans ? (row == c0 + e ? 1.f : 0.f)
-                             : ((p.state_in && live) ? p.state_in[((size_t)bh * D + row) * D + c0 + e]
-                                                     : 0.f);
-            tmem_st16(tl + c0, v);
-            store_row16_bf16(mimg, row, c0, v);
+            for (int u = 0; u < 16; ++u)
+                r[u] = (src && c_lo + 4 * u < c_hi)
+                           ? __ldg(reinterpret_cast<const float4*>(src + c_lo + 4 * u))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int c0 = c_lo + 16 * k;
+                if (c0 < c_hi) {
+                    float v[16];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        v[4 * u] = r[4 * k + u].x;
+                        v[4 * u + 1] = r[4 * k + u].y;
+                        v[4 * u + 2] = r[4 * k + u].z;
+                        v[4 * u + 3] = r[4 * k + u].w;
+                    }
+                    if (trans)
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) v[e] = (row == c0 + e) ? 1.f : 0.f;
+                    tmem_st16(tl + c0, v);
+                    store_row16_bf16(mimg, row, c0, v);
+                }
+            }
         }
         float z = 0.f;
-        if (RELU && p.z_in && live) z = p.z_in[(size_t)bh * D + row];
+        if (RELU && h == 0 && p.z_in && live) z = p.z_in[(size_t)bh * D + row];
         tmem_wait_st();
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(mready);
 
+        // the decay of step f + 1 is read during step f
+        auto alpha_of = [&](int f) -> float {
+            if (RELU || f >= nsteps) return 1.f;
+            return __ldg(p.alpha + (size_t)bh * F + step_frame(p.f0 + f, F, p.rev_chunk));
+        };
+        float al_next = alpha_of(0);
         int s = 0;
         uint32_t ph = 0;
         bool ok = true;     // every epilogue warp runs every named barrier, even after an abort
@@ -477,37 +513,60 @@ tc_chain_kernel(const TcParams p) {
             ok = ok && mbar_wait(&full[s], ph, ab, 0x204);
             if (!RELU) ok = ok && mbar_wait(mdone, f & 1, ab, 0x205);
             tc_fence_after();
-            const float al = RELU ? 1.f : p.alpha[frame];
+            const float al = al_next;
+            al_next = alpha_of(f + 1);
             const uint8_t* st = ring + s * kStage;
             const float* bq = reinterpret_cast<const float*>(st + (RELU ? 0 : kImg));
             if (issuer && p.want_output) bulk_wait_read<0>();   // image free for rewriting
-            named_bar_sync(1, kEpiThreads);
+            named_bar_sync(1, kChainEpi);
             const bool last = (f == nsteps - 1);
             float* sout = trans ? p.trans_out : p.state_out;
-            for (int c0 = 0; c0 < D && ok; c0 += 16) {
-                float v[16];
-                tmem_ld16(tl + c0, v);
+            for (int c0 = c_lo; c0 < c_hi && ok; c0 += 32) {
+                const bool two = c0 + 16 < c_hi;
+                float v0[16], v1[16];
+                tmem_ld16(tl + c0, v0);
+                if (two) tmem_ld16(tl + c0 + 16, v1);
+                float4 b[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    b[u] = (trans || (u >= 4 && !two))
+                               ? make_float4(0.f, 0.f, 0.f, 0.f)
+                               : *reinterpret_cast<const float4*>(bq + ((c0 / 4 + u) * 128 + row) * 4);
                 tmem_wait_ld();
+                // reset: the state restarts from B (the TMEM value is not read,
+                // so a non-finite leftover cannot leak in)
+                auto upd = [&](float& x, float bv) { x = reset ? bv : fmaf(al, x, bv); };
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const float4 b = trans ? make_float4(0.f, 0.f, 0.f, 0.f)
-                                           : *reinterpret_cast<const float4*>(
-                                                 bq + ((c0 / 4 + u) * 128 + row) * 4);
-                    const float ae = reset ? 0.f : al;
-                    v[4 * u] = reset ? b.x : fmaf(ae, v[4 * u], b.x);
-                    v[4 * u + 1] = reset ? b.y : fmaf(ae, v[4 * u + 1], b.y);
-                    v[4 * u + 2] = reset ? b.z : fmaf(ae, v[4 * u + 2], b.z);
-                    v[4 * u + 3] = reset ? b.w : fmaf(ae, v[4 * u + 3], b.w);
+                    upd(v0[4 * u], b[u].x);
+                    upd(v0[4 * u + 1], b[u].y);
+                    upd(v0[4 * u + 2], b[u].z);
+                    upd(v0[4 * u + 3], b[u].w);
+                    upd(v1[4 * u], b[4 + u].x);
+                    upd(v1[4 * u + 1], b[4 + u].y);
+                    upd(v1[4 * u + 2], b[4 + u].z);
+                    upd(v1[4 * u + 3], b[4 + u].w);
                 }
-                tmem_st16(tl + c0, v);
-                store_row16_bf16(mimg, row, c0, v);
-                if (last && sout && live)
+                tmem_st16(tl + c0, v0);
+                store_row16_bf16(mimg, row, c0, v0);
+                if (two) {
+                    tmem_st16(tl + c0 + 16, v1);
+                    store_row16_bf16(mimg, row, c0 + 16, v1);
+                }
+                if (last && sout && live) {
+                    float* so = sout + ((size_t)bh * D + row) * D + c0;
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
-                        *reinterpret_cast<float4*>(sout + ((size_t)bh * D + row) * D + c0 + 4 * u) =
-                            make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                        *reinterpret_cast<float4*>(so + 4 * u) =
+                            make_float4(v0[4 * u], v0[4 * u + 1], v0[4 * u + 2], v0[4 * u + 3]);
+                    if (two)
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            *reinterpret_cast<float4*>(so + 16 + 4 * u) =
+                                make_float4(v1[4 * u], v1[4 * u + 1], v1[4 * u + 2], v1[4 * u + 3]);
+                }
             }
-            if (RELU && ok) {
+            if (RELU && h == 0 && ok) {
                 z += reinterpret_cast<const float*>(st + kQuadMat)[row];
                 if (p.want_output) p.zf[frame * 128 + row] = z;
                 if (last && p.z_out && live) p.z_out[(size_t)bh * D + row] = z;
@@ -517,7 +576,7 @@ tc_chain_kernel(const TcParams p) {
             tmem_wait_st();
             fence_proxy_async_smem();
             tc_fence_before();
-            named_bar_sync(1, kEpiThreads);
+            named_bar_sync(1, kChainEpi);
             if (issuer && p.want_output && ok) {
                 bulk_store(p.mimg + frame * kImg, mimg, kImg);
                 bulk_commit();
@@ -800,6 +859,25 @@ int tc_chunk(const ScanArgs& a, int nsm) {
     return std::max(1, std::min(c, std::max(a.F, 1)));
 }
 
+constexpr int kMaxHeadGroups = 8;
+
+// Head groups of a one-chunk call.  With a single frame chunk the chain of
+// every head waits for the whole gram and holds up the whole output; heads
+// are independent, so with two groups the chain of the first half of the
+// heads runs beside the gram of the second half.  More groups lose: every
+// group's chain still takes its F latency-bound steps and its gram and output
+// their fill and drain (LA_TC_HEAD_GROUPS overrides, 1 .. min(B H, 8)).
+int tc_head_groups(const ScanArgs& a, int nsm, int Fc) {
+    const int BH = a.B * a.H;
+    if (a.trans_out || Fc < a.F || a.F < 1) return 1;
+    int g = ((long)BH * a.F >= 2L * nsm && BH >= 8) ? 2 : 1;
+    if (const char* e = std::getenv("LA_TC_HEAD_GROUPS")) {
+        const int v = std::atoi(e);
+        if (v > 0) g = std::min(v, std::min(BH, kMaxHeadGroups));
+    }
+    return g;
+}
+
 // Streams and events of one device for the chunk pipeline (gram kernels on
 // the caller's stream, chain and output kernels on two streams of the
 // library's own, forked from and joined back to the caller's stream).
@@ -808,6 +886,11 @@ struct TcCtx {
     bool ready = false;
     cudaStream_t s_chain = nullptr, s_out = nullptr;
     cudaEvent_t start = nullptr, gram = nullptr, chain = nullptr, out = nullptr;
+    // head groups: chain and output of group g on s_grp[g] (high priority),
+    // after its gram (grp_in[g]); the caller's stream joins every grp_done[g]
+    bool grp_ready = false;
+    cudaStream_t s_grp[kMaxHeadGroups] = {};
+    cudaEvent_t grp_in[kMaxHeadGroups] = {}, grp_done[kMaxHeadGroups] = {};
 };
 std::mutex g_tc_mu[kMaxDevicesTc];
 TcCtx g_tc_ctx[kMaxDevicesTc];
@@ -820,6 +903,19 @@ cudaError_t tc_ctx_init(TcCtx& c) {
     for (cudaEvent_t* p : evs)
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(p, cudaEventDisableTiming);
     if (e == cudaSuccess) c.ready = true;
+    return e;
+}
+
+cudaError_t tc_ctx_init_groups(TcCtx& c) {
+    if (c.grp_ready) return cudaSuccess;
+    int lo = 0, hi = 0;
+    cudaError_t e = cudaDeviceGetStreamPriorityRange(&lo, &hi);
+    for (int g = 0; g < kMaxHeadGroups && e == cudaSuccess; ++g) {
+        e = cudaStreamCreateWithPriority(&c.s_grp[g], cudaStreamNonBlocking, hi);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c.grp_in[g], cudaEventDisableTiming);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&c.grp_done[g], cudaEventDisableTiming);
+    }
+    if (e == cudaSuccess) c.grp_ready = true;
     return e;
 }
 
@@ -846,6 +942,7 @@ cudaError_t launch_tc_mode(const ScanArgs& a, cudaStream_t st) {
     p.rev_chunk = a.rev_chunk;
     p.beta_tok = a.beta_tok;
     p.trans_out = a.trans_out;
+    p.bh0 = 0;
 
     const uint64_t bhf = (uint64_t)p.BH * p.F;
     CUtensorMap mK, mV, mQ, mO;
@@ -888,11 +985,12 @@ cudaError_t launch_tc_mode(const ScanArgs& a, cudaStream_t st) {
         else
             tc_gram_kernel<RELU><<<grid, thr, smem_gram, s>>>(p, mK, mV);
     };
-    if (nchunks == 1) {
+    const int ngroups = nchunks == 1 ? tc_head_groups(a, nsm, Fc) : 1;
+    if (nchunks == 1 && ngroups == 1) {
         set_chunk(0);
         const int grid_f = (int)std::min<uint64_t>(bhf, (uint64_t)nsm);
         gram(grid_f, st);
-        tc_chain_kernel<RELU><<<p.BH * (p.trans_out ? 2 : 1), 192,
+        tc_chain_kernel<RELU><<<p.BH * (p.trans_out ? 2 : 1), kChainThreads,
                                 RELU ? smem_chain_relu : smem_chain_gdn, st>>>(p);
         if (p.want_output) tc_output_kernel<RELU><<<grid_f, thr, smem_out, st>>>(p, mQ, mO);
         return cudaGetLastError();
@@ -901,7 +999,10 @@ cudaError_t launch_tc_mode(const ScanArgs& a, cudaStream_t st) {
     // gram(c + 1) and output(c - 1), which share the other SMs.  Every chunk
     // writes its own frames of the clip-sized buffers, so only gram -> chain
     // -> output of the same chunk (and chain -> chain through the carried
-    // state, in stream order) must be ordered.
+    // state, in stream order) must be ordered.  A one-chunk call pipelines
+    // over head groups instead: a group's launches cover heads
+    // [bh0, bh0 + BH) of the same buffers, so again only its own gram ->
+    // chain -> output are ordered.
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevicesTc)
         return cudaErrorInvalidDevice;
@@ -909,11 +1010,44 @@ cudaError_t launch_tc_mode(const ScanArgs& a, cudaStream_t st) {
     TcCtx& cx = g_tc_ctx[dev];
     cudaError_t e = tc_ctx_init(cx);
     if (e != cudaSuccess) return e;
-    const int share = std::max(8, nsm - p.BH);
     auto ok = [&](cudaError_t x) {
         if (x != cudaSuccess && e == cudaSuccess) e = x;
         return e == cudaSuccess;
     };
+    if (ngroups > 1) {
+        // Head groups: the grams in order on the caller's stream; the chain
+        // and output of group g on stream g, so that the chains of several
+        // groups (each a few microseconds per frame whatever its head count)
+        // overlap one another and the grams and outputs of other groups.
+        ok(tc_ctx_init_groups(cx));
+        const int BH = p.BH;
+        int recorded = 0;
+        set_chunk(0);
+        for (int g = 0; g < ngroups && e == cudaSuccess; ++g) {
+            p.bh0 = (int)((long)g * BH / ngroups);
+            p.BH = (int)((long)(g + 1) * BH / ngroups) - p.bh0;
+            const int grid = std::min(p.BH * p.Fc, std::max(8, nsm - p.BH));
+            cudaStream_t sg = cx.s_grp[g];
+            gram(grid, st);
+            ok(cudaGetLastError());
+            ok(cudaEventRecord(cx.grp_in[g], st));
+            ok(cudaStreamWaitEvent(sg, cx.grp_in[g], 0));
+            tc_chain_kernel<RELU><<<p.BH, kChainThreads, RELU ? smem_chain_relu : smem_chain_gdn, sg>>>(p);
+            ok(cudaGetLastError());
+            if (p.want_output) {
+                tc_output_kernel<RELU><<<grid, thr, smem_out, sg>>>(p, mQ, mO);
+                ok(cudaGetLastError());
+            }
+            if (ok(cudaEventRecord(cx.grp_done[g], sg))) recorded = g + 1;
+        }
+        // join: the caller's stream continues after every group's output
+        for (int g = 0; g < recorded; ++g) {
+            const cudaError_t j = cudaStreamWaitEvent(st, cx.grp_done[g], 0);
+            if (j != cudaSuccess && e == cudaSuccess) e = j;
+        }
+        return e;
+    }
+    const int share = std::max(8, nsm - p.BH);
     ok(cudaEventRecord(cx.start, st));
     ok(cudaStreamWaitEvent(cx.s_chain, cx.start, 0));
     ok(cudaStreamWaitEvent(cx.s_out, cx.start, 0));
@@ -924,7 +1058,7 @@ cudaError_t launch_tc_mode(const ScanArgs& a, cudaStream_t st) {
         ok(cudaGetLastError());
         ok(cudaEventRecord(cx.gram, st));
         ok(cudaStreamWaitEvent(cx.s_chain, cx.gram, 0));
-        tc_chain_kernel<RELU><<<p.BH, 192, RELU ? smem_chain_relu : smem_chain_gdn, cx.s_chain>>>(p);
+        tc_chain_kernel<RELU><<<p.BH, kChainThreads, RELU ? smem_chain_relu : smem_chain_gdn, cx.s_chain>>>(p);
         ok(cudaGetLastError());
         ok(cudaEventRecord(cx.chain, cx.s_chain));
         if (p.want_output) {
@@ -950,8 +1084,10 @@ bool tc_eligible(const ScanArgs& a) {
 size_t tc_workspace_bytes(const ScanArgs& a) { return ws_layout(a).total; }
 
 int tc_kernel_count(const ScanArgs& a) {
-    const int Fc = tc_chunk(a, device_sm_count());
-    return (a.o ? 3 : 2) * ((a.F + Fc - 1) / Fc);
+    const int nsm = device_sm_count();
+    const int Fc = tc_chunk(a, nsm);
+    const int nchunks = (a.F + Fc - 1) / Fc;
+    return (a.o ? 3 : 2) * nchunks * (nchunks == 1 ? tc_head_groups(a, nsm, Fc) : 1);
 }
 
 cudaError_t launch_tc(const ScanArgs& a, cudaStream_t st) {

@@ -211,8 +211,27 @@ def test_three_kernel_path_chunk_count(F, chunks, monkeypatch):
 
 
 def test_three_kernel_pipeline_needs_free_sms():
-    # 80 heads would hold more than half of the SMs with chain CTAs: one chunk
-    assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 4, 20, 64, 880, 128) == ("tcgen05", 3)
+    # 80 heads would hold more than half of the SMs with chain CTAs: one frame
+    # chunk, pipelined over two head groups instead
+    assert la.la_plan(la.LA_MODE_GDN_REVERSE, la.LA_BF16, 4, 20, 64, 880, 128) == ("tcgen05", 6)
+
+
+@pytest.mark.parametrize("B,H,F,groups", [(4, 20, 8, 2), (4, 20, 1, 1), (3, 20, 4, 1),
+                                          (1, 60, 16, 2), (1, 80, 64, 2), (1, 7, 24, 1)])
+def test_three_kernel_head_groups(B, H, F, groups, monkeypatch):
+    """A one-chunk call with at least 8 heads and B H F >= 2 x 148 items runs
+    its heads in two groups, three kernels per group."""
+    monkeypatch.setenv("LA_SCAN_NO_FUSE", "1")
+    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, B, H, F, 880, 128) == ("tcgen05", 3 * groups)
+    assert la.la_plan(la.LA_MODE_RELU, la.LA_BF16, B, H, F, 880, 128) == ("tcgen05", 3 * groups)
+
+
+def test_three_kernel_head_groups_override(monkeypatch):
+    monkeypatch.setenv("LA_SCAN_NO_FUSE", "1")
+    monkeypatch.setenv("LA_TC_HEAD_GROUPS", "3")
+    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 4, 20, 8, 880, 128) == ("tcgen05", 9)
+    monkeypatch.setenv("LA_TC_HEAD_GROUPS", "1000")      # at most one group per head
+    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 5, 8, 880, 128) == ("tcgen05", 15)
 
 
 def test_reversed_scan_chunks_align_with_pipeline_chunks(monkeypatch):

@@ -392,7 +392,8 @@ def test_three_kernel_chunk_pipeline_is_exact(mode, monkeypatch):
 def test_plan_of_the_workloads():
     assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 20, 181, 880, 128) == ("tcgen05_fused", 1)
     assert la.la_plan(la.LA_MODE_RELU, la.LA_BF16, 1, 20, 21, 1560, 112) == ("tcgen05_fused", 1)
-    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 4, 20, 8, 880, 128) == ("tcgen05", 3)
+    # 80 heads of 8 frames: one frame chunk, pipelined over two head groups
+    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 4, 20, 8, 880, 128) == ("tcgen05", 6)
     assert la.la_plan(la.LA_MODE_GDN, la.LA_F32, 1, 2, 8, 64, 32)[0] == "simt_f32"
     # 8 pipeline chunks of 64 frames, three kernels each
     assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 1, 16, 512, 1024, 256) == ("tcgen05_wide", 24)
@@ -432,8 +433,36 @@ def test_fused_kernel_at_its_head_limit_with_slot_reuse(mode):
 
 def test_many_heads_use_the_three_kernel_path():
     spec = synth.small(B=15, H=20, F=2, S=64, D=64, dtype="bf16", seed=37)
-    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 15, 20, 2, 64, 64) == ("tcgen05", 3)
-    _compare(spec, "gdn", heads=[(0, 0), (7, 13), (14, 19)])
+    # 300 heads of 2 frames: two head groups of 150
+    assert la.la_plan(la.LA_MODE_GDN, la.LA_BF16, 15, 20, 2, 64, 64) == ("tcgen05", 6)
+    _compare(spec, "gdn", heads=[(0, 0), (7, 9), (7, 10), (14, 19)])
+
+
+@pytest.mark.parametrize("mode", ["relu", "gdn"])
+def test_three_kernel_head_groups_are_exact(mode, monkeypatch):
+    """A one-chunk call on the three-kernel path runs as a pipeline of head
+    groups (chain of one group beside the gram of the next and the output of
+    the one before): any grouping gives the same bits, and the oracle's values
+    on every head."""
+    spec = synth.small(B=4, H=20, F=8, S=200, D=128, dtype="bf16", seed=73, keys_l2=True,
+                       alpha=("sigmoid_normal", 3.0, 1.0), beta=("sigmoid_normal", 0.0, 1.0))
+    m = la.LA_MODE_GDN if mode == "gdn" else la.LA_MODE_RELU
+    assert la.la_plan(m, la.LA_BF16, 4, 20, 8, 200, 128) == ("tcgen05", 6)     # 2 groups
+    inp = device_inputs(spec)
+    m0n, z0n = synth.random_state(spec, 0.05)
+    m0, z0 = torch.from_numpy(m0n).cuda(), torch.from_numpy(z0n).cuda()
+    runs = []
+    for groups in ("1", "3", "8"):
+        monkeypatch.setenv("LA_TC_HEAD_GROUPS", groups)
+        runs.append(_run(spec, mode, inp, m0, z0 if mode == "relu" else None))
+    torch.cuda.synchronize()
+    for o, so, zo in runs[1:]:
+        assert torch.equal(o.view(torch.int16), runs[0][0].view(torch.int16))
+        assert torch.equal(so, runs[0][1])
+        if mode == "relu":
+            assert torch.equal(zo, runs[0][2])
+    monkeypatch.delenv("LA_TC_HEAD_GROUPS")
+    _compare(spec, mode, with_state=True)
 
 
 def test_device_wait_timeout_is_reported_and_the_context_stays_usable(monkeypatch):
