@@ -67,15 +67,31 @@ struct Abort {
     }
 };
 
+// The same test with cluster-scope acquire, for a phase completed by arrivals
+// of the other CTA of a cluster (whose shared-memory writes it must see).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
 // Wait until the phase of `bar` with parity `parity` has completed.  Returns
 // false (and raises the block's abort flag) after kWaitLimitNs, or soon after
 // another thread of the block, or another block of the launch, gave up.
+// `cluster`: acquire at cluster scope (arrivals from the other CTA of a pair).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Abort& ab,
-                                          uint32_t where) {
-    if (mbar_try_wait(bar, parity)) return true;
+                                          uint32_t where, bool cluster = false) {
+    auto test = [&]() {
+        return cluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity);
+    };
+    if (test()) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 0;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (test()) return true;
         if (ab.raised()) return false;
         if ((it & 15) == 15) {
             if (*reinterpret_cast<volatile unsigned int*>(ab.status) != 0) {
@@ -225,6 +241,72 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
         ::"r"(smem_u32(bar)) : "memory");
 }
 
+// ----------------------------------------------------------------------------
+// CTA pairs: clusters of two CTAs whose tensor cores work as one (cta_group::2)
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t ncluster_x() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+// Barrier over every thread of every CTA of the cluster (release / acquire).
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive (release at cluster scope) on the mbarrier at the shared-memory
+// offset of `bar` in CTA `cta` of the cluster (this CTA's own included).
+__device__ __forceinline__ void mbar_arrive_cluster(uint64_t* bar, uint32_t cta) {
+    asm volatile(
+        "{\n\t.reg .b32 ra;\n\t"
+        "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+        "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}"
+        ::"r"(smem_u32(bar)), "r"(cta) : "memory");
+}
+// Tensor memory of a pair: one warp of each CTA (the same warp index) takes
+// part; both CTAs receive the same address at the same offset.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(dst)), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;"
+                 ::"r"(taddr), "r"(ncols) : "memory");
+}
+// Pair MMA, issued by the even CTA: D (M = 256: rows 128 c .. 128 c + 127 in
+// CTA c's tensor memory) (+)= A B^T, where CTA c supplies rows 128 c ..
+// 128 c + 127 of A and columns (N / 2) c .. (N / 2)(c + 1) - 1 of B, each
+// from its own shared memory at the descriptors' offsets.
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate) : "memory");
+}
+// Arrive once on the mbarrier at the offset of `bar` in CTA `cta` of the pair
+// when all pair MMAs this thread issued before have completed.
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint32_t cta) {
+    asm volatile(
+        "{\n\t.reg .b32 ra;\n\t"
+        "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [ra];\n\t}"
+        ::"r"(smem_u32(bar)), "r"(cta) : "memory");
+}
+
 // 32 lanes x 32 bit, 16 consecutive columns per thread (thread i <-> lane base+i).
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     uint32_t r[16];
@@ -252,6 +334,14 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16]) 
 }
 __device__ __forceinline__ void tmem_wait_ld() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// Columns col .. col + 16 nu - 1 (nu <= 4, warp-uniform) of the thread's lane
+// as nu 16-column loads in flight at once, then one wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, int nu, float (&v)[4][16]) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+        if (u < nu) tmem_ld16(taddr + 16 * u, v[u]);
+    tmem_wait_ld();
 }
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");

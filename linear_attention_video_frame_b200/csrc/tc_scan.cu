@@ -238,33 +238,44 @@ tc_gram_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapK,
                 const float sg = bt * p.k_scale * p.k_scale, sw = bt * p.k_scale;
                 if (issuer) bulk_wait_read<0>();       // staging free again
                 named_bar_sync(1, kEpiThreads);
-                for (int c0 = 0; c0 < D && ok; c0 += 16) {
-                    float v[16];
-                    tmem_ld16(tl + c0, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) v[e] *= sg;
-                    store_row16_bf16(stage_img, row, c0, v);
-                }
-                for (int c0 = 0; c0 < D && ok; c0 += 16) {
-                    float v[16];
-                    tmem_ld16(tl + 128 + c0, v);
-                    tmem_wait_ld();
+                for (int c0 = 0; c0 < D && ok; c0 += 64) {
+                    float v[4][16];
+                    const int nu = min(4, (D - c0) / 16);
+                    tmem_ld64(tl + c0, nu, v);
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
-                        *reinterpret_cast<float4*>(bq + ((c0 / 4 + u) * 128 + row) * 4) =
-                            make_float4(v[4 * u] * sw, v[4 * u + 1] * sw, v[4 * u + 2] * sw,
-                                        v[4 * u + 3] * sw);
+                        if (u < nu) {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) v[u][e] *= sg;
+                            store_row16_bf16(stage_img, row, c0 + 16 * u, v[u]);
+                        }
+                }
+                for (int c0 = 0; c0 < D && ok; c0 += 64) {
+                    float v[4][16];
+                    const int nu = min(4, (D - c0) / 16);
+                    tmem_ld64(tl + 128 + c0, nu, v);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (u < nu)
+#pragma unroll
+                            for (int w = 0; w < 4; ++w)
+                                *reinterpret_cast<float4*>(bq + (((c0 + 16 * u) / 4 + w) * 128 + row) * 4) =
+                                    make_float4(v[u][4 * w] * sw, v[u][4 * w + 1] * sw,
+                                                v[u][4 * w + 2] * sw, v[u][4 * w + 3] * sw);
                 }
             } else if (ok) {
-                for (int c0 = 0; c0 < D; c0 += 16) {
-                    float v[16];
-                    tmem_ld16(tl + 128 + c0, v);
-                    tmem_wait_ld();
+                for (int c0 = 0; c0 < D; c0 += 64) {
+                    float v[4][16];
+                    const int nu = min(4, (D - c0) / 16);
+                    tmem_ld64(tl + 128 + c0, nu, v);
 #pragma unroll
                     for (int u = 0; u < 4; ++u)
-                        *reinterpret_cast<float4*>(bq + ((c0 / 4 + u) * 128 + row) * 4) =
-                            make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                        if (u < nu)
+#pragma unroll
+                            for (int w = 0; w < 4; ++w)
+                                *reinterpret_cast<float4*>(bq + (((c0 + 16 * u) / 4 + w) * 128 + row) * 4) =
+                                    make_float4(v[u][4 * w], v[u][4 * w + 1], v[u][4 * w + 2],
+                                                v[u][4 * w + 3]);
                 }
                 float v[16];
                 tmem_ld16(tl, v);
@@ -723,15 +734,19 @@ tc_output_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapQ,
                 uint8_t* os = ostage + ob * 32768;
                 const float inv = (RELU && ok) ? 1.f / denbuf[a * 128 + row] : 1.f;
                 const uint32_t tl = tbase + (uint32_t(q * 32) << 16) + a * 128;
-                for (int c0 = 0; c0 < D && ok; c0 += 16) {
-                    float v[16];
-                    tmem_ld16(tl + c0, v);
-                    tmem_wait_ld();
-                    if (RELU) {
+                for (int c0 = 0; c0 < D && ok; c0 += 64) {
+                    float v[4][16];
+                    const int nu = min(4, (D - c0) / 16);
+                    tmem_ld64(tl + c0, nu, v);
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) v[e] *= inv;
-                    }
-                    store_row16_bf16(os, row, c0, v);
+                    for (int u = 0; u < 4; ++u)
+                        if (u < nu) {
+                            if (RELU) {
+#pragma unroll
+                                for (int e = 0; e < 16; ++e) v[u][e] *= inv;
+                            }
+                            store_row16_bf16(os, row, c0 + 16 * u, v[u]);
+                        }
                 }
                 tc_fence_before();
                 __syncwarp();

@@ -116,6 +116,71 @@ __device__ __forceinline__ uint32_t quad_off(int row, int col) {
     return ((uint32_t)(col >> 2) * 128u + (uint32_t)row) * 4u + (uint32_t)(col & 3);
 }
 
+// Read-out of one gram item (workspace item `item` = 2 loc + r: key-row block
+// r of chunk-local step loc) by one epilogue group g (half of the 512
+// accumulator columns; thread <-> accumulator row `row`, TMEM lane base in tl).
+template <bool RELU, bool TOKB>
+__device__ __forceinline__ void gram_readout(const WideParams& p, uint32_t tl, int item, int g,
+                                             int row) {
+    // four 16-column TMEM loads in flight per wait
+    float v[4][16];
+    auto load64 = [&](uint32_t col) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) tmem_ld16(tl + col + 16 * u, v[u]);
+        tmem_wait_ld();
+    };
+    if (!RELU) {
+        const int frame = global_frame(p, item >> 1);
+        const float al = step_alpha(p, item >> 1), bt = TOKB ? 1.f : p.beta[frame];
+        const float sg = -al * bt * p.k_scale * p.k_scale, sw = bt * p.k_scale;
+        if (g == 0) {
+            // the G''[r] image goes straight from registers to its workspace slot
+            uint8_t* gi = p.gimg + (size_t)item * kGImg;
+            for (int c0 = 0; c0 < kDW; c0 += 64) {
+                load64(c0);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[u][e] *= sg;
+                    store_row16(gi, 16384, row, c0 + 16 * u, v[u]);
+                }
+            }
+        } else {
+            for (int c0 = 0; c0 < kDW; c0 += 64) {
+                load64(256 + c0);
+                uint4* bt4 = p.btil + ((size_t)item * 2 + (c0 >> 7)) * kBTile;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int jc = ((c0 + 16 * u) & 127) >> 3;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        bt4[(jc + h) * 128 + row] = make_uint4(
+                            pack_bf16x2(v[u][8 * h] * sw, v[u][8 * h + 1] * sw),
+                            pack_bf16x2(v[u][8 * h + 2] * sw, v[u][8 * h + 3] * sw),
+                            pack_bf16x2(v[u][8 * h + 4] * sw, v[u][8 * h + 5] * sw),
+                            pack_bf16x2(v[u][8 * h + 6] * sw, v[u][8 * h + 7] * sw));
+                }
+            }
+        }
+    } else {
+        float* bq = p.bmat + (size_t)item * kQuad;
+        for (int c0 = 128 * g; c0 < 128 * g + 128; c0 += 64) {
+            load64(c0);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int w = 0; w < 4; ++w)
+                    *reinterpret_cast<float4*>(bq + quad_off(row, c0 + 16 * u + 4 * w)) =
+                        make_float4(v[u][4 * w], v[u][4 * w + 1], v[u][4 * w + 2], v[u][4 * w + 3]);
+        }
+        if (g == 0) {
+            tmem_ld16(tl + 256, v[0]);
+            tmem_wait_ld();
+            p.dz[(size_t)item * 128 + row] = v[0][0];
+        }
+    }
+}
+
 // ============================================================================
 // gram: per-frame contractions over tokens, one key-row block per CTA
 // ============================================================================
@@ -308,55 +373,9 @@ wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
         int li = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
-            const int frame = global_frame(p, item >> 1);
             if (!(ok = mbar_wait(accfull, li & 1, ab, 0x604))) break;
             tc_fence_after();
-            const uint32_t tl = tbase + (uint32_t(q * 32) << 16);
-            if (!RELU) {
-                const float al = step_alpha(p, item >> 1), bt = TOKB ? 1.f : p.beta[frame];
-                const float sg = -al * bt * p.k_scale * p.k_scale, sw = bt * p.k_scale;
-                // the G''[r] image goes straight from registers to its workspace slot
-                uint8_t* gi = p.gimg + (size_t)item * kGImg;
-                for (int c0 = 0; c0 < kDW && g == 0; c0 += 16) {
-                    float v[16];
-                    tmem_ld16(tl + c0, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) v[e] *= sg;
-                    store_row16(gi, 16384, row, c0, v);
-                }
-                for (int c0 = 0; c0 < kDW && g == 1; c0 += 16) {
-                    float v[16];
-                    tmem_ld16(tl + 256 + c0, v);
-                    tmem_wait_ld();
-                    uint4* bt = p.btil + ((size_t)item * 2 + (c0 >> 7)) * kBTile;
-                    const int jc = (c0 & 127) >> 3;
-#pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        bt[(jc + h) * 128 + row] = make_uint4(
-                            pack_bf16x2(v[8 * h] * sw, v[8 * h + 1] * sw),
-                            pack_bf16x2(v[8 * h + 2] * sw, v[8 * h + 3] * sw),
-                            pack_bf16x2(v[8 * h + 4] * sw, v[8 * h + 5] * sw),
-                            pack_bf16x2(v[8 * h + 6] * sw, v[8 * h + 7] * sw));
-                }
-            } else {
-                float* bq = p.bmat + (size_t)item * kQuad;
-                for (int c0 = 128 * g; c0 < 128 * g + 128; c0 += 16) {
-                    float v[16];
-                    tmem_ld16(tl + c0, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        *reinterpret_cast<float4*>(bq + quad_off(row, c0 + 4 * u)) =
-                            make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
-                }
-                if (g == 0) {
-                    float v[16];
-                    tmem_ld16(tl + 256, v);
-                    tmem_wait_ld();
-                    p.dz[(size_t)item * 128 + row] = v[0];
-                }
-            }
+            gram_readout<RELU, TOKB>(p, tbase + (uint32_t(q * 32) << 16), item, g, row);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(accempty);
@@ -365,6 +384,241 @@ wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
     tc_fence_before();
     __syncthreads();
     if (warp == 1) tmem_dealloc(tbase, 512);
+}
+
+// ============================================================================
+// gram on a CTA pair (cta_group::2): one cluster of two CTAs per (b, h, f)
+// ============================================================================
+// The pair computes the item's 256 x 512 accumulator [K^T K | K^T V] (ReLU:
+// [phi(K)^T V | phi(K)^T 1]) with M = 256 MMAs that the even CTA issues.
+// CTA c holds key columns 128 c .. 128 c + 127 of every K and V tile: they
+// are at once its 128 rows of A = K^T and its 128 columns of B = K or V.  Its
+// tensor memory receives accumulator rows 128 c .. 128 c + 127, i.e. key-row
+// block r = c of the single-CTA kernel, which the same read-out handles.  So
+// every K and V byte is fetched once per frame and each CTA's shared memory
+// serves half the operand bytes of the single-CTA kernel.
+//
+// Barriers (every wait bounded):
+//   full[s]   (each CTA)  this CTA's TMA bytes of stage s have landed
+//   ready[s]  (even CTA)  stage s usable by the pair's MMAs: with no transform
+//                         the odd CTA's warp 1 forwards its full[s] (the even
+//                         CTA's MMA issuer waits on its own full[s] too); with
+//                         a transform, the four transform warps of both CTAs
+//                         arrive when their pass is done
+//   empty[s]  (each CTA)  the pair's MMAs have read stage s (commit to each CTA)
+//   accfull   (each CTA)  the item's accumulator is complete (commit to each CTA)
+//   accempty  (even CTA)  all 16 epilogue warps of the pair have read the TMEM
+// Warps: 0 TMA producer; 1 TMEM (both CTAs), MMA issuer (even CTA) or
+// forwarder (odd CTA); 2-5 and 6-9 (10-13 with a transform) the two epilogue
+// groups; 6-9 with a transform: phi(K) (ReLU) or sqrt(beta_t) row scaling.
+constexpr int kPairStages = 6;
+constexpr uint32_t kPairTile = 2 * kBoxG;                  // 16 KB: 128 columns x 64 tokens
+constexpr uint32_t kPairStage = 2 * kPairTile;             // K | V
+constexpr size_t kSmemWidePair = 1024 + kPairStages * kPairStage + 2048 + 512;
+
+template <bool RELU, bool TOKB = false>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(wide_gram_threads(RELU || TOKB), 1)
+wide_gram_pair_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
+                      const __grid_constant__ CUtensorMap mapV) {
+    constexpr bool XF = RELU || TOKB;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* ring = smem;                                  // kPairStages x (K 16 KB | V 16 KB)
+    uint8_t* ones = ring + kPairStages * kPairStage;       // 2 KB of bf16 1.0 (ReLU)
+    uint64_t* full = reinterpret_cast<uint64_t*>(ones + 2048);
+    uint64_t* empty = full + kPairStages;
+    uint64_t* ready = empty + kPairStages;
+    uint64_t* accfull = ready + kPairStages;
+    uint64_t* accempty = accfull + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accempty + 1);
+    uint32_t* abort_flag = tmem_slot + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int cid = (int)cluster_id_x(), ncl = (int)ncluster_x();
+    const int D = p.D;
+    // 64-column boxes of this CTA's half that hold data (the rest stay zero)
+    const int nbl = max(0, min(2, (D + 63) / 64 - 2 * (int)rank));
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPairStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&ready[s], XF ? 8 : 1);
+        }
+        mbar_init(accfull, 1);
+        mbar_init(accempty, 16);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    for (int s = 0; s < kPairStages; ++s)
+        for (int t = 0; t < 2; ++t)
+            for (int b = nbl; b < 2; ++b) {
+                uint4* z = reinterpret_cast<uint4*>(ring + s * kPairStage + t * kPairTile + b * kBoxG);
+                for (int i = threadIdx.x; i < (int)(kBoxG / 16); i += blockDim.x)
+                    z[i] = make_uint4(0, 0, 0, 0);
+            }
+    if (RELU)
+        for (int i = threadIdx.x; i < 2048 / 4; i += blockDim.x)
+            reinterpret_cast<uint32_t*>(ones)[i] = 0x3F803F80u;
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, 512);
+        tmem_relinquish_pair();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();            // both CTAs' barriers, zero boxes and TMEM ready
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    const Abort ab{abort_flag, p.status};
+    const int nitems = p.BH * p.Fc;
+    const int nt = (p.S + kTokG - 1) / kTokG;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&mapK);
+            tma_prefetch_desc(&mapV);
+            const uint64_t pol = policy_evict_first();
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int item = cid; item < nitems && ok; item += ncl) {
+                const int frame = global_frame(p, item);
+                for (int t = 0; t < nt; ++t) {
+                    if (!(ok = mbar_wait(&empty[s], ph ^ 1, ab, 0x611))) break;
+                    uint8_t* st = ring + s * kPairStage;
+                    mbar_expect_tx(&full[s], 2 * nbl * kBoxG);
+                    for (int b = 0; b < nbl; ++b) {
+                        const int x = 128 * (int)rank + 64 * b;
+                        tma_load_3d(st + b * kBoxG, &mapK, &full[s], x, t * kTokG, frame, pol);
+                        tma_load_3d(st + kPairTile + b * kBoxG, &mapV, &full[s], x, t * kTokG,
+                                    frame, pol);
+                    }
+                    if (++s == kPairStages) { s = 0; ph ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            // ---------------- MMA issuer of the pair ----------------
+            const uint32_t idW = idesc_bf16(256, kDW, true, true);
+            const uint32_t idZ = idesc_bf16(256, 16, true, false);
+            const uint64_t ones_d = sdesc_sw128(smem_u32(ones), 16, 1024);
+            // GDN: G at columns [0, 256), B~ at [256, 512); ReLU: dM at [0, 256), dz at 256.
+            const uint32_t dA = tbase, dB = tbase + 256;
+            int s = 0, li = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int item = cid; item < nitems && ok; item += ncl, ++li) {
+                if (!(ok = mbar_wait(accempty, (li & 1) ^ 1, ab, 0x612, true))) break;
+                tc_fence_after();
+                for (int t = 0; t < nt; ++t) {
+                    if (!XF && !(ok = mbar_wait(&full[s], ph, ab, 0x613))) break;
+                    if (!(ok = mbar_wait(&ready[s], ph, ab, 0x614, true))) break;
+                    tc_fence_after();
+                    const uint32_t sk = smem_u32(ring + s * kPairStage), sv = sk + kPairTile;
+#pragma unroll
+                    for (int k = 0; k < kTokG / 16; ++k) {
+                        // A = this CTA's K columns ^T (MN-major, 2 boxes), B = K or V
+                        // (MN-major, this CTA's 128 of the N = 256 columns)
+                        const uint64_t ak = sdesc_sw128(sk + k * 2048, kBoxG, 1024);
+                        const uint64_t bv = sdesc_sw128(sv + k * 2048, kBoxG, 1024);
+                        const uint32_t acc = (t | k) ? 1u : 0u;
+                        if (RELU) {
+                            mma_bf16_pair(dA, ak, bv, idW, acc);
+                            mma_bf16_pair(dB, ak, ones_d, idZ, acc);
+                        } else {
+                            mma_bf16_pair(dA, ak, ak, idW, acc);
+                            mma_bf16_pair(dB, ak, bv, idW, acc);
+                        }
+                    }
+                    mma_commit_pair(&empty[s], 0);
+                    mma_commit_pair(&empty[s], 1);
+                    if (++s == kPairStages) { s = 0; ph ^= 1; }
+                }
+                if (ok) {
+                    mma_commit_pair(accfull, 0);
+                    mma_commit_pair(accfull, 1);
+                }
+            }
+        } else if (lane == 0 && !XF) {
+            // ---------------- odd CTA: forward each landed stage ----------------
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int item = cid; item < nitems && ok; item += ncl)
+                for (int t = 0; t < nt; ++t) {
+                    if (!(ok = mbar_wait(&full[s], ph, ab, 0x615))) break;
+                    mbar_arrive_cluster(&ready[s], 0);
+                    if (++s == kPairStages) { s = 0; ph ^= 1; }
+                }
+        }
+    } else if (XF && warp >= 6 && warp < 10) {
+        // ---------------- transform of this CTA's K (and V) columns ----------------
+        const int tl = threadIdx.x - 192;          // 0..127
+        const int row = tl & 63;
+        int s = 0;
+        uint32_t ph = 0;
+        bool ok = true;
+        for (int item = cid; item < nitems && ok; item += ncl) {
+            const float* bsrc = TOKB ? p.beta_tok + (size_t)global_frame(p, item) * p.S : nullptr;
+            float bv_next = (TOKB && row < p.S) ? __ldg(bsrc + row) : 0.f;   // gates one tile ahead
+            for (int t = 0; t < nt; ++t) {
+                const float bv = bv_next;
+                if (TOKB) {
+                    const int tok_n = (t + 1) * kTokG + row;
+                    bv_next = (t + 1 < nt && tok_n < p.S) ? __ldg(bsrc + tok_n) : 0.f;
+                }
+                if (!(ok = mbar_wait(&full[s], ph, ab, 0x616))) break;
+                uint8_t* st = ring + s * kPairStage;
+                if (TOKB) {
+                    // thread -> token row `row` of K (tl < 64) or V: 8 columns per chunk
+                    const float sb = sqrtf(fmaxf(bv, 0.f));
+                    const __nv_bfloat162 gsc = __floats2bfloat162_rn(sb, sb);
+                    uint8_t* const base = st + (tl >> 6) * kPairTile;
+                    for (int c = 0; c < 8 * nbl; ++c) {
+                        uint4* pc = reinterpret_cast<uint4*>(base + (c >> 3) * kBoxG + sw128_off(row, c & 7));
+                        uint4 x = *pc;
+                        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&x);
+                        h[0] = __hmul2(h[0], gsc); h[1] = __hmul2(h[1], gsc);
+                        h[2] = __hmul2(h[2], gsc); h[3] = __hmul2(h[3], gsc);
+                        *pc = x;
+                    }
+                } else {
+                    uint4* kt = reinterpret_cast<uint4*>(st);
+                    for (int i = tl; i < nbl * (int)kBoxG / 16; i += 128) {
+                        uint4 x = kt[i];
+                        x.x = relu_bf16x2(x.x); x.y = relu_bf16x2(x.y);
+                        x.z = relu_bf16x2(x.z); x.w = relu_bf16x2(x.w);
+                        kt[i] = x;
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(&ready[s], 0);
+                if (++s == kPairStages) { s = 0; ph ^= 1; }
+            }
+        }
+    } else if (warp >= 2) {
+        // ---------------- epilogue: key-row block r = rank ----------------
+        const int q = warp & 3, row = q * 32 + lane;
+        const int g = warp < 6 ? 0 : 1;                 // half of the accumulator columns
+        int li = 0;
+        bool ok = true;
+        for (int item = cid; item < nitems && ok; item += ncl, ++li) {
+            if (!(ok = mbar_wait(accfull, li & 1, ab, 0x617))) break;
+            tc_fence_after();
+            gram_readout<RELU, TOKB>(p, tbase + (uint32_t(q * 32) << 16), 2 * item + (int)rank, g, row);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(accempty, 0);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();            // no CTA leaves while its pair may still reach its memory
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tbase, 512);
 }
 
 // ============================================================================
@@ -909,6 +1163,19 @@ WideLayout wide_layout(const ScanArgs& a) {
 }
 
 constexpr size_t kSmemWideGram = 1024 + 3 * 2 * kGTile + 2048 + 256;
+static_assert(kSmemWidePair <= 232448, "pair gram smem");
+
+// LA_WIDE_PAIR=1 runs the gram on CTA pairs (cta_group::2) instead of one CTA
+// per key-row block.  The pair halves the operand bytes each SM loads and
+// reads, but the gram is not bound by them: the item's accumulator fills all
+// 512 TMEM columns, so the read-out and the next item's MMAs take turns, and
+// the pair adds a cross-CTA hand-off to every stage.  Measured slower (full
+// 512-frame D = 256 calls, GDN / ReLU: 4.65 / 5.72 ms on pairs, 4.49 / 5.03
+// ms one CTA per block), so the one-CTA kernel is the default.
+bool wide_pair_gram() {
+    const char* e = std::getenv("LA_WIDE_PAIR");
+    return e && e[0] == '1';
+}
 constexpr size_t kSmemWideChain = 1024 + 2 * kGImg + kMImg + 256;
 template <bool RELU>
 constexpr size_t smem_wide_out() {
@@ -972,12 +1239,16 @@ cudaError_t launch_wide_mode(const ScanArgs& a, cudaStream_t st) {
                           !make_tmap_bf16_3d(&mO, a.o, a.D, a.S, bhf, 64, kTokO)))
         return cudaErrorInvalidValue;
 
+    const bool pair = wide_pair_gram();
     {
-        const void* kernels[] = {a.beta_tok ? reinterpret_cast<const void*>(wide_gram_kernel<false, true>)
-                                            : reinterpret_cast<const void*>(wide_gram_kernel<RELU>),
-                                 reinterpret_cast<const void*>(wide_chain_gdn_kernel),
+        const void* gk = pair ? (a.beta_tok ? reinterpret_cast<const void*>(wide_gram_pair_kernel<false, true>)
+                                            : reinterpret_cast<const void*>(wide_gram_pair_kernel<RELU>))
+                              : (a.beta_tok ? reinterpret_cast<const void*>(wide_gram_kernel<false, true>)
+                                            : reinterpret_cast<const void*>(wide_gram_kernel<RELU>));
+        const void* kernels[] = {gk, reinterpret_cast<const void*>(wide_chain_gdn_kernel),
                                  reinterpret_cast<const void*>(wide_output_kernel<RELU>)};
-        const int bytes[] = {(int)kSmemWideGram, (int)kSmemWideChain, (int)smem_wide_out<RELU>()};
+        const int bytes[] = {(int)(pair ? kSmemWidePair : kSmemWideGram), (int)kSmemWideChain,
+                             (int)smem_wide_out<RELU>()};
         for (int i = 0; i < 3; ++i) {
             const cudaError_t e = ensure_dyn_smem(kernels[i], bytes[i]);
             if (e != cudaSuccess) return e;
@@ -1032,10 +1303,20 @@ cudaError_t launch_wide_mode(const ScanArgs& a, cudaStream_t st) {
         const int grid = std::min(items, share);
         // gram(c) overwrites the buffers chain(c - 2) read
         if (ci >= 2) ok(cudaStreamWaitEvent(st, cx.chain[b], 0));
-        if (!RELU && p.beta_tok)
+        if (pair) {
+            // one CTA pair per (b, h, f); the grid is a whole number of pairs
+            const int grid2 = 2 * std::max(1, std::min(p.BH * p.Fc, share / 2));
+            if (!RELU && p.beta_tok)
+                wide_gram_pair_kernel<false, true>
+                    <<<grid2, wide_gram_threads(true), kSmemWidePair, st>>>(p, mK, mV);
+            else
+                wide_gram_pair_kernel<RELU>
+                    <<<grid2, wide_gram_threads(RELU), kSmemWidePair, st>>>(p, mK, mV);
+        } else if (!RELU && p.beta_tok) {
             wide_gram_kernel<false, true><<<grid, wide_gram_threads(true), kSmemWideGram, st>>>(p, mK, mV);
-        else
+        } else {
             wide_gram_kernel<RELU><<<grid, wide_gram_threads(RELU), kSmemWideGram, st>>>(p, mK, mV);
+        }
         ok(cudaGetLastError());
         ok(cudaEventRecord(cx.gram[b], st));
         // chain(c) needs gram(c), and overwrites the images output(c - 2) read

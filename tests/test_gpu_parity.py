@@ -340,6 +340,53 @@ def test_wide_tensor_core_path_matches_simt_path(mode, D, monkeypatch):
     assert rel_err(to_np(m_tc), to_np(m_simt)) <= TOL_BF16
 
 
+@pytest.mark.parametrize("mode", ["relu", "gdn", "gdn_token_beta"])
+@pytest.mark.parametrize("D", [144, 192, 256])
+def test_wide_gram_on_cta_pairs_matches_one_cta_kernel(mode, D, monkeypatch):
+    """With LA_WIDE_PAIR=1 the wide gram runs on CTA pairs (M = 256 MMAs, each
+    CTA holding its 128 key columns of K and V); the default one-CTA-per-key-row-
+    block kernel computes the same products with M = 128 MMAs over whole tiles.  Both sum the same
+    16-token slices in the same order into fp32, so they agree to rounding, and
+    both match the oracle (ragged last token tile, key columns past D padded)."""
+    spec = synth.small(B=2, H=2, F=7, S=200, D=D, dtype="bf16", seed=47, keys_l2=True,
+                       alpha=("sigmoid_normal", 3.0, 1.0), beta=("sigmoid_normal", 0.0, 1.0))
+    inp = device_inputs(spec)
+    B, H, F, S = spec.B, spec.H, spec.F, spec.S
+    m0n, z0n = synth.random_state(spec, 0.05)
+    m0, z0 = torch.from_numpy(m0n).cuda(), torch.from_numpy(z0n).cuda()
+    if mode == "gdn_token_beta":
+        gates = torch.from_numpy(synth.token_gates(spec)).cuda()
+        assert la.la_plan(la.LA_MODE_GDN_TOKEN_BETA, la.LA_BF16, B, H, F, S, D)[0] == "tcgen05_wide"
+
+        def run():
+            so = torch.empty((B, H, D, D), device="cuda")
+            ws = la.workspace_for(la.LA_MODE_GDN_TOKEN_BETA, B, H, F, S, D)
+            o = la.la_scan_gdn_token_beta(inp["q"], inp["k"], inp["v"], inp["alpha"], gates,
+                                          spec.k_scale, state_in=m0, state_out=so, workspace=ws)
+            _check_status(ws)
+            return o, so, None
+    else:
+        m = la.LA_MODE_GDN if mode == "gdn" else la.LA_MODE_RELU
+        assert la.la_plan(m, la.LA_BF16, B, H, F, S, D)[0] == "tcgen05_wide"
+
+        def run():
+            return _run(spec, mode, inp, m0, z0 if mode == "relu" else None)
+    monkeypatch.setenv("LA_WIDE_PAIR", "1")
+    o_p, m_p, z_p = run()
+    monkeypatch.delenv("LA_WIDE_PAIR")
+    o_1, m_1, z_1 = run()
+    torch.cuda.synchronize()
+    assert torch.isfinite(o_p.float()).all() and torch.isfinite(m_p).all()
+    e_o = rel_err(to_np(o_p), to_np(o_1))
+    e_m = rel_err(to_np(m_p), to_np(m_1))
+    print(f"\n[pair vs one-CTA gram] {mode} D={D}: output {e_o:.3e} state {e_m:.3e}")
+    assert e_o <= 1e-2 * TOL_BF16 and e_m <= 1e-2 * TOL_BF16
+    if mode == "relu":
+        assert rel_err(to_np(z_p), to_np(z_1)) < 1e-6
+    if mode != "gdn_token_beta":
+        _compare(spec, mode, with_state=True)
+
+
 @pytest.mark.parametrize("mode", ["relu", "gdn"])
 def test_wide_path_chunking_is_exact(mode, monkeypatch):
     """The wide path pipelines frame chunks and carries the fp32 state between
