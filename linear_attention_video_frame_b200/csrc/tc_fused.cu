@@ -31,6 +31,8 @@
 //                    in frame order, so frame f is out once the flag of its
 //                    parity reaches f + 1)
 //   output -> chain: mimg_consumed[slot] = f + 1 once the image is in smem
+//                    (with output items split in token halves: each half adds 1
+//                    and the slot of frame f is free once it counts 2 (f / kRM))
 //   chain -> gram  : chain_done[head][g & 1] >= g + 1, g = f - kRG, frees gram
 //                    slot f (frame g was consumed before it was published)
 // Every spin is bounded; a block that gives up records LA_ERR_TIMEOUT in the
@@ -150,6 +152,7 @@ struct FusedParams {
     int den_col;               // ReLU, D <= 112: z_f rides in column D (hi) and D + 1 (lo) of
                                // the state image, so one MMA gives numerator and denominator
     int skip_publish;          // test hook: frame of head 0 whose gram_ready is never set
+    int out_split;             // output items cover one token half of a frame each (Item.pad)
     // fused input preparation (GDN, PREP instantiation): RMSNorm, ReLU, 3D RoPE of K and Q
     int H;
     const float* q_weight;     // [H, D] or NULL
@@ -190,20 +193,36 @@ __device__ __forceinline__ Item decode_ticket(const FusedParams& p, uint32_t t) 
         if (t < BH * F) it = Item{kItemGram, (int)(t % BH), (int)(t / BH), 0};
         return it;
     }
+    // output items per (head, frame): the frame, or its two token halves
+    // (part in Item.pad; all heads' first halves, then all second halves)
+    const uint32_t no = p.out_split ? 2 : 1, per = (1 + no) * BH;
     const uint32_t L = p.lag;
     const uint32_t g0 = min(L, F) * BH;
     if (t < g0) return Item{kItemGram, (int)(t % BH), (int)(t / BH), 0};
     uint32_t u = t - g0;
     const uint32_t nm = F > L ? F - L : 0;
-    if (u < nm * 2 * BH) {
-        const uint32_t j = L + u / (2 * BH), r = u % (2 * BH);
+    if (u < nm * per) {
+        const uint32_t j = L + u / per, r = u % per;
         if (r < BH) return Item{kItemGram, (int)r, (int)j, 0};
-        return Item{kItemOut, (int)(r - BH), (int)(j - L), 0};
+        const uint32_t o = r - BH;
+        return Item{kItemOut, (int)(o % BH), (int)(j - L), (int)(o / BH)};
     }
-    u -= nm * 2 * BH;
+    u -= nm * per;
     const uint32_t f0 = F > L ? F - L : 0;
-    if (u < (F - f0) * BH) return Item{kItemOut, (int)(u % BH), (int)(f0 + u / BH), 0};
+    if (u < (F - f0) * no * BH) {
+        const uint32_t o = u % (no * BH);
+        return Item{kItemOut, (int)(o % BH), (int)(f0 + u / (no * BH)), (int)(o / BH)};
+    }
     return it;
+}
+
+// Output tiles [lo, hi) of an output item: the whole frame, or one of its two
+// token halves (split only when a frame has at least two output tiles).
+__device__ __forceinline__ void out_range(const FusedParams& p, const Item& it, int nto, int& lo,
+                                          int& hi) {
+    const int h = (nto + 1) >> 1;
+    lo = (p.out_split && it.pad) ? h : 0;
+    hi = (p.out_split && !it.pad) ? h : nto;
 }
 
 // ============================================================================
@@ -347,9 +366,11 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                             if (RELU) bulk_load_hint(zbuf, p.zf + ms * 128, 512, mfull, pol);
                         }
                     };
-                    const int early = LA_FUSED_EARLY_Q ? min(nto, kWStages) : 0;
-                    for (int t = 0; t < nto; ++t) {
-                        if (t == early) fetch_state();
+                    int t_lo, t_hi;
+                    out_range(p, it, nto, t_lo, t_hi);
+                    const int early = LA_FUSED_EARLY_Q ? min(t_hi - t_lo, kWStages) : 0;
+                    for (int t = t_lo; t < t_hi; ++t) {
+                        if (t - t_lo == early) fetch_state();
                         ok = ok && mbar_wait(&empty[s], ph ^ 1, ab, 0x406);
                         if (ok) {
                             uint8_t* st = ring + s * 32768;
@@ -359,7 +380,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                         }
                         if (++s == kWStages) { s = 0; ph ^= 1; }
                     }
-                    if (early == nto) fetch_state();
+                    if (early == t_hi - t_lo) fetch_state();
                 }
             }
         }
@@ -417,9 +438,13 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                     if (!(ok = mbar_wait(mfull, nout & 1, ab, 0x415))) break;
                     ++nout;
                     // The image is in shared memory: its ring slot may be rewritten.
-                    st_release_gpu(&p.mimg_consumed[(size_t)it.bh * kRM + it.f % kRM], it.f + 1);
+                    uint32_t* mc = &p.mimg_consumed[(size_t)it.bh * kRM + it.f % kRM];
+                    if (p.out_split) add_release_gpu(mc, 1u);
+                    else st_release_gpu(mc, it.f + 1);
                     const uint32_t mb = smem_u32(mbuf);
-                    for (int t = 0; t < nto && ok; ++t) {
+                    int t_lo, t_hi;
+                    out_range(p, it, nto, t_lo, t_hi);
+                    for (int t = t_lo; t < t_hi && ok; ++t) {
                         const uint32_t qa = qctr & 3;
                         ok = mbar_wait(&qempty[qa], ((qctr >> 2) & 1) ^ 1, ab, 0x416) &&
                              mbar_wait((RELU || PREP) ? &xform[s] : &full[s], ph, ab, 0x417);
@@ -545,7 +570,9 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                     LA_TRACE_EVENT(5, frame);
                 }
             } else {
-                for (int t = 0; t < nto; ++t) {
+                int t_lo, t_hi;
+                out_range(p, it, nto, t_lo, t_hi);
+                for (int t = t_lo; t < t_hi; ++t) {
                     const uint32_t qa = qctr & 3;
                     if (leader) {
                         ok = ok && mbar_wait(&qfull[qa], (qctr >> 2) & 1, ab, 0x424);
@@ -596,7 +623,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                         if (leader && go) {
                             tma_store_3d_hint(mO, sb, blk * 64, t * kTokO, frame, pol_stream);
                             bulk_commit();
-                            if (t == nto - 1 && blk == nblk - 1) LA_TRACE_EVENT(6, frame);
+                            if (t == t_hi - 1 && blk == nblk - 1) LA_TRACE_EVENT(6, frame);
                         }
                     }
                 }
@@ -653,10 +680,11 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                     prep_t[i] = make_float2(c, sn);
                 }
             named_bar_sync(2, 192);
-            const int ntile = gram ? ntg : nto;
+            int t_lo = 0, t_hi = ntg;
+            if (!gram) out_range(p, it, nto, t_lo, t_hi);
             const int rows = gram ? kTokG : kTokO;
             const uint32_t box = gram ? kBoxG : kBoxO;
-            for (int t = 0; t < ntile; ++t) {
+            for (int t = t_lo; t < t_hi; ++t) {
                 if (leader) {
                     ok = ok && mbar_wait(&full[s], ph, ab, 0x442);
                     bc2[bcn & 1] = ok;
@@ -764,7 +792,9 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                 p.beta_tok + ((size_t)it.bh * F + step_frame(it.f, F, p.rev_chunk)) * p.S;
             // the gates of a tile are fetched one tile ahead, off the critical path
             float bv_next = (gram && row < p.S) ? __ldg(bsrc + row) : 0.f;
-            for (int t = 0; t < (gram ? ntg : nto); ++t) {
+            int t_lo = 0, t_hi = ntg;
+            if (!gram) out_range(p, it, nto, t_lo, t_hi);
+            for (int t = t_lo; t < t_hi; ++t) {
                 const float bv = bv_next;
                 const int tok_n = (t + 1) * kTokG + row;
                 bv_next = (gram && t + 1 < ntg && tok_n < p.S) ? __ldg(bsrc + tok_n) : 0.f;
@@ -844,7 +874,9 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
             } else {
                 if (leader) ok = ok && mbar_wait(mfull, nout & 1, ab, 0x433);
                 ++nout;
-                for (int t = 0; t < nto; ++t) {
+                int t_lo, t_hi;
+                out_range(p, it, nto, t_lo, t_hi);
+                for (int t = t_lo; t < t_hi; ++t) {
                     const uint32_t qa = qctr & 3;
                     if (leader) {
                         if (!p.den_col)
@@ -1203,8 +1235,10 @@ __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) 
             int i = 0;                    // this frame is the i-th of its parity
             for (int f = par; f < F; f += 2, ++i) {
                 const size_t msidx = (size_t)bh * kRM + f % kRM;
-                if (p.want_output && f >= kRM && seen < (uint32_t)(f - kRM + 1) &&
-                    !wait_flag_ge(&p.mimg_consumed[msidx], f - kRM + 1, ab, 0x509))
+                // the slot's previous frame f - kRM has been read by its output item(s)
+                const uint32_t need = p.out_split ? 2u * (uint32_t)(f / kRM) : (uint32_t)(f - kRM + 1);
+                if (p.want_output && f >= kRM && seen < need &&
+                    !wait_flag_ge(&p.mimg_consumed[msidx], need, ab, 0x509))
                     break;
                 LA_TRACE_EVENT(24, (uint64_t)bh * F + f);
                 if (!mbar_wait(&iready[par], i & 1, ab, 0x508)) break;
@@ -1343,6 +1377,16 @@ cudaError_t launch_fused_mode(const ScanArgs& a, cudaStream_t st) {
     p.frame_offset = a.prep.frame_offset;
     p.rope_base = p.rope ? a.prep.rope_base : 10000.f;
     p.skip_publish = -1;
+    // Split output items into token halves when there are few per worker
+    // (short clips: the last frames' outputs otherwise leave most workers
+    // idle); LA_FUSED_OUT_SPLIT=0/1 overrides.
+    {
+        const int nto = (a.S + 127) / 128;
+        const long workers = std::max(1, device_sm_count() - p.BH);
+        p.out_split = (nto >= 2 && (long)p.BH * p.F < 4 * workers) ? 1 : 0;
+        if (const char* e = std::getenv("LA_FUSED_OUT_SPLIT"))
+            p.out_split = (e[0] == '1' && nto >= 2) ? 1 : 0;
+    }
     if (const char* e = std::getenv("LA_SCAN_TEST_SKIP_PUBLISH")) p.skip_publish = std::atoi(e);
     const int nsm = device_sm_count();
     p.n_chain = p.BH;                 // one chain block per (b, h)

@@ -467,6 +467,61 @@ def test_fused_kernel_matches_three_kernel_path(mode, monkeypatch):
         assert rel_err(to_np(z_f), to_np(z_3)) < 1e-5
 
 
+@pytest.mark.parametrize("mode", ["relu", "gdn", "gdn_reverse", "gdn_token_beta"])
+def test_fused_output_items_in_token_halves_are_exact(mode, monkeypatch):
+    """Short clips split each output item into two token halves (two items
+    read the frame's state image; the chain reuses the slot after both).  Each
+    output tile is computed the same way either way, so the bits agree; 21
+    frames reuse every hand-off slot; S = 650 leaves a ragged last tile."""
+    spec = synth.small(B=2, H=6, F=21, S=650, D=112 if mode == "relu" else 128, dtype="bf16",
+                       seed=75, keys_l2=True,
+                       alpha=("sigmoid_normal", 3.0, 1.0), beta=("sigmoid_normal", 0.0, 1.0))
+    B, H, F, S, D = spec.B, spec.H, spec.F, spec.S, spec.D
+    inp = device_inputs(spec)
+    m0n, z0n = synth.random_state(spec, 0.05)
+    m0, z0 = torch.from_numpy(m0n).cuda(), torch.from_numpy(z0n).cuda()
+    gates = torch.from_numpy(synth.token_gates(spec)).cuda() if mode == "gdn_token_beta" else None
+    mcode = {"relu": la.LA_MODE_RELU, "gdn": la.LA_MODE_GDN, "gdn_reverse": la.LA_MODE_GDN_REVERSE,
+             "gdn_token_beta": la.LA_MODE_GDN_TOKEN_BETA}[mode]
+    assert la.la_plan(mcode, la.LA_BF16, B, H, F, S, D) == ("tcgen05_fused", 1)
+
+    def run():
+        ws = la.workspace_for(mcode, B, H, F, S, D)
+        so = torch.empty((B, H, D, D), device="cuda")
+        zo = torch.empty((B, H, D), device="cuda")
+        if mode == "relu":
+            o = la.la_scan_relu(inp["q"], inp["k"], inp["v"], state_in=m0, z_in=z0, state_out=so,
+                                z_out=zo, eps=spec.eps, workspace=ws)
+        elif mode == "gdn":
+            o = la.la_scan_gdn(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"],
+                               spec.k_scale, state_in=m0, state_out=so, workspace=ws)
+        elif mode == "gdn_reverse":
+            o = la.la_scan_gdn_reverse(inp["q"], inp["k"], inp["v"], inp["alpha"], inp["beta"],
+                                       spec.k_scale, 8, workspace=ws)
+            so = None
+        else:
+            o = la.la_scan_gdn_token_beta(inp["q"], inp["k"], inp["v"], inp["alpha"], gates,
+                                          spec.k_scale, state_in=m0, state_out=so, workspace=ws)
+        _check_status(ws)
+        return o, so, zo
+
+    runs = []
+    for split in ("1", "0"):
+        monkeypatch.setenv("LA_FUSED_OUT_SPLIT", split)
+        runs.append(run())
+    torch.cuda.synchronize()
+    (o1, s1, z1), (o0, s0, z0_) = runs
+    assert torch.isfinite(o1.float()).all()
+    assert torch.equal(o1.view(torch.int16), o0.view(torch.int16))
+    if s1 is not None:
+        assert torch.equal(s1, s0)
+    if mode == "relu":
+        assert torch.equal(z1, z0_)
+    if mode in ("relu", "gdn"):
+        monkeypatch.setenv("LA_FUSED_OUT_SPLIT", "1")
+        _compare(spec, mode, with_state=True, heads=[(0, 0), (1, 5)])
+
+
 @pytest.mark.parametrize("mode", ["relu", "gdn"])
 def test_fused_kernel_at_its_head_limit_with_slot_reuse(mode):
     # 49 (b, h) pairs: one chain block each on a 148-SM B200 (the fused
