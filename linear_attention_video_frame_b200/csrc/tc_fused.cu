@@ -261,7 +261,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
         for (int s = 0; s < kWStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-            mbar_init(&xform[s], PREP ? 6 : 4);
+            mbar_init(&xform[s], (PREP || TOKB) ? 6 : 4);      // transform warps
         }
         mbar_init(mfull, 1);
         mbar_init(mempty, RELU ? 5 : 1);
@@ -753,22 +753,24 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                 if (++s == kWStages) { s = 0; ph ^= 1; }
             }
         }
-    } else if (TOKB && warp < 10) {
+    } else if (TOKB) {
         // ---------------- per-token update gate: sqrt(beta_t) on K and V rows ----------------
         // Every token row of a gram item's K and V tiles is scaled by
         // sqrt(beta_t) in shared memory (bf16), so the unchanged contractions
         // give Kh^T diag(beta) Kh and Kh^T diag(beta) V (SANA-WM paper
         // summary, section 3, "Hybrid GDN/Softmax Attention", per-token update
-        // gate).  Thread tl scales row tl % 64 of K (tl < 64) or of V; output
-        // tiles pass untouched (through the same barrier protocol).
-        const int tl = threadIdx.x - 192;          // 0..127
+        // gate).  Six warps: unit u = tl + 192 i of a tile is 16-byte chunk
+        // (u / 64) % nch of row u % 64 of K (u < 64 nch) or V, so a thread
+        // always works on row tl % 64 and needs one gate per tile.  Every
+        // thread waits for the stage itself (no barrier per tile); output
+        // tiles pass untouched through the same wait / arrive protocol.
+        const int tl = threadIdx.x - 192;          // 0..191
         const bool leader = (tl == 0);
         const int row = tl & 63;
-        const int nch = D / 8;
-        uint32_t iq = 0, ph = 0, bcn = 0;
+        const int nch = D / 8, nunits = 2 * 64 * nch;
+        uint32_t iq = 0, ph = 0;
         int s = 0;
         bool ok = true;
-        int* bc2 = bc_ok + 2;
         while (true) {
             if (leader) {
                 const int qi = iq % kIQ;
@@ -781,8 +783,9 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                 bc_item[1] = it;
             }
             ++iq;
-            named_bar_sync(2, 128);
+            named_bar_sync(2, 192);
             const Item it = bc_item[1];
+            named_bar_sync(2, 192);                // bc_item read before the next write
             if (it.type == kItemStop) break;
             // Output tiles are not touched, but they pass through the same
             // wait / arrive protocol: every use of a ring stage completes one
@@ -798,18 +801,17 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                 const float bv = bv_next;
                 const int tok_n = (t + 1) * kTokG + row;
                 bv_next = (gram && t + 1 < ntg && tok_n < p.S) ? __ldg(bsrc + tok_n) : 0.f;
-                if (leader) {
-                    ok = ok && mbar_wait(&full[s], ph, ab, 0x452);
-                    bc2[bcn & 1] = ok;
-                }
-                named_bar_sync(2, 128);
-                if (bc2[(bcn++) & 1] && gram) {
+                ok = ok && mbar_wait(&full[s], ph, ab, 0x452);
+                if (ok && gram) {
                     const float sb = sqrtf(fmaxf(bv, 0.f));
                     const __nv_bfloat162 g = __floats2bfloat162_rn(sb, sb);
-                    uint8_t* const base = ring + s * 32768 + (tl >> 6) * 16384;   // K or V
+                    uint8_t* const tile = ring + s * 32768;
 #pragma unroll 4
-                    for (int c = 0; c < nch; ++c) {
-                        uint4* pc = reinterpret_cast<uint4*>(base + (c >> 3) * kBoxG + sw128_off(row, c & 7));
+                    for (int u = tl; u < nunits; u += 192) {
+                        const int tv = u >= 64 * nch ? 1 : 0;                 // K or V
+                        const int c = (u - tv * 64 * nch) >> 6;
+                        uint4* pc = reinterpret_cast<uint4*>(tile + tv * 16384 + (c >> 3) * kBoxG +
+                                                             sw128_off(row, c & 7));
                         uint4 x = *pc;
                         __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&x);
                         h[0] = __hmul2(h[0], g); h[1] = __hmul2(h[1], g);
