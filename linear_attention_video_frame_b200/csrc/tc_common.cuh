@@ -106,6 +106,41 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     }
 }
 
+// True once this block or another block of the call gave up.
+__device__ __forceinline__ bool aborted(const Abort& ab) {
+    return ab.raised() || *reinterpret_cast<volatile unsigned int*>(ab.status) != 0;
+}
+
+// After an abort: wait, up to kDrainNs and whatever the abort flag says, for
+// the phase of `bar` with parity `parity` to complete, i.e. for the copies or
+// MMAs that arrive on it to land, so that none is still in flight when the
+// block frees its tensor memory and exits.
+constexpr uint64_t kDrainNs = 50000000ull;   // 50 ms
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return;
+    const uint64_t t0 = global_timer_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_timer_ns() - t0 > kDrainNs) return;
+}
+
+// Parity of the last phase a role armed on each barrier of a ring (the
+// producer's loads on full[s], the MMA issuer's commits on empty[s]), as two
+// register bitmasks: bit s of `used` set once stage s was armed, bit s of
+// `par` the parity of its last armed phase.
+struct PhaseLog {
+    uint32_t used = 0, par = 0;
+    __device__ __forceinline__ void note(int s, uint32_t ph) {
+        used |= 1u << s;
+        par = (par & ~(1u << s)) | ((ph & 1u) << s);
+    }
+    // Only after an abort: the normal path consumed every phase it armed.
+    __device__ __forceinline__ void drain_if_aborted(uint64_t* bars, int n, const Abort& ab) const {
+        if (!aborted(ab)) return;
+        for (int s = 0; s < n && s < 32; ++s)
+            if ((used >> s) & 1u) mbar_drain(&bars[s], (par >> s) & 1u);
+    }
+};
+
 // ----------------------------------------------------------------------------
 // Proxy fences
 // ----------------------------------------------------------------------------

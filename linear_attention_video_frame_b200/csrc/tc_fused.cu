@@ -319,6 +319,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
             uint32_t iq = 0, nout = 0, ph = 0;
             int s = 0;
             bool ok = true;
+            PhaseLog armed, armed_m;     // loads in flight are waited for after an abort
             LA_TRACE_WRITER(0);
             while (true) {
                 Item it{kItemStop, 0, 0, 0};
@@ -346,6 +347,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                             tma_load_3d(st + kBoxG, mK, &full[s], 64, t * kTokG, frame, pol);
                             tma_load_3d(st + 16384, mV, &full[s], 0, t * kTokG, frame, pol);
                             tma_load_3d(st + 16384 + kBoxG, mV, &full[s], 64, t * kTokG, frame, pol);
+                            armed.note(s, ph);
                         }
                         if (++s == kWStages) { s = 0; ph ^= 1; }
                     }
@@ -364,6 +366,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                             mbar_expect_tx(mfull, kImg + (RELU ? 512 : 0));
                             bulk_load_hint(mbuf, p.mimg + ms * kImg, kImg, mfull, pol);
                             if (RELU) bulk_load_hint(zbuf, p.zf + ms * 128, 512, mfull, pol);
+                            armed_m.note(0, (nout - 1) & 1);
                         }
                     };
                     int t_lo, t_hi;
@@ -377,12 +380,15 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                             mbar_expect_tx(&full[s], 2 * kBoxO);
                             tma_load_3d(st, mQ, &full[s], 0, t * kTokO, frame, pol);
                             tma_load_3d(st + kBoxO, mQ, &full[s], 64, t * kTokO, frame, pol);
+                            armed.note(s, ph);
                         }
                         if (++s == kWStages) { s = 0; ph ^= 1; }
                     }
                     if (early == t_hi - t_lo) fetch_state();
                 }
             }
+            armed.drain_if_aborted(full, kWStages, ab);
+            armed_m.drain_if_aborted(mfull, 1, ab);
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
@@ -394,6 +400,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
             uint32_t iq = 0, ph = 0, qctr = 0, nout = 0;
             int s = 0;
             bool ok = true;
+            PhaseLog armed;     // MMAs in flight are waited for after an abort
             while (ok) {
                 const int qi = iq % kIQ;
                 if (!(ok = mbar_wait(&iqfull[qi], (iq / kIQ) & 1, ab, 0x411))) break;
@@ -429,6 +436,7 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                             }
                         }
                         mma_commit(&empty[s]);
+                        armed.note(s, ph);
                         if (++s == kWStages) { s = 0; ph ^= 1; }
                     }
                     if (!ok) break;
@@ -459,12 +467,14 @@ __device__ __forceinline__ void worker_role(const FusedParams& p, uint8_t* smem,
                         }
                         mma_commit(&empty[s]);
                         mma_commit(&qfull[qa]);
+                        armed.note(s, ph);
                         if (++s == kWStages) { s = 0; ph ^= 1; }
                     }
                     if (!ok) break;
                     mma_commit(mempty);
                 }
             }
+            armed.drain_if_aborted(empty, kWStages, ab);
         }
     } else if (warp < 6) {
         // ---------------- epilogue (4 warps; the leader waits, all follow) ----------------
@@ -1005,6 +1015,7 @@ __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) 
             int s = 0;
             uint32_t ph = 0;
             const uint64_t pol_last_use = LA_POL_STREAM();
+            PhaseLog armed;     // loads in flight are waited for after an abort
             LA_TRACE_WRITER(0);
             for (int f = 0; f < F; ++f) {
                 const size_t sidx = (size_t)bh * kRG + f % kRG;
@@ -1022,14 +1033,17 @@ __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) 
                     bulk_load_hint(st, p.dz + sidx * 128, 512, &gfull[s], pol_last_use);
                 }
                 bulk_load_hint(st + kImg, p.bimg + sidx * kImg, kImg, &gfull[s], pol_last_use);
+                armed.note(s, ph);
                 if (++s == kCStages) { s = 0; ph ^= 1; }
             }
+            armed.drain_if_aborted(gfull, kCStages, ab);
         }
     } else if (warp == 1) {
         // ---------------- MMA (GDN): D[:, half] += G'' bf16(M_{f-1})[:, half] ----------------
         if (!RELU && lane == 0) {
             int s = 0;
             uint32_t ph = 0;
+            PhaseLog armed, armed_h;     // MMAs in flight are waited for after an abort
             LA_TRACE_WRITER(3);
             for (int f = 0; f < F; ++f) {
                 if (!mbar_wait(&gfull[s], ph, ab, 0x503)) break;
@@ -1049,11 +1063,15 @@ __device__ __forceinline__ void chain_role(const FusedParams& p, uint8_t* smem) 
                         mma_bf16(tM + 64 * h, ad, bd, idH, 1u);
                     }
                     mma_commit(&mdone[h]);
+                    armed_h.note(h, f & 1);
                 }
                 if (!ok) break;
                 mma_commit(&gempty[s]);
+                armed.note(s, ph);
                 if (++s == kCStages) { s = 0; ph ^= 1; }
             }
+            armed.drain_if_aborted(gempty, kCStages, ab);
+            armed_h.drain_if_aborted(mdone, nhalf, ab);
         }
     } else if (warp < 10) {
         // ---------------- epilogue: two independent column halves ----------------

@@ -168,6 +168,7 @@ tc_gram_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapK,
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
+            PhaseLog armed;     // loads in flight are waited for after an abort
             for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
             const int item = global_item(p, it);
                 for (int t = 0; t < nt; ++t) {
@@ -178,9 +179,11 @@ tc_gram_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapK,
                     tma_load_3d(st + kBoxG, &mapK, &full[s], 64, t * kTokG, item, pol);
                     tma_load_3d(st + 16384, &mapV, &full[s], 0, t * kTokG, item, pol);
                     tma_load_3d(st + 16384 + kBoxG, &mapV, &full[s], 64, t * kTokG, item, pol);
+                    armed.note(s, ph);
                     if (++s == kGStages) { s = 0; ph ^= 1; }
                 }
             }
+            armed.drain_if_aborted(full, kGStages, ab);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -190,6 +193,7 @@ tc_gram_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapK,
             int s = 0, li = 0;
             uint32_t ph = 0;
             bool ok = true;
+            PhaseLog armed;
             for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++li) {
             const int item = global_item(p, it);
                 const int slot = li & 1;
@@ -215,10 +219,12 @@ tc_gram_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapK,
                         }
                     }
                     mma_commit(&empty[s]);
+                    armed.note(s, ph);
                     if (++s == kGStages) { s = 0; ph ^= 1; }
                 }
                 if (ok) mma_commit(&accfull[slot]);
             }
+            armed.drain_if_aborted(empty, kGStages, ab);    // MMAs in flight
         }
     } else if (warp < 6) {
         // ---------------- epilogue: TMEM -> workspace ----------------
@@ -419,6 +425,7 @@ tc_chain_kernel(const TcParams p) {
         if (lane == 0) {
             int s = 0;
             uint32_t ph = 0;
+            PhaseLog armed;     // loads in flight are waited for after an abort
             for (int f = 0; f < nsteps; ++f) {
                 if (!mbar_wait(&empty[s], ph ^ 1, ab, 0x201)) break;
                 const size_t frame = (size_t)bh * F + step_frame(p.f0 + f, F, p.rev_chunk);
@@ -433,14 +440,17 @@ tc_chain_kernel(const TcParams p) {
                     bulk_load(st, p.bmat + frame * (kQuadMat / 4), kQuadMat, &full[s]);
                     bulk_load(st + kQuadMat, p.dz + frame * 128, 512, &full[s]);
                 }
+                armed.note(s, ph);
                 if (++s == kCStages) { s = 0; ph ^= 1; }
             }
+            armed.drain_if_aborted(full, kCStages, ab);
         }
     } else if (warp == 1) {
         if (!RELU && lane == 0) {
             const uint32_t idC = idesc_bf16(128, D, false, true, /*negate_a=*/true);
             int s = 0;
             uint32_t ph = 0;
+            PhaseLog armed;     // MMAs in flight are waited for after an abort
             for (int f = 0; f < nsteps; ++f) {
                 if (!mbar_wait(&full[s], ph, ab, 0x202)) break;
                 if (!mbar_wait(mready, f & 1, ab, 0x203)) break;
@@ -453,8 +463,10 @@ tc_chain_kernel(const TcParams p) {
                 }
                 mma_commit(mdone);
                 mma_commit(&empty[s]);
+                armed.note(s, ph);
                 if (++s == kCStages) { s = 0; ph ^= 1; }
             }
+            armed.drain_if_aborted(empty, kCStages, ab);
         }
     } else {
         // ------------- epilogue: thread <-> (state row, column half) -------------
@@ -670,6 +682,7 @@ tc_output_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapQ,
             int s = 0, li = 0;
             uint32_t ph = 0;
             bool ok = true;
+            PhaseLog armed_q, armed_m;     // loads in flight are waited for after an abort
             for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++li) {
             const int item = global_item(p, it);
                 const int mb = li & 1;
@@ -677,15 +690,19 @@ tc_output_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapQ,
                 mbar_expect_tx(&mfull[mb], kImg + (RELU ? 512 : 0));
                 bulk_load(mbuf + mb * kImg, p.mimg + (size_t)item * kImg, kImg, &mfull[mb]);
                 if (RELU) bulk_load(zbuf + mb * 128, p.zf + (size_t)item * 128, 512, &mfull[mb]);
+                armed_m.note(mb, (li >> 1) & 1);
                 for (int t = 0; t < nt; ++t) {
                     if (!(ok = mbar_wait(&qempty[s], ph ^ 1, ab, 0x302))) break;
                     uint8_t* st = qring + s * 32768;
                     mbar_expect_tx(&qfull[s], 2 * kBoxO);
                     tma_load_3d(st, &mapQ, &qfull[s], 0, t * kTokO, item, pol);
                     tma_load_3d(st + kBoxO, &mapQ, &qfull[s], 64, t * kTokO, item, pol);
+                    armed_q.note(s, ph);
                     if (++s == kOStages) { s = 0; ph ^= 1; }
                 }
             }
+            armed_q.drain_if_aborted(qfull, kOStages, ab);
+            armed_m.drain_if_aborted(mfull, 2, ab);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -693,6 +710,7 @@ tc_output_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapQ,
             int s = 0, li = 0, gt = 0;
             uint32_t ph = 0;
             bool ok = true;
+            PhaseLog armed;     // MMAs in flight are waited for after an abort
             for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++li) {
             const int item = global_item(p, it);
                 const int mb = li & 1;
@@ -711,10 +729,12 @@ tc_output_kernel(const TcParams p, const __grid_constant__ CUtensorMap mapQ,
                     }
                     mma_commit(&qempty[s]);
                     mma_commit(&accfull[a]);
+                    armed.note(s, ph);
                     if (++s == kOStages) { s = 0; ph ^= 1; }
                 }
                 if (ok) mma_commit(&mempty[mb]);
             }
+            armed.drain_if_aborted(qempty, kOStages, ab);
         }
     } else if (warp < 6) {
         // ---------------- epilogue: TMEM -> bf16 -> TMA store ----------------

@@ -257,6 +257,7 @@ wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
+            PhaseLog armed;     // loads in flight are waited for after an abort
             for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x) {
                 const int frame = global_frame(p, item >> 1);
                 for (int t = 0; t < nt; ++t) {
@@ -268,9 +269,11 @@ wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
                         tma_load_3d(st + kGTile + b * kBoxG, &mapV, &full[s], 64 * b, t * kTokG,
                                     frame, pol);
                     }
+                    armed.note(s, ph);
                     if (++s == kStages) { s = 0; ph ^= 1; }
                 }
             }
+            armed.drain_if_aborted(full, kStages, ab);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -282,6 +285,7 @@ wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
             int s = 0, li = 0;
             uint32_t ph = 0;
             bool ok = true;
+            PhaseLog armed;     // MMAs in flight are waited for after an abort
             for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
                 const int r = item & 1;
                 if (!(ok = mbar_wait(accempty, (li & 1) ^ 1, ab, 0x602))) break;
@@ -306,10 +310,12 @@ wide_gram_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapK,
                         }
                     }
                     mma_commit(&empty[s]);
+                    armed.note(s, ph);
                     if (++s == kStages) { s = 0; ph ^= 1; }
                 }
                 if (ok) mma_commit(accfull);
             }
+            armed.drain_if_aborted(empty, kStages, ab);
         }
     } else if (TOKB && warp >= 6 && warp < 10) {
         // ---------------- per-token gate: sqrt(beta_t) on the K and V rows ----------------
@@ -482,6 +488,7 @@ wide_gram_pair_kernel(const WideParams p, const __grid_constant__ CUtensorMap ma
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
+            PhaseLog armed;     // loads in flight are waited for after an abort
             for (int item = cid; item < nitems && ok; item += ncl) {
                 const int frame = global_frame(p, item);
                 for (int t = 0; t < nt; ++t) {
@@ -494,9 +501,11 @@ wide_gram_pair_kernel(const WideParams p, const __grid_constant__ CUtensorMap ma
                         tma_load_3d(st + kPairTile + b * kBoxG, &mapV, &full[s], x, t * kTokG,
                                     frame, pol);
                     }
+                    armed.note(s, ph);
                     if (++s == kPairStages) { s = 0; ph ^= 1; }
                 }
             }
+            armed.drain_if_aborted(full, kPairStages, ab);
         }
     } else if (warp == 1) {
         if (lane == 0 && rank == 0) {
@@ -509,6 +518,7 @@ wide_gram_pair_kernel(const WideParams p, const __grid_constant__ CUtensorMap ma
             int s = 0, li = 0;
             uint32_t ph = 0;
             bool ok = true;
+            PhaseLog armed;     // MMAs in flight are waited for after an abort
             for (int item = cid; item < nitems && ok; item += ncl, ++li) {
                 if (!(ok = mbar_wait(accempty, (li & 1) ^ 1, ab, 0x612, true))) break;
                 tc_fence_after();
@@ -534,6 +544,7 @@ wide_gram_pair_kernel(const WideParams p, const __grid_constant__ CUtensorMap ma
                     }
                     mma_commit_pair(&empty[s], 0);
                     mma_commit_pair(&empty[s], 1);
+                    armed.note(s, ph);
                     if (++s == kPairStages) { s = 0; ph ^= 1; }
                 }
                 if (ok) {
@@ -541,6 +552,7 @@ wide_gram_pair_kernel(const WideParams p, const __grid_constant__ CUtensorMap ma
                     mma_commit_pair(accfull, 1);
                 }
             }
+            armed.drain_if_aborted(empty, kPairStages, ab);
         } else if (lane == 0 && !XF) {
             // ---------------- odd CTA: forward each landed stage ----------------
             int s = 0;
@@ -671,6 +683,7 @@ wide_chain_gdn_kernel(const WideParams p) {
 
     if (warp == 0) {
         if (lane == 0) {
+            PhaseLog armed;     // loads in flight are waited for after an abort
             for (int f = 0; f < F; ++f) {
                 bool ok = true;
                 for (int r = 0; r < 2 && ok; ++r) {
@@ -678,14 +691,17 @@ wide_chain_gdn_kernel(const WideParams p) {
                     mbar_expect_tx(&gfull[r], kGImg);
                     bulk_load(stage + r * kGImg, p.gimg + ((size_t)bh * F + f) * 2 * kGImg + r * kGImg,
                               kGImg, &gfull[r]);
+                    armed.note(r, f & 1);
                 }
                 if (!ok) break;
             }
+            armed.drain_if_aborted(gfull, 2, ab);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             const uint32_t idC = idesc_bf16(128, 128, false, true);
             const uint32_t ib = smem_u32(img);
+            PhaseLog armed;     // MMAs in flight are waited for after an abort
             for (int f = 0; f < F; ++f) {
                 if (!mbar_wait(mready, f & 1, ab, 0x702)) break;
                 bool ok = true;
@@ -699,10 +715,12 @@ wide_chain_gdn_kernel(const WideParams p) {
                         mma_bf16(tM + r * 128, ad, bd, idC, 1u);
                     }
                     mma_commit(&gempty[r]);
+                    armed.note(r, f & 1);
                 }
                 if (!ok) break;
                 mma_commit(mdone);
             }
+            armed.drain_if_aborted(gempty, 2, ab);
         }
     } else if (warp < 10) {
         // ---------------- epilogue ----------------
@@ -953,6 +971,7 @@ wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
             int s = 0, li = 0;
             uint32_t ph = 0;
             bool ok = true;
+            PhaseLog armed_q, armed_m;     // loads in flight are waited for after an abort
             for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
                 const int frame = global_frame(p, item);
                 const int nq = nt * nbx;                   // Q boxes of the item
@@ -961,6 +980,7 @@ wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
                     mbar_expect_tx(&qfull[s], kBoxO);
                     tma_load_3d(qring + s * kBoxO, &mapQ, &qfull[s], 64 * (g % nbx),
                                 (g / nbx) * kTokO, frame, pol);
+                    armed_q.note(s, ph);
                     if (++s == kQS) { s = 0; ph ^= 1; }
                 };
                 const int early = min(nq, kQS);
@@ -971,8 +991,11 @@ wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
                 mbar_expect_tx(mfull, 2 * kMImg + (RELU ? 1024 : 0));
                 bulk_load(mbuf, p.mimg + (size_t)item * 2 * kMImg, 2 * kMImg, mfull);
                 if (RELU) bulk_load(zbuf, p.zf + (size_t)item * 256, 1024, mfull);
+                armed_m.note(0, li & 1);
                 for (int g = early; g < nq; ++g) load_q(g);
             }
+            armed_q.drain_if_aborted(qfull, kQS, ab);
+            armed_m.drain_if_aborted(mfull, 1, ab);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -981,6 +1004,7 @@ wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
             int s = 0, li = 0, gt = 0;
             uint32_t ph = 0;
             bool ok = true;
+            PhaseLog armed;     // MMAs in flight are waited for after an abort
             for (int item = blockIdx.x; item < nitems && ok; item += gridDim.x, ++li) {
                 if (!(ok = mbar_wait(mfull, li & 1, ab, 0x803))) break;
                 tc_fence_after();
@@ -999,12 +1023,14 @@ wide_output_kernel(const WideParams p, const __grid_constant__ CUtensorMap mapQ,
                             mma_bf16(tbase + a * 256, ad, bd, idO, (b | kk) ? 1u : 0u);
                         }
                         mma_commit(&qempty[s]);
+                        armed.note(s, ph);
                         if (++s == kQS) { s = 0; ph ^= 1; }
                     }
                     if (ok) mma_commit(&accfull[a]);
                 }
                 if (ok) mma_commit(mempty);
             }
+            armed.drain_if_aborted(qempty, kQS, ab);
         }
     } else if (warp < 6) {
         // ---------------- epilogue: TMEM -> bf16 -> TMA store ----------------
