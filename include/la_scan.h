@@ -42,13 +42,16 @@
  *              la_query_device_status reports.
  * Streams.     Wide heads (bf16, D > 128) and the three-kernel path on
  *              clips of 32 or more frames pipeline frame chunks over two
- *              streams of the library's own, forked from `stream` (after the
- *              work already queued on it) and joined back to it, so the call
- *              is still ordered on `stream` as a whole (and can be captured
- *              into a CUDA graph).  The first such call on a device creates
- *              those streams and a few events and keeps them until the
- *              process exits; calls on one device serialise their
- *              enqueueing on a lock.
+ *              streams of the library's own; one-chunk three-kernel calls
+ *              with many heads run two head groups, each group's chain and
+ *              output on a further stream of the library's own.  These
+ *              streams are forked from `stream` (after the work already
+ *              queued on it) and joined back to it, so the call is still
+ *              ordered on `stream` as a whole (and can be captured into a
+ *              CUDA graph).  The first such call on a device creates those
+ *              streams and a few events and keeps them until the process
+ *              exits; calls on one device serialise their enqueueing on a
+ *              lock.
  * Aliasing.    state_in == state_out (and z_in == z_out) is allowed (in
  *              place).  o must not overlap q, k or v.
  * NULL state.  state_in == NULL (z_in == NULL) means a zero initial state;
@@ -457,8 +460,9 @@ LA_API la_status la_query_device_status(void* workspace, cudaStream_t stream);
  * kernels one call launches in *kernels (if not NULL) and returns the name
  * of the kernel path: "tcgen05_fused" (bf16, 64 <= D <= 128, few heads: one
  * persistent kernel), "tcgen05" (bf16, 64 <= D <= 128, many heads: three
- * kernels), "tcgen05_wide" (bf16, 128 < D <= 256: three kernels per frame
- * chunk) or "simt_f32" (float32 inputs, D < 64); NULL for an unsupported
+ * kernels per frame chunk or head group), "tcgen05_wide" (bf16,
+ * 128 < D <= 256: three kernels per frame chunk) or "simt_f32" (float32
+ * inputs, D < 64); NULL for an unsupported
  * shape.  No counterpart in the pages: it lets a caller check which
  * kernels its calls use. */
 LA_API const char* la_plan(la_mode mode, la_dtype dt, int B, int H, int F, int S, int D,
